@@ -1,0 +1,203 @@
+"""ctypes wrapper of the float64 CPU oracle (``oracle/hils_oracle.c``).
+
+TEST INFRASTRUCTURE: imported only by the tests, the smoke check and the CPU
+baseline leg of the benchmark.  The product library never imports it.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hils_oracle.c")
+_LIB = os.path.join(_HERE, "_build", "libhils_oracle.so")
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I = ctypes.POINTER(ctypes.c_int)
+
+
+def build(force=False):
+    """Compile the oracle with gcc (IEEE float64: no fast-math, no contraction)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    os.makedirs(os.path.dirname(_LIB), exist_ok=True)
+    tmp = _LIB + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-fopenmp", "-ffp-contract=off", "-fPIC",
+                           "-shared", "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        L = _lib
+        L.hils_oracle_set_mutant.argtypes = [ctypes.c_int]
+        L.hils_oracle_group_scores.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, _D, _D]
+        L.hils_oracle_topk.argtypes = [ctypes.c_int, ctypes.c_int, _D, _I]
+        L.hils_oracle_topk.restype = ctypes.c_int
+        L.hils_oracle_select.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_long,
+                                         ctypes.c_double, _D, _D, _I, _D]
+        L.hils_oracle_attend.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_long,
+                                         ctypes.c_double, _D, _I, _D, _D, _D, _D, _D, _D, _D]
+        L.hils_oracle_tie_alternatives.argtypes = [ctypes.c_int, ctypes.c_int, _D, ctypes.c_double, ctypes.c_int, _I]
+        L.hils_oracle_tie_alternatives.restype = ctypes.c_int
+        L.hils_oracle_forward.argtypes = [ctypes.c_int] * 8 + [ctypes.c_long, ctypes.c_double, _D, _D, _D, _D,
+                                                               _D, _I, _D, _D, ctypes.c_int]
+        L.hils_oracle_forward.restype = ctypes.c_int
+        L.hils_oracle_max_threads.restype = ctypes.c_int
+    return _lib
+
+
+def _dp(a):
+    return a.ctypes.data_as(_D) if a is not None else None
+
+
+def _ip(a):
+    return a.ctypes.data_as(_I) if a is not None else None
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def set_mutant(m):
+    lib().hils_oracle_set_mutant(int(m))
+
+
+def max_threads():
+    return lib().hils_oracle_max_threads()
+
+
+def default_scale(d):
+    return 1.0 / np.sqrt(d)
+
+
+def forward(Q, K, V, L, C, k, q_offset=0, scale=None, nthreads=None):
+    """Whole forward pass.  Q [B,H,N,d], K/V [B,Hkv,T,d], L [B,Hkv,ceil(T/C),d] (float64).
+
+    Returns dict with O [B,H,N,d], sel [B,Hkv,N,k+1], s and w [B,H,N,k+1].
+    """
+    Q, K, V, L = _f64(Q), _f64(K), _f64(V), _f64(L)
+    B, H, N, d = Q.shape
+    _, Hkv, T, _ = K.shape
+    assert L.shape == (B, Hkv, -(-T // C), d), L.shape
+    scale = default_scale(d) if scale is None else scale
+    O = np.zeros((B, H, N, d))
+    sel = np.zeros((B, Hkv, N, k + 1), dtype=np.int32)
+    s = np.zeros((B, H, N, k + 1))
+    w = np.zeros((B, H, N, k + 1))
+    nthreads = max_threads() if nthreads is None else nthreads
+    rc = lib().hils_oracle_forward(B, H, Hkv, N, T, d, C, k, q_offset, scale, _dp(Q), _dp(K), _dp(V), _dp(L),
+                                   _dp(O), _ip(sel), _dp(s), _dp(w), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the shapes")
+    return {"O": O, "sel": sel, "s": s, "w": w}
+
+
+def group_scores(q, Lrows, scale):
+    q, Lrows = _f64(q), _f64(Lrows)
+    G, d = q.shape
+    out = np.zeros(Lrows.shape[0])
+    lib().hils_oracle_group_scores(G, d, Lrows.shape[0], scale, _dp(q), _dp(Lrows), _dp(out))
+    return out
+
+
+def topk(shat, n_past, k):
+    shat = _f64(shat)
+    sel = np.zeros(max(k, 1), dtype=np.int32)
+    lib().hils_oracle_topk(n_past, k, _dp(shat), _ip(sel))
+    return sel[:k]
+
+
+def select(q, Lrows, C, k, pos, scale):
+    """q [G,d]; Lrows [>= pos//C + 1, d] landmarks from chunk 0.  Returns (sel[k+1], shat[c_i+1])."""
+    q = _f64(q)
+    G, d = q.shape
+    ci = pos // C
+    Lrows = _f64(Lrows[:ci + 1])
+    sel = np.zeros(k + 1, dtype=np.int32)
+    shat = np.zeros(ci + 1)
+    lib().hils_oracle_select(G, d, C, k, pos, scale, _dp(q), _dp(Lrows), _ip(sel), _dp(shat))
+    return sel, shat
+
+
+def attend(q, sel, Lsel, Ksel, Vsel, C, pos, scale, want_chunks=False):
+    """q [G,d]; sel [k+1]; Lsel [k+1,d]; Ksel/Vsel [k+1,C,d].  Returns dict s, w [G,k+1], o [G,d] (+ oc)."""
+    q = _f64(q)
+    G, d = q.shape
+    ns = len(sel)
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    Lsel, Ksel, Vsel = _f64(Lsel), _f64(Ksel), _f64(Vsel)
+    assert Ksel.shape == (ns, C, d) and Vsel.shape == (ns, C, d) and Lsel.shape == (ns, d)
+    s = np.zeros((G, ns))
+    w = np.zeros((G, ns))
+    o = np.zeros((G, d))
+    oc = np.zeros((G, ns, d)) if want_chunks else None
+    lib().hils_oracle_attend(G, d, C, ns - 1, pos, scale, _dp(q), _ip(sel), _dp(Lsel), _dp(Ksel), _dp(Vsel),
+                             _dp(s), _dp(w), _dp(o), _dp(oc))
+    out = {"s": s, "w": w, "o": o}
+    if want_chunks:
+        out["oc"] = oc
+    return out
+
+
+def tie_alternatives(shat, n_past, k, eps, max_alts=64):
+    """Alternative top-k selections within the near-tie band (first = primary); None if too many."""
+    shat = _f64(shat)
+    alts = np.zeros((max_alts, max(k, 1)), dtype=np.int32)
+    n = lib().hils_oracle_tie_alternatives(n_past, k, _dp(shat), eps, max_alts, _ip(alts))
+    if n < 0:
+        return None
+    return [alts[a, :k].copy() for a in range(n)]
+
+
+# ---------------------------------------------------------------------------
+# Sampled evaluation on a synthetic workload: rebuilds only the rows it needs.
+
+def sample_query(w, b, g, i, eps=1e-3, max_alts=16):
+    """Oracle answer for query group (b, g, i) of workload w (a synth Workload).
+
+    Returns dict: pos, shat (group scores of chunks 0..c_i), alts (list of
+    (sel[k+1], s[G,k+1], w[G,k+1], o[G,d])) with the primary selection first,
+    or alts=None when the near-tie band is too large to enumerate.
+    """
+    from synth import workloads as W
+    pos = w.q_offset + i
+    ci = pos // w.C
+    scale = default_scale(w.d)
+    heads = np.arange(g * w.G, (g + 1) * w.G)
+    q, _ = W.q_rows(w, b, heads, np.array([i]))
+    q = q[:, 0, :]
+    Lrows, _ = W.l_rows(w, b, g, 0, ci + 1)
+    sel, shat = select(q, Lrows, w.C, w.k, pos, scale)
+    alts = tie_alternatives(shat, ci, w.k, eps, max_alts)
+    res = {"pos": pos, "shat": shat, "alts": None}
+    if alts is None:
+        alts = [sel[:w.k]]
+    out = []
+    kv_cache = {}
+    for a in alts:
+        full = np.concatenate([a, [ci]]).astype(np.int32)
+        Ls = np.zeros((w.k + 1, w.d))
+        Ks = np.zeros((w.k + 1, w.C, w.d))
+        Vs = np.zeros((w.k + 1, w.C, w.d))
+        for j, c in enumerate(full):
+            if c < 0:
+                continue
+            c = int(c)
+            if c not in kv_cache:
+                t0, t1 = c * w.C, min((c + 1) * w.C, w.T)
+                kv_cache[c] = (W.k_rows(w, b, g, t0, t1)[0], W.v_rows(w, b, g, t0, t1)[0])
+            kk, vv = kv_cache[c]
+            Ls[j] = Lrows[c]
+            Ks[j, :kk.shape[0]] = kk
+            Vs[j, :vv.shape[0]] = vv
+        r = attend(q, full, Ls, Ks, Vs, w.C, pos, scale)
+        out.append((full, r["s"], r["w"], r["o"]))
+    res["alts"] = out
+    res["ambiguous_overflow"] = tie_alternatives(shat, ci, w.k, eps, max_alts) is None
+    return res
