@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of the HiLS attention forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl hils|reference]
+
+One step = one pass of the whole path (landmark scoring + top-k selection, then
+chunk attention + fusion) over the workload's synthetic inputs, which are
+resident in HBM.  Default workload: prefill at training length, bf16 GQA
+(B=4, H=32, Hkv=8, N=8192, d=128, C=64, k=16).  Under torchrun every rank runs
+its own copy of the workload (the path has no exchange step: replicas, weak
+scaling); the device time is the maximum over ranks.  Rank 0 prints one JSON
+line.  ``--impl reference`` times the float64 CPU oracle instead, on bounded
+samples of the same workload.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HiLS fwd tokens/s (prefill) & decode KV GB/s at 1 B200; % of tensor/HBM roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_8k")
+    ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-blocks", type=int, default=16, help="64-query blocks in the oracle sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per step
+
+def attention_flops(w):
+    """Nominal attention FLOPs: 4*N*(k+1)*C*d per head (QK^T and PV over k+1 chunks)."""
+    return 4.0 * w.N * (w.k + 1) * w.C * w.d * w.B * w.H
+
+
+def scoring_flops(w):
+    """Group scores over the visible chunks (2d per query group and chunk) + per-head slot scores."""
+    vis = sum((w.q_offset + i) // w.C for i in range(w.N))
+    return 2.0 * w.d * vis * w.B * w.Hkv + 2.0 * w.d * (w.k + 1) * w.N * w.B * w.H
+
+
+def decode_bytes(w):
+    """Landmarks of the past chunks + keys and values of the k+1 selected chunks, per step (N == 1)."""
+    es = 2 if w.dtype == "bf16" else 4
+    ci = w.q_offset // w.C
+    return es * w.B * w.Hkv * w.d * (ci + (min(w.k, ci) + 1) * 2 * w.C)
+
+
+def landmark_bytes(w):
+    es = 2 if w.dtype == "bf16" else 4
+    return es * w.B * w.Hkv * w.d * (w.q_offset // w.C)
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        self.proc.wait()
+        self.file.flush()
+        rows = [l.split(", ") for l in open(self.file.name) if l.strip()]
+        os.unlink(self.file.name)
+        sm = []
+        smax = None
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                s, mx, pw = float(r[1]), float(r[2]), float(r[3])
+            except (ValueError, IndexError):
+                continue
+            smax = mx
+            if pw > 250.0:         # under load
+                sm.append(s)
+                for n, v in zip(names, r[5:9]):
+                    if v.strip() == "Active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples_under_load": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+
+def dist_setup(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allmax(ws, vals):
+    import torch
+    t = torch.tensor(vals, dtype=torch.float64, device="cuda")
+    if ws > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def cpu_baseline(w, n_blocks, block=64, seed=5):
+    """The float64 oracle on a bounded sample: n_blocks blocks of `block` consecutive queries of batch 0.
+
+    Returns (value in the workload's unit, cores, description)."""
+    import numpy as np
+    from oracle import oracle as orc
+    from synth import workloads as W
+    cores = orc.max_threads()
+    rng = np.random.default_rng(seed)
+    if w.N == 1:
+        # decode: a bounded number of (b, g) query groups, every one a full decode of its sequence
+        n_groups = min(w.B * w.Hkv, n_blocks)
+        items = [(b, g) for b in range(w.B) for g in range(w.Hkv)][:n_groups]
+        t = 0.0
+        ci = w.q_offset // w.C
+        for (b, g) in items:
+            Lr, _ = W.l_rows(w, b, g, 0, ci + 1)
+            q, _ = W.q_rows(w, b, np.arange(g * w.G, (g + 1) * w.G), np.array([0]))
+            sel_c = None
+            t0 = time.perf_counter()
+            sel, _ = orc.select(q[:, 0], Lr, w.C, w.k, w.q_offset, orc.default_scale(w.d))
+            t += time.perf_counter() - t0
+            sel_c = [int(c) for c in sel if c >= 0]
+            Ls = np.zeros((w.k + 1, w.d))
+            Ks = np.zeros((w.k + 1, w.C, w.d))
+            Vs = np.zeros((w.k + 1, w.C, w.d))
+            for j, c in enumerate(sel):
+                if c < 0:
+                    continue
+                t0_, t1_ = c * w.C, min((c + 1) * w.C, w.T)
+                Ks[j, :t1_ - t0_] = W.k_rows(w, b, g, t0_, t1_)[0]
+                Vs[j, :t1_ - t0_] = W.v_rows(w, b, g, t0_, t1_)[0]
+                Ls[j] = Lr[c]
+            t0 = time.perf_counter()
+            orc.attend(q[:, 0], sel, Ls, Ks, Vs, w.C, w.q_offset, orc.default_scale(w.d))
+            t += time.perf_counter() - t0
+        per_group_bytes = decode_bytes(w) / (w.B * w.Hkv)
+        return (per_group_bytes * len(items) / t / 1e9, 1,
+                "%d of %d decode query groups (b, kv-head), one thread each, host input generation untimed"
+                % (len(items), w.B * w.Hkv))
+    b = 0
+    K = np.stack([W.k_rows(w, b, g, 0, w.T)[0] for g in range(w.Hkv)])[None]
+    V = np.stack([W.v_rows(w, b, g, 0, w.T)[0] for g in range(w.Hkv)])[None]
+    L = np.stack([W.l_rows(w, b, g, 0, w.nL)[0] for g in range(w.Hkv)])[None]
+    starts = sorted(set(int(x) for x in rng.integers(0, (w.N - block) // block + 1, size=n_blocks) * block))
+    t = 0.0
+    ntok = 0
+    for i0 in starts:
+        Qb, _ = W.q_rows(w, b, np.arange(w.H), np.arange(i0, i0 + block))
+        t0 = time.perf_counter()
+        orc.forward(Qb[None], K, V, L, w.C, w.k, q_offset=w.q_offset + i0, nthreads=cores)
+        t += time.perf_counter() - t0
+        ntok += block
+    return (ntok / t, cores, "%d blocks of %d consecutive queries (all %d heads) of batch 0 at random offsets; "
+            "OpenMP over query groups; host input generation untimed" % (len(starts), block, w.H))
+
+
+def run_reference(args, w):
+    ws, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    unit = "tokens/s" if w.N > 1 else "GB/s"
+    vals = []
+    for s in range(args.warmup + args.steps):
+        v, cores, desc = cpu_baseline(w, n_blocks=2, seed=100 + s)
+        if s >= args.warmup:
+            vals.append(v)
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def config_of(w, n):
+    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "T": w.T, "d": w.d, "C": w.C,
+            "k": w.k, "q_offset": w.q_offset, "dtype_in": w.dtype, "dtype_out": w.dtype,
+            "parallelism": "replicas x%d (no exchange step)" % n,
+            "l2": "inputs larger than L2 (no flush)" if (w.B * w.H * w.N * w.d * 2 > 126e6 or
+                                                         w.B * w.Hkv * w.T * w.d * 4 > 126e6) else "L2 flushed"}
+
+
+def run_hils(args, w):
+    import torch
+    import chunk_wise_hierarchical_hils_b200 as hils
+    from synth import gpu as synth_gpu
+
+    ws, rank, local = dist_setup(args)
+    dev = synth_gpu.alloc_inputs(w)
+    dt = {"f32": hils.HILS_F32, "bf16": hils.HILS_BF16}[w.dtype]
+    p = hils.problem(w.B, w.H, w.Hkv, w.N, w.T, w.d, w.C, w.k, w.q_offset, dt, dt)
+    tdt = dev["Q"].dtype
+    O = torch.empty((w.B, w.H, w.N, w.d), dtype=tdt, device="cuda")
+    sel_idx = torch.empty((w.B, w.Hkv, w.N, max(w.k, 1)), dtype=torch.int32, device="cuda")
+    sel_score = torch.empty((w.B, w.H, w.N, w.k + 1), dtype=torch.float32, device="cuda")
+    ws_sel = torch.empty(max(hils.hils_score_select_workspace_size(p), 16), dtype=torch.uint8, device="cuda")
+    ws_att = torch.empty(max(hils.hils_chunk_attend_fuse_workspace_size(p), 16), dtype=torch.uint8, device="cuda")
+    ws_fwd = torch.empty(hils.hils_forward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        hils.hils_score_select(p, dev["Q"], dev["L"], sel_idx, sel_score, ws_sel, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        hils.hils_chunk_attend_fuse(p, dev["Q"], dev["K"], dev["V"], sel_idx, sel_score, O, ws_att, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hils.hils_sync_status(stream) != hils.HILS_OK:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(ws)
+    torch.cuda.synchronize()
+    sampler.start()
+    start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(end)
+    k1 = [e[0].elapsed_time(e[1]) for e in evs]
+    k2 = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms, k1_avg, k2_avg = allmax(ws, [total_ms, statistics.mean(k1), statistics.mean(k2)])
+    ms_step = total_ms / args.steps
+
+    # end to end through the public call with host buffers
+    pin = {k: v.cpu().pin_memory() for k, v in dev.items()}
+    Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = Oh.numel() * Oh.element_size()
+
+    def e2e_step():
+        for k in dev:
+            dev[k].copy_(pin[k], non_blocking=True)
+        hils.hils_forward(p, dev["Q"], dev["K"], dev["V"], dev["L"], O, ws_fwd, stream)
+        Oh.copy_(O, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allmax(ws, [e0.elapsed_time(e1) / args.e2e_steps])[0]
+    if hils.hils_sync_status(stream) != hils.HILS_OK:
+        raise RuntimeError("device-side timeout")
+
+    pk, pk_kind = peaks()
+    if w.N > 1:
+        unit = "tokens/s"
+        per_step_units = w.B * w.N
+        fl = attention_flops(w)
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        if w.dtype == "f32":
+            peak = peak / 2.0   # tf32 nominal ratio to bf16 (1.1 vs 2.25 PFLOP/s dense)
+        achieved = fl / (k2_avg * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "chunk_attend_fuse (prefill)", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_kind": pk_kind + " bf16 sustained", "algorithmic_flops_per_launch": fl,
+                "launch_ms": k2_avg, "select_ms": k1_avg}
+    else:
+        unit = "GB/s"
+        per_step_units = decode_bytes(w) / 1e9
+        lb = landmark_bytes(w)
+        achieved = lb / (k1_avg * 1e-3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"bound": "hbm", "kernel": "score_select (decode landmark scan)", "achieved": achieved,
+                "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                "peak_kind": pk_kind + " copy", "algorithmic_bytes_per_launch": lb, "launch_ms": k1_avg,
+                "attend_ms": k2_avg}
+    value = ws * per_step_units / (ms_step * 1e-3)
+    e2e_value = ws * per_step_units / (e2e_ms * 1e-3)
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded Philox4x32-10 inputs)",
+            "config": config_of(w, ws), "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "steps": args.e2e_steps},
+            "gpu_launches": 2 * args.steps, "clocks": clocks}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, cores, desc = cpu_baseline(w, args.cpu_blocks)
+        line["cpu_baseline"] = {"value": v, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    from synth.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_hils(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,245 @@
+// api.cu -- the C ABI of libhils.so: validation, workspace sizing, dispatch.
+#include <math.h>
+#include <mutex>
+
+#include "internal.h"
+
+namespace hils {
+
+namespace {
+
+__device__ unsigned int g_status;   // device-side status word (one per device)
+
+constexpr long long kDefaultWaitLimit = 1ll << 24;   // polls; roughly a second of spinning
+long long g_wait_limit = kDefaultWaitLimit;
+std::mutex g_mu;
+
+hils_status device_ctl(DeviceCtl *ctl)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HILS_ERR_CUDA;
+    static unsigned int *addr[64] = {nullptr};
+    if (dev < 0 || dev >= 64) return HILS_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!addr[dev]) {
+        void *a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_status) != cudaSuccess) return HILS_ERR_CUDA;
+        addr[dev] = static_cast<unsigned int *>(a);
+    }
+    ctl->status = addr[dev];
+    ctl->wait_limit = g_wait_limit;
+    return HILS_OK;
+}
+
+bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+hils_status resolve(const hils_problem *p, Dims *o)
+{
+    if (!p) return HILS_ERR_INVALID_ARG;
+    if (p->B < 1 || p->H < 1 || p->Hkv < 1 || p->N < 1 || p->T < 1 || p->d < 1 || p->C < 1 || p->k < 0)
+        return HILS_ERR_INVALID_ARG;
+    if (p->H % p->Hkv) return HILS_ERR_INVALID_ARG;
+    if (p->q_offset < 0 || (long long)p->q_offset + p->N > p->T) return HILS_ERR_INVALID_ARG;
+    if ((p->in_dtype != HILS_F32 && p->in_dtype != HILS_BF16) ||
+        (p->out_dtype != HILS_F32 && p->out_dtype != HILS_BF16))
+        return HILS_ERR_INVALID_ARG;
+    if (!(p->scale >= 0.f) || isinf(p->scale)) return HILS_ERR_INVALID_ARG;
+    if (p->d != 64 && p->d != 128) return HILS_ERR_UNSUPPORTED;
+    if (p->C != 32 && p->C != 64 && p->C != 128) return HILS_ERR_UNSUPPORTED;
+    if (p->k > HILS_MAX_K) return HILS_ERR_UNSUPPORTED;
+    const int G = p->H / p->Hkv;
+    if (G > HILS_MAX_GROUP) return HILS_ERR_UNSUPPORTED;
+    if ((long long)p->B * p->Hkv > 65535 || p->B > 65535) return HILS_ERR_UNSUPPORTED;
+    o->B = p->B; o->H = p->H; o->Hkv = p->Hkv; o->G = G;
+    o->N = p->N; o->T = p->T; o->d = p->d; o->C = p->C; o->k = p->k;
+    o->nL = (p->T + p->C - 1) / p->C;
+    o->q_offset = p->q_offset;
+    o->scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+    if (o->N == 1) {
+        const DecodePlan plan = decode_plan(*o);
+        if ((size_t)plan.sort_n * 8 + (size_t)o->d * 4 > 200 * 1024) return HILS_ERR_UNSUPPORTED;
+    }
+    return HILS_OK;
+}
+
+size_t sel_idx_bytes(const Dims &p) { return align_up((size_t)p.B * p.Hkv * p.N * p.k * sizeof(int32_t), 256); }
+size_t sel_score_bytes(const Dims &p) { return align_up((size_t)p.B * p.H * p.N * (p.k + 1) * sizeof(float), 256); }
+size_t select_ws(const Dims &p) { return p.N == 1 ? decode_select_ws_bytes(p) : 0; }
+size_t attend_ws(const Dims &p) { return p.N == 1 ? decode_attend_ws_bytes(p) : 0; }
+
+hils_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA; }
+
+hils_status check_ws(void *ws, size_t have, size_t need)
+{
+    if (need == 0) return HILS_OK;
+    if (!ws || have < need) return HILS_ERR_WORKSPACE;
+    if (!aligned16(ws)) return HILS_ERR_INVALID_ARG;
+    return HILS_OK;
+}
+
+hils_status do_select(const Dims &p, hils_dtype in, const void *Q, const void *L, int32_t *sel_idx,
+                      float *sel_score, void *ws, cudaStream_t s)
+{
+    if (p.N == 1) return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, s));
+    return from_cuda(launch_select_prefill(p, in, Q, L, sel_idx, sel_score, s));
+}
+
+hils_status do_attend(const Dims &p, hils_dtype in, hils_dtype out, const void *Q, const void *K,
+                      const void *V, const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
+                      cudaStream_t s)
+{
+    if (p.N == 1) return from_cuda(launch_attend_decode(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, s));
+    DeviceCtl ctl;
+    hils_status st = device_ctl(&ctl);
+    if (st != HILS_OK) return st;
+    return from_cuda(launch_attend_prefill(p, in, out, Q, K, V, sel_idx, sel_score, O, ctl, s));
+}
+
+}  // namespace
+
+// Prefill dispatch: the tensor-core kernel when it covers the shape, else CUDA cores.
+cudaError_t launch_attend_prefill(const Dims &p, hils_dtype in, hils_dtype out, const void *Q, const void *K,
+                                  const void *V, const int32_t *sel_idx, const float *sel_score, void *O,
+                                  const DeviceCtl &ctl, cudaStream_t s)
+{
+    (void)ctl;
+    return launch_attend_prefill_simt(p, in, out, Q, K, V, sel_idx, sel_score, O, s);
+}
+
+}  // namespace hils
+
+using namespace hils;
+
+extern "C" {
+
+const char *hils_status_string(int status)
+{
+    switch (status) {
+    case HILS_OK: return "HILS_OK";
+    case HILS_ERR_INVALID_ARG: return "HILS_ERR_INVALID_ARG: null or misaligned pointer, or invalid shape";
+    case HILS_ERR_UNSUPPORTED: return "HILS_ERR_UNSUPPORTED: shape outside the implemented set (d, C, k, group)";
+    case HILS_ERR_CUDA: return "HILS_ERR_CUDA: a CUDA runtime call failed";
+    case HILS_ERR_TIMEOUT: return "HILS_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case HILS_ERR_WORKSPACE: return "HILS_ERR_WORKSPACE: workspace missing or too small";
+    default: return "unknown hils status";
+    }
+}
+
+int hils_version(void) { return HILS_VERSION; }
+
+hils_status hils_validate(const hils_problem *p)
+{
+    Dims d;
+    return resolve(p, &d);
+}
+
+hils_status hils_score_select_workspace_size(const hils_problem *p, size_t *bytes)
+{
+    Dims d;
+    if (!bytes) return HILS_ERR_INVALID_ARG;
+    hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    *bytes = select_ws(d);
+    return HILS_OK;
+}
+
+hils_status hils_chunk_attend_fuse_workspace_size(const hils_problem *p, size_t *bytes)
+{
+    Dims d;
+    if (!bytes) return HILS_ERR_INVALID_ARG;
+    hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    *bytes = attend_ws(d);
+    return HILS_OK;
+}
+
+hils_status hils_forward_workspace_size(const hils_problem *p, size_t *bytes)
+{
+    Dims d;
+    if (!bytes) return HILS_ERR_INVALID_ARG;
+    hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    const size_t scratch = select_ws(d) > attend_ws(d) ? select_ws(d) : attend_ws(d);
+    *bytes = sel_idx_bytes(d) + sel_score_bytes(d) + scratch;
+    return HILS_OK;
+}
+
+hils_status hils_score_select(const hils_problem *p, const void *Q, const void *L, int32_t *sel_idx,
+                              float *sel_score, void *workspace, size_t workspace_bytes, void *stream)
+{
+    Dims d;
+    hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    if (!Q || !L || !sel_score || (d.k > 0 && !sel_idx)) return HILS_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(L) || (sel_idx && !aligned16(sel_idx)) || !aligned16(sel_score))
+        return HILS_ERR_INVALID_ARG;
+    st = check_ws(workspace, workspace_bytes, select_ws(d));
+    if (st != HILS_OK) return st;
+    return do_select(d, p->in_dtype, Q, L, sel_idx, sel_score, workspace, static_cast<cudaStream_t>(stream));
+}
+
+hils_status hils_chunk_attend_fuse(const hils_problem *p, const void *Q, const void *K, const void *V,
+                                   const int32_t *sel_idx, const float *sel_score, void *O, void *workspace,
+                                   size_t workspace_bytes, void *stream)
+{
+    Dims d;
+    hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    if (!Q || !K || !V || !sel_score || !O || (d.k > 0 && !sel_idx)) return HILS_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(sel_score) ||
+        (sel_idx && !aligned16(sel_idx)))
+        return HILS_ERR_INVALID_ARG;
+    st = check_ws(workspace, workspace_bytes, attend_ws(d));
+    if (st != HILS_OK) return st;
+    return do_attend(d, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, workspace,
+                     static_cast<cudaStream_t>(stream));
+}
+
+hils_status hils_forward(const hils_problem *p, const void *Q, const void *K, const void *V, const void *L,
+                         void *O, void *workspace, size_t workspace_bytes, void *stream)
+{
+    Dims d;
+    hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    if (!Q || !K || !V || !L || !O) return HILS_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(L) || !aligned16(O))
+        return HILS_ERR_INVALID_ARG;
+    size_t need = 0;
+    hils_forward_workspace_size(p, &need);
+    st = check_ws(workspace, workspace_bytes, need);
+    if (st != HILS_OK) return st;
+    char *ws = static_cast<char *>(workspace);
+    int32_t *sel_idx = reinterpret_cast<int32_t *>(ws);
+    float *sel_score = reinterpret_cast<float *>(ws + sel_idx_bytes(d));
+    void *scratch = ws + sel_idx_bytes(d) + sel_score_bytes(d);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = do_select(d, p->in_dtype, Q, L, sel_idx, sel_score, scratch, s);
+    if (st != HILS_OK) return st;
+    return do_attend(d, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, scratch, s);
+}
+
+hils_status hils_sync_status(void *stream)
+{
+    DeviceCtl ctl;
+    hils_status st = device_ctl(&ctl);
+    if (st != HILS_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HILS_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpy(&v, ctl.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return HILS_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpy(ctl.status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return HILS_ERR_CUDA;
+        return HILS_ERR_TIMEOUT;
+    }
+    return HILS_OK;
+}
+
+hils_status hils_set_wait_limit(long long polls)
+{
+    if (polls < 0) return HILS_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_wait_limit = polls == 0 ? kDefaultWaitLimit : polls;
+    return HILS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// attend_simt.cuh -- one warp attends one head to one staged chunk (CUDA cores).
+//
+// "Hierarchical Sparse Attention Done Right" (arXiv 2607.02980v1), Abstract and
+// Sec. 3 "Hierarchical softmax": the query attends inside the chunk with a
+// softmax over the chunk's visible tokens only; the normalised chunk output is
+// then weighted by the chunk's fusion weight.
+#pragma once
+
+#include "common.cuh"
+
+namespace hils {
+
+// Copy rows [0, n_rows) of a chunk (row stride D) from global to shared memory
+// with 16-byte vectors, all threads of the block.
+template <typename Tin, int D>
+__device__ __forceinline__ void stage_rows(Tin *dst, const Tin *src, int n_rows)
+{
+    constexpr int VEC = 16 / sizeof(Tin);
+    const int n_vec = n_rows * D / VEC;
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+    for (int e = threadIdx.x; e < n_vec; e += blockDim.x) d[e] = __ldg(s + e);
+}
+
+// logit of key row krow for the scaled query in shared memory; each lane walks
+// the 8-element segments in a lane-rotated order so that lanes reading
+// different rows hit different banks.
+template <typename Tin, int D>
+__device__ __forceinline__ float dot_rotated(const float *qsm, const Tin *krow, int lane)
+{
+    constexpr int NSEG = D / 8;
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+    for (int x = 0; x < NSEG; ++x) {
+        const int seg = (x + lane) & (NSEG - 1);
+        float kv[8], qv[8];
+        lds8(krow + seg * 8, kv);
+        lds8(qsm + seg * 8, qv);
+#pragma unroll
+        for (int u = 0; u < 8; u += 2) {
+            a0 = fmaf(qv[u], kv[u], a0);
+            a1 = fmaf(qv[u + 1], kv[u + 1], a1);
+        }
+    }
+    return a0 + a1;
+}
+
+// acc[x] (element lane + 32 x of the head's output) += coef * o_c, where o_c is
+// the softmax-weighted mean of the staged value rows over the n_vis visible
+// tokens (n_vis <= 128).
+template <typename Tin, int D>
+__device__ __forceinline__ void warp_attend_chunk(const float *qsm, const Tin *Ks, const Tin *Vs, int n_vis,
+                                                  float coef, float *acc)
+{
+    const int lane = threadIdx.x & 31;
+    float lg[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int t = lane + 32 * m;
+        lg[m] = (t < n_vis) ? dot_rotated<Tin, D>(qsm, Ks + (size_t)t * D, lane) : -INFINITY;
+    }
+    const float mx = warp_max(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])));
+    float e[4], sum = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        e[m] = (lane + 32 * m < n_vis) ? expf(lg[m] - mx) : 0.f;
+        sum += e[m];
+    }
+    sum = warp_sum(sum);
+    float oc[D / 32];
+#pragma unroll
+    for (int x = 0; x < D / 32; ++x) oc[x] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        if (32 * m >= n_vis) break;
+#pragma unroll 8
+        for (int tt = 0; tt < 32; ++tt) {
+            const int t = 32 * m + tt;
+            const float pt = __shfl_sync(0xFFFFFFFFu, e[m], tt);
+            if (t < n_vis) {
+                const Tin *vr = Vs + (size_t)t * D;
+#pragma unroll
+                for (int x = 0; x < D / 32; ++x) oc[x] = fmaf(pt, to_float(vr[lane + 32 * x]), oc[x]);
+            }
+        }
+    }
+    const float c = coef / sum;
+#pragma unroll
+    for (int x = 0; x < D / 32; ++x) acc[x] = fmaf(c, oc[x], acc[x]);
+}
+
+// Fusion weights of the slots [j0, j1) for one head: softmax over all ns slot
+// scores (-inf = empty slot).  Warp-cooperative; lane 0.. writes w[j - j0].
+__device__ __forceinline__ void warp_fusion_weights(const float *score_row, int ns, int j0, int j1, float *w)
+{
+    const int lane = threadIdx.x & 31;
+    float mx = -INFINITY;
+    for (int j = lane; j < ns; j += 32) mx = fmaxf(mx, score_row[j]);
+    mx = warp_max(mx);
+    float z = 0.f;
+    for (int j = lane; j < ns; j += 32) {
+        const float s = score_row[j];
+        z += (s == -INFINITY) ? 0.f : expf(s - mx);
+    }
+    z = warp_sum(z);
+    for (int j = j0 + lane; j < j1; j += 32) {
+        const float s = score_row[j];
+        w[j - j0] = (s == -INFINITY) ? 0.f : expf(s - mx) / z;
+    }
+}
+
+}  // namespace hils

@@ -1,0 +1,58 @@
+// internal.h -- resolved problem description and kernel launchers (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/hils.h"
+
+namespace hils {
+
+// Problem with derived quantities, passed by value to every kernel.
+struct Dims {
+    int B, H, Hkv, G;
+    int N, T, d, C, k;
+    int nL;          // landmarks per sequence, ceil(T / C)
+    int q_offset;
+    float scale;     // resolved: never 0
+};
+
+// Device-side status shared by all kernels of the library.
+struct DeviceCtl {
+    unsigned int *status;   // HILS_OK or HILS_ERR_TIMEOUT, sticky until read
+    long long wait_limit;   // polls before a bounded wait gives up
+};
+
+// Decode selection layout in the workspace.
+struct DecodePlan {
+    int spl;        // candidate chunks per split CTA (power of two)
+    int nsplit;     // split CTAs per (b, g)
+    int sort_n;     // power of two >= max(spl, nsplit * k)
+    int slots_per_cta;  // attend: selected chunks per CTA
+    int nsplit2;        // attend: CTAs per (b, g)
+};
+
+DecodePlan decode_plan(const Dims &p);
+size_t decode_select_ws_bytes(const Dims &p);
+size_t decode_attend_ws_bytes(const Dims &p);
+
+// Launchers return the cudaGetLastError() of their launch.
+cudaError_t launch_select_prefill(const Dims &p, hils_dtype in, const void *Q, const void *L,
+                                  int32_t *sel_idx, float *sel_score, cudaStream_t s);
+cudaError_t launch_select_decode(const Dims &p, hils_dtype in, const void *Q, const void *L,
+                                 int32_t *sel_idx, float *sel_score, void *ws, cudaStream_t s);
+cudaError_t launch_attend_prefill(const Dims &p, hils_dtype in, hils_dtype out, const void *Q,
+                                  const void *K, const void *V, const int32_t *sel_idx,
+                                  const float *sel_score, void *O, const DeviceCtl &ctl,
+                                  cudaStream_t s);
+cudaError_t launch_attend_prefill_simt(const Dims &p, hils_dtype in, hils_dtype out, const void *Q,
+                                       const void *K, const void *V, const int32_t *sel_idx,
+                                       const float *sel_score, void *O, cudaStream_t s);
+cudaError_t launch_attend_decode(const Dims &p, hils_dtype in, hils_dtype out, const void *Q,
+                                 const void *K, const void *V, const int32_t *sel_idx,
+                                 const float *sel_score, void *O, void *ws, cudaStream_t s);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace hils

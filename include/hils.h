@@ -1,0 +1,159 @@
+/*
+ * hils.h -- C ABI of the HiLS attention forward library (libhils.so), sm_100a.
+ *
+ * Hierarchical Landmark Sparse (HiLS) attention, as described in
+ * "Hierarchical Sparse Attention Done Right: Toward Infinite Context Modeling"
+ * (arXiv 2607.02980v1, summary page):
+ *   - Abstract: each query attends independently inside every retrieved chunk;
+ *     the per-chunk outputs are fused according to chunk retrieval scores.
+ *   - Sec. 3 Methodology, "Sparse training": each query scores all chunk
+ *     summaries (landmarks) and keeps the top-K chunks.
+ *   - Sec. 3 Methodology, "Hierarchical softmax": softmax inside each chunk,
+ *     then a softmax over the chunks' surrogate masses fuses the chunk outputs.
+ *   - Sec. 4 Practical Design Choices, "Architecture": under GQA the heads of a
+ *     group share one retrieved chunk set, gathered once.
+ *   - Sec. 2 Preliminary: chunks are a uniform partition of the sequence.
+ *
+ * Definition computed (query i at position p = q_offset + i, own chunk
+ * c_i = floor(p / C), head h in kv-group g = h / (H / Hkv), scale s):
+ *   1. retrieval score  s_{h,c} = s * <q_{h,i}, L_{g,c}>;
+ *      group score      S_{g,c} = mean over the group's heads of s_{h,c}.
+ *   2. selection: the min(k, c_i) past chunks c < c_i with the largest group
+ *      scores (equal scores: lower chunk index first), in rank order; the own
+ *      chunk c_i is always added as slot k.
+ *   3. inside each selected chunk: softmax over the tokens c*C .. c*C+C-1 that
+ *      are at positions <= p, of s * <q, k_j>; chunk output o_c = sum p_j v_j.
+ *   4. fusion weights w_{h,c} = softmax over the selected slots of s_{h,c};
+ *      output o_{h,i} = sum_c w_{h,c} o_c.
+ *
+ * Tensor layouts (all row-major, contiguous, device memory, 16-byte aligned):
+ *   Q  [B][H][N][d]        in_dtype
+ *   K  [B][Hkv][T][d]      in_dtype
+ *   V  [B][Hkv][T][d]      in_dtype
+ *   L  [B][Hkv][nL][d]     in_dtype, nL = ceil(T / C), row c = landmark of chunk c
+ *   O  [B][H][N][d]        out_dtype
+ *   sel_idx   [B][Hkv][N][k]   int32: selected past chunks in rank order, -1 padded
+ *   sel_score [B][H][N][k+1]   float: s_{h,c} of each slot (slot k = own chunk),
+ *                              -INFINITY for empty slots
+ * Prefill: q_offset = 0, N = T.  Single-token decode: N = 1, q_offset = T - 1
+ * (the new token's key/value already at position T-1; the landmark of a partial
+ * last chunk is supplied by the caller).  Any 0 <= q_offset, q_offset + N <= T
+ * is accepted.
+ *
+ * Ownership: the caller allocates and owns every buffer, including the
+ * workspace; the library allocates no device memory on these calls.
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ * stream) and validate their arguments before any launch: a status other than
+ * HILS_OK from the call itself means nothing was launched.  Device-side
+ * failures of bounded waits are reported by hils_sync_status().
+ * Thread safety: calls may come from several host threads; kernels that share
+ * one workspace must not overlap on the GPU.
+ */
+#ifndef HILS_H
+#define HILS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HILS_API __attribute__((visibility("default")))
+#else
+#define HILS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HILS_VERSION 100    /* 1.0.0 */
+#define HILS_MAX_K 64       /* largest supported top-k */
+#define HILS_MAX_GROUP 16   /* largest supported H / Hkv */
+
+typedef enum {
+    HILS_OK = 0,
+    HILS_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misaligned pointer */
+    HILS_ERR_UNSUPPORTED = 2,   /* valid but not implemented: d, C, k or group size */
+    HILS_ERR_CUDA = 3,          /* a CUDA runtime call failed */
+    HILS_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up */
+    HILS_ERR_WORKSPACE = 5      /* workspace pointer null or smaller than required */
+} hils_status;
+
+typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
+
+typedef struct {
+    int B, H, Hkv;        /* batch, query heads, key/value heads (H % Hkv == 0) */
+    int N;                /* queries per sequence */
+    int T;                /* keys/values per sequence */
+    int d;                /* head dimension: 64 or 128 */
+    int C;                /* chunk size: 32, 64 or 128 */
+    int k;                /* past chunks retrieved per query: 0..HILS_MAX_K */
+    int q_offset;         /* position of query 0 */
+    hils_dtype in_dtype;  /* Q, K, V, L */
+    hils_dtype out_dtype; /* O */
+    float scale;          /* logit and retrieval-score scale; 0 selects 1/sqrt(d) */
+} hils_problem;
+
+/* Human-readable name of a status code (static string, never NULL). */
+HILS_API const char *hils_status_string(int status);
+
+/* Library version, HILS_VERSION of the build. */
+HILS_API int hils_version(void);
+
+/* Check a problem description without launching anything. */
+HILS_API hils_status hils_validate(const hils_problem *p);
+
+/* Workspace bytes each entry point needs for problem p (may be 0). */
+HILS_API hils_status hils_score_select_workspace_size(const hils_problem *p, size_t *bytes);
+HILS_API hils_status hils_chunk_attend_fuse_workspace_size(const hils_problem *p, size_t *bytes);
+HILS_API hils_status hils_forward_workspace_size(const hils_problem *p, size_t *bytes);
+
+/*
+ * Steps 1-2 plus the per-head slot scores of step 4 (Sec. 3 "Sparse training";
+ * Sec. 4 GQA retrieval).  Reads Q and L; writes sel_idx [B][Hkv][N][k] and
+ * sel_score [B][H][N][k+1].  sel_idx may be NULL only when k == 0.
+ */
+HILS_API hils_status hils_score_select(const hils_problem *p, const void *Q, const void *L,
+                              int32_t *sel_idx, float *sel_score,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Steps 3-4 (Abstract; Sec. 3 "Hierarchical softmax") for a given selection:
+ * gathers the selected chunks' keys and values once per kv-group, attends
+ * inside each, and fuses with softmax(sel_score) per head.  Writes O.
+ * sel_idx entries must be -1 or a past chunk of the query (0 <= c < c_i);
+ * anything else is undefined behaviour checked only by the debug build.
+ */
+HILS_API hils_status hils_chunk_attend_fuse(const hils_problem *p, const void *Q, const void *K,
+                                   const void *V, const int32_t *sel_idx,
+                                   const float *sel_score, void *O,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The whole forward pass (steps 1-4): hils_score_select then
+ * hils_chunk_attend_fuse with the intermediate selection kept in the
+ * workspace.  N = 1 runs the single-token decode kernels.
+ */
+HILS_API hils_status hils_forward(const hils_problem *p, const void *Q, const void *K, const void *V,
+                         const void *L, void *O, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/*
+ * Synchronise `stream` and report device-side status since the last call:
+ * HILS_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the kernel then
+ * skipped its remaining work and released its resources), HILS_ERR_CUDA if
+ * the synchronisation failed, else HILS_OK.  Clears the recorded status.
+ */
+HILS_API hils_status hils_sync_status(void *stream);
+
+/*
+ * Debug/test control of the bounded waits: the number of polls a kernel makes
+ * on a barrier before it records HILS_ERR_TIMEOUT and gives up.  0 restores the
+ * default (about one second).  Affects kernels launched afterwards.
+ */
+HILS_API hils_status hils_set_wait_limit(long long polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HILS_H */

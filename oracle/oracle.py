@@ -156,48 +156,72 @@ def tie_alternatives(shat, n_past, k, eps, max_alts=64):
 
 
 # ---------------------------------------------------------------------------
-# Sampled evaluation on a synthetic workload: rebuilds only the rows it needs.
+# One query group at a time, for sampled comparisons on large inputs.
 
-def sample_query(w, b, g, i, eps=1e-3, max_alts=16):
-    """Oracle answer for query group (b, g, i) of workload w (a synth Workload).
+def evaluate_query(q, Lrows, fetch_kv, C, k, pos, scale, eps=1e-3, max_alts=16):
+    """Oracle answer for one query group.
 
-    Returns dict: pos, shat (group scores of chunks 0..c_i), alts (list of
-    (sel[k+1], s[G,k+1], w[G,k+1], o[G,d])) with the primary selection first,
-    or alts=None when the near-tie band is too large to enumerate.
+    q [G,d]; Lrows [>= c_i+1, d] landmarks from chunk 0; fetch_kv(c) -> (K rows, V rows)
+    of chunk c (at most C rows each).  Returns dict: shat (group scores of chunks
+    0..c_i), overflow (near-tie band too large to enumerate), alts: list of
+    (sel[k+1], s[G,k+1], w[G,k+1], o[G,d]), the primary selection first and then
+    every other selection a near tie (score gap <= eps) would allow.
     """
-    from synth import workloads as W
-    pos = w.q_offset + i
-    ci = pos // w.C
-    scale = default_scale(w.d)
-    heads = np.arange(g * w.G, (g + 1) * w.G)
-    q, _ = W.q_rows(w, b, heads, np.array([i]))
-    q = q[:, 0, :]
-    Lrows, _ = W.l_rows(w, b, g, 0, ci + 1)
-    sel, shat = select(q, Lrows, w.C, w.k, pos, scale)
-    alts = tie_alternatives(shat, ci, w.k, eps, max_alts)
-    res = {"pos": pos, "shat": shat, "alts": None}
-    if alts is None:
-        alts = [sel[:w.k]]
+    q = _f64(q)
+    G, d = q.shape
+    ci = pos // C
+    sel, shat = select(q, Lrows, C, k, pos, scale)
+    alts = tie_alternatives(shat, ci, k, eps, max_alts)
+    overflow = alts is None
+    if overflow:
+        alts = [sel[:k]]
+    cache = {}
     out = []
-    kv_cache = {}
     for a in alts:
         full = np.concatenate([a, [ci]]).astype(np.int32)
-        Ls = np.zeros((w.k + 1, w.d))
-        Ks = np.zeros((w.k + 1, w.C, w.d))
-        Vs = np.zeros((w.k + 1, w.C, w.d))
+        Ls = np.zeros((k + 1, d))
+        Ks = np.zeros((k + 1, C, d))
+        Vs = np.zeros((k + 1, C, d))
         for j, c in enumerate(full):
+            c = int(c)
             if c < 0:
                 continue
-            c = int(c)
-            if c not in kv_cache:
-                t0, t1 = c * w.C, min((c + 1) * w.C, w.T)
-                kv_cache[c] = (W.k_rows(w, b, g, t0, t1)[0], W.v_rows(w, b, g, t0, t1)[0])
-            kk, vv = kv_cache[c]
+            if c not in cache:
+                cache[c] = fetch_kv(c)
+            kk, vv = cache[c]
             Ls[j] = Lrows[c]
             Ks[j, :kk.shape[0]] = kk
             Vs[j, :vv.shape[0]] = vv
-        r = attend(q, full, Ls, Ks, Vs, w.C, pos, scale)
+        r = attend(q, full, Ls, Ks, Vs, C, pos, scale)
         out.append((full, r["s"], r["w"], r["o"]))
-    res["alts"] = out
-    res["ambiguous_overflow"] = tie_alternatives(shat, ci, w.k, eps, max_alts) is None
+    return {"pos": pos, "shat": shat, "alts": out, "overflow": overflow}
+
+
+def sample_queries(w, items, eps=1e-3, max_alts=16):
+    """Oracle answers for query groups items = [(b, g, i), ...] of a synth Workload.
+
+    Inputs are rebuilt from the seeded generator, slice by slice; landmarks are
+    generated once per (b, g).
+    """
+    from synth import workloads as W
+    scale = default_scale(w.d)
+    res = [None] * len(items)
+    by_bg = {}
+    for n, (b, g, i) in enumerate(items):
+        by_bg.setdefault((int(b), int(g)), []).append((n, int(i)))
+    for (b, g), lst in by_bg.items():
+        ci_max = max((w.q_offset + i) // w.C for _, i in lst)
+        Lrows, _ = W.l_rows(w, b, g, 0, ci_max + 1)
+        heads = np.arange(g * w.G, (g + 1) * w.G)
+        kv_cache = {}
+
+        def fetch(c, b=b, g=g, kv_cache=kv_cache):
+            if c not in kv_cache:
+                t0, t1 = c * w.C, min((c + 1) * w.C, w.T)
+                kv_cache[c] = (W.k_rows(w, b, g, t0, t1)[0], W.v_rows(w, b, g, t0, t1)[0])
+            return kv_cache[c]
+
+        qs, _ = W.q_rows(w, b, heads, np.array([i for _, i in lst]))
+        for a, (n, i) in enumerate(lst):
+            res[n] = evaluate_query(qs[:, a, :], Lrows, fetch, w.C, w.k, w.q_offset + i, scale, eps, max_alts)
     return res

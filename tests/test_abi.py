@@ -1,0 +1,96 @@
+"""The C-ABI library loads and exports every symbol include/hils.h declares; host-side validation (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunk_wise_hierarchical_hils_b200 as hils
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "hils.h")).read()
+    return sorted(set(re.findall(r"HILS_API\s+[\w\s\*]+?\b(hils_\w+)\s*\(", src)))
+
+
+def test_header_symbols_exported():
+    names = declared_symbols()
+    assert len(names) >= 11
+    lib = ctypes.CDLL(hils.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(hils.EXPORTS) | set(names)
+    assert hils.hils_version() == 100
+
+
+def test_struct_layout_matches_header():
+    # 11 ints + 1 float, no padding
+    assert ctypes.sizeof(hils.hils_problem) == 12 * 4
+
+
+def prob(**kw):
+    base = dict(B=2, H=8, Hkv=2, N=256, T=256, d=128, C=64, k=4)
+    base.update(kw)
+    return hils.problem(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({}, hils.HILS_OK),
+    ({"H": 6, "Hkv": 4}, hils.HILS_ERR_INVALID_ARG),
+    ({"N": 0}, hils.HILS_ERR_INVALID_ARG),
+    ({"N": 200, "T": 256, "q_offset": 100}, hils.HILS_ERR_INVALID_ARG),
+    ({"N": 1, "T": 256, "q_offset": 255}, hils.HILS_OK),
+    ({"d": 96}, hils.HILS_ERR_UNSUPPORTED),
+    ({"C": 48}, hils.HILS_ERR_UNSUPPORTED),
+    ({"k": 65}, hils.HILS_ERR_UNSUPPORTED),
+    ({"k": -1}, hils.HILS_ERR_INVALID_ARG),
+    ({"H": 64, "Hkv": 2}, hils.HILS_ERR_UNSUPPORTED),
+    ({"scale": float("nan")}, hils.HILS_ERR_INVALID_ARG),
+    ({"scale": -1.0}, hils.HILS_ERR_INVALID_ARG),
+])
+def test_validation(kw, status):
+    assert hils.hils_validate(prob(**kw)) == status
+
+
+def test_bad_dtype():
+    p = prob()
+    p.in_dtype = 7
+    assert hils.hils_validate(p) == hils.HILS_ERR_INVALID_ARG
+
+
+def test_errors_before_launch():
+    """Null pointers, misalignment and short workspaces are rejected on the host."""
+    p = prob(N=1, T=256, q_offset=255)
+    with pytest.raises(hils.HilsError) as e:
+        hils.hils_forward(p, 0, 16, 16, 16, 16, (16, 1 << 30), stream=0)
+    assert e.value.status == hils.HILS_ERR_INVALID_ARG
+    with pytest.raises(hils.HilsError) as e:
+        hils.hils_forward(p, 24, 16, 16, 16, 16, (16, 1 << 30), stream=0)
+    assert e.value.status == hils.HILS_ERR_INVALID_ARG
+    need = hils.hils_forward_workspace_size(p)
+    with pytest.raises(hils.HilsError) as e:
+        hils.hils_forward(p, 16, 16, 16, 16, 16, (16, need - 1), stream=0)
+    assert e.value.status == hils.HILS_ERR_WORKSPACE
+    with pytest.raises(hils.HilsError) as e:
+        hils.hils_score_select(prob(), 16, 16, 0, 16, stream=0)
+    assert e.value.status == hils.HILS_ERR_INVALID_ARG
+
+
+def test_workspace_sizes():
+    p = prob()
+    assert hils.hils_score_select_workspace_size(p) == 0
+    assert hils.hils_forward_workspace_size(p) >= 2 * 2 * 256 * 4 * 4 + 2 * 8 * 256 * 5 * 4
+    pd = prob(B=16, H=32, Hkv=8, N=1, T=131072, k=32, q_offset=131071)
+    assert hils.hils_score_select_workspace_size(pd) > 0
+    assert hils.hils_forward_workspace_size(pd) >= max(hils.hils_score_select_workspace_size(pd),
+                                                       hils.hils_chunk_attend_fuse_workspace_size(pd))
+    with pytest.raises(hils.HilsError):
+        hils.hils_forward_workspace_size(prob(d=80))
+
+
+def test_status_strings():
+    for s in range(6):
+        assert hils.hils_status_string(s).startswith("HILS_")
+    assert "unknown" in hils.hils_status_string(99)

@@ -1,0 +1,99 @@
+"""GPU vs oracle, whole tensors, small shapes that span several tiles and a ragged tail.
+
+Every query group of every case is compared: exact chunk sets (near ties
+within 1e-3 excepted, as enumerated by the oracle), slot scores within 1e-4,
+outputs within 1e-4 (float32 inputs) or 1e-2 (bf16 inputs).
+"""
+import numpy as np
+import pytest
+import torch
+
+import parity
+from synth.workloads import WORKLOADS, Workload
+
+pytestmark = pytest.mark.gpu
+
+
+def wl(name, **kw):
+    base = dict(B=1, H=4, Hkv=2, N=512, T=512, d=128, C=64, k=4, q_offset=0, dtype="bf16", seed=100,
+                l_mode="chunkmean")
+    base.update(kw)
+    return Workload(name, **base)
+
+
+CASES = [
+    WORKLOADS["tiny_f32"],
+    wl("g4_d128_c64_ragged", B=2, H=8, Hkv=2, N=1000, T=1000, k=5, seed=101),
+    wl("g1_d64_c32", H=2, Hkv=2, N=700, T=700, d=64, C=32, k=7, seed=102, l_mode="iid"),
+    wl("g8_d128_c128", H=16, Hkv=2, N=640, T=640, C=128, k=3, seed=103),
+    wl("f32_g2_d128_c64", H=4, Hkv=2, N=300, T=300, k=2, dtype="f32", seed=104),
+    wl("k0_own_chunk_only", N=333, T=333, k=0, seed=105),
+    wl("k16_more_than_visible", N=200, T=200, C=32, k=16, seed=106),
+    wl("chunked_prefill_offset", N=256, T=1024, q_offset=768, k=6, seed=107),
+    wl("g16", H=16, Hkv=1, N=200, T=200, k=3, seed=108),
+    wl("k64_max", H=2, Hkv=1, N=300, T=4200, q_offset=3900, C=32, k=64, seed=109, l_mode="iid"),
+    wl("needles", B=1, H=8, Hkv=2, N=2048, T=2048, k=4, seed=110, l_mode="iid", n_needles=8, needle_period=128),
+]
+DECODE = [
+    wl("decode_ragged_T", B=3, H=8, Hkv=2, N=1, T=1000, q_offset=999, k=4, seed=120),
+    wl("decode_f32_d64", B=2, H=4, Hkv=1, N=1, T=4096 + 17, q_offset=4096 + 16, d=64, C=32, k=8, dtype="f32",
+       seed=121),
+    wl("decode_first_chunk", B=2, H=4, Hkv=2, N=1, T=5, q_offset=4, k=4, seed=122),
+    wl("decode_k0", B=2, H=4, Hkv=2, N=1, T=700, q_offset=699, k=0, seed=123),
+    wl("decode_long_split", B=2, H=8, Hkv=2, N=1, T=64 * 3000 + 5, q_offset=64 * 3000 + 4, k=32, seed=124,
+       l_mode="iid"),
+    wl("decode_k64_c128", B=1, H=16, Hkv=4, N=1, T=128 * 700, q_offset=128 * 700 - 1, C=128, k=64, seed=125,
+       l_mode="iid"),
+]
+
+
+def _check(st):
+    assert st["fail"] == [], st["fail"][:5]
+
+
+@pytest.mark.parametrize("w", CASES + DECODE, ids=lambda w: w.name)
+def test_parity_small(w):
+    st, _ = parity.run_small(w)
+    print(w.name, {k: v for k, v in st.items() if k != "fail"})
+    _check(st)
+
+
+@pytest.mark.parametrize("w", [CASES[1], DECODE[0]], ids=lambda w: w.name)
+def test_bf16_output(w):
+    st, _ = parity.run_small(w, out_dtype="bf16")
+    _check(st)
+
+
+@pytest.mark.parametrize("w", [CASES[1], CASES[4], DECODE[1]], ids=lambda w: w.name)
+def test_stepwise_equals_forward(w):
+    st, (O1, s1, c1) = parity.run_small(w, stepwise=True)
+    _check(st)
+    _, (O2, s2, c2) = parity.run_small(w, stepwise=False)
+    assert torch.equal(O1, O2) and torch.equal(s1, s2) and torch.equal(c1, c2)
+
+
+def test_exact_ties_lowest_index():
+    """Planted exact duplicate landmarks: ties go to the lower chunk index, bit-exactly."""
+    w = wl("ties", B=1, H=4, Hkv=1, N=1024, T=1024, C=32, k=6, seed=130, l_mode="iid")
+    from synth import workloads as W
+    inp = W.full_inputs(w)
+    arr = {k: v[0].copy() for k, v in inp.items()}
+    raw = {k: v[1].copy() for k, v in inp.items()}
+    # landmark of chunk c = level[c % 5] * (mean query direction): five well separated score levels
+    qbar = arr["Q"][0].mean(axis=(0, 1))
+    levels = np.array([0.5, -1.0, 2.0, 0.0, 1.0])
+    from synth.philox import f64_to_f32, f32_to_bf16_bits, bf16_bits_to_f64
+    for c in range(w.nL):
+        bits = f32_to_bf16_bits(f64_to_f32(levels[c % 5] * qbar * 4.0))
+        raw["L"][0, 0, c] = bits
+        arr["L"][0, 0, c] = bf16_bits_to_f64(bits)
+    dev = {k: parity.to_device(v, w.dtype) for k, v in raw.items()}
+    O, sel_idx, sel_score = parity.gpu_run(w, dev)
+    items = parity.all_items(w)
+    sel, s, o = parity.gather_gpu(w, O, sel_idx, sel_score, items)
+    ans = parity.answers_from_arrays(w, arr, items, eps=0.0)
+    for n, a in enumerate(ans):
+        prim = [int(c) for c in a["alts"][0][0][:w.k]]
+        assert [int(c) for c in sel[n]] == prim, (items[n], sel[n], prim)
+    st = parity.compare(w, items, ans, sel, s, o)
+    _check(st)
