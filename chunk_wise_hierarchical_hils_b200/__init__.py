@@ -48,7 +48,7 @@ class HilsError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError("libhils.so is not built (expected at %s); run "
-                          "`python -m chunk_wise_hierarchical_hils_b200.build`" % LIB_PATH)
+                          "`python chunk_wise_hierarchical_hils_b200/build.py`" % LIB_PATH)
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.POINTER(hils_problem)
     vp, sz = ctypes.c_void_p, ctypes.c_size_t

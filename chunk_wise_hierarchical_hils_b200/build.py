@@ -1,6 +1,6 @@
 """Build libhils.so in-tree with nvcc for sm_100a.
 
-    python -m chunk_wise_hierarchical_hils_b200.build [--verbose]
+    python chunk_wise_hierarchical_hils_b200/build.py [--verbose]
 
 Each .cu under csrc/ is compiled to an object in _build/, then all are linked
 into _lib/libhils.so (CUDA runtime linked statically).
