@@ -167,7 +167,7 @@ def cpu_baseline(w, n_blocks, block=64, seed=5):
     rng = np.random.default_rng(seed)
     if w.N == 1:
         # decode: a bounded number of (b, g) query groups, every one a full decode of its sequence
-        n_groups = min(w.B * w.Hkv, n_blocks)
+        n_groups = min(w.B * w.Hkv, max(1, n_blocks // 4))
         items = [(b, g) for b in range(w.B) for g in range(w.Hkv)][:n_groups]
         t = 0.0
         ci = w.q_offset // w.C
@@ -295,13 +295,16 @@ def run_hils(args, w):
     ms_step = total_ms / args.steps
 
     # end to end through the public call with host buffers
-    pin = {k: v.cpu().pin_memory() for k, v in dev.items()}
+    # prefill: every input crosses PCIe each step; decode: only the new query token does (the key/value
+    # and landmark caches are state that stays resident across decode steps)
+    e2e_names = ["Q", "K", "V", "L"] if w.N > 1 else ["Q"]
+    pin = {k: dev[k].cpu().pin_memory() for k in e2e_names}
     Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
     d2h = Oh.numel() * Oh.element_size()
 
     def e2e_step():
-        for k in dev:
+        for k in e2e_names:
             dev[k].copy_(pin[k], non_blocking=True)
         hils.hils_forward(p, dev["Q"], dev["K"], dev["V"], dev["L"], O, ws_fwd, stream)
         Oh.copy_(O, non_blocking=True)
@@ -350,7 +353,7 @@ def run_hils(args, w):
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded Philox4x32-10 inputs)",
             "config": config_of(w, ws), "roofline": roof,
             "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms, "steps": args.e2e_steps},
+                    "ms_per_step": e2e_ms, "steps": args.e2e_steps, "inputs_copied": e2e_names},
             "gpu_launches": 2 * args.steps, "clocks": clocks}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, cores, desc = cpu_baseline(w, args.cpu_blocks)
