@@ -26,7 +26,9 @@ HILS_MAX_GROUP = 16
 
 EXPORTS = ("hils_status_string", "hils_version", "hils_validate", "hils_score_select_workspace_size",
            "hils_chunk_attend_fuse_workspace_size", "hils_forward_workspace_size", "hils_score_select",
-           "hils_chunk_attend_fuse", "hils_forward", "hils_sync_status", "hils_set_wait_limit")
+           "hils_chunk_attend_fuse", "hils_forward", "hils_sync_status", "hils_set_wait_limit",
+           "hils_decode_score_select_noalloc")
+HILS_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
 class hils_problem(ctypes.Structure):
@@ -64,6 +66,7 @@ def _load():
     lib.hils_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hils_sync_status.argtypes = [vp]
     lib.hils_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.hils_decode_score_select_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
     for n in EXPORTS[2:]:
         if n not in ("hils_status_string", "hils_version"):
             getattr(lib, n).restype = ctypes.c_int
@@ -164,6 +167,15 @@ def hils_sync_status(stream=None):
 
 def hils_set_wait_limit(polls):
     _check(_lib.hils_set_wait_limit(int(polls)), "hils_set_wait_limit")
+
+
+def hils_decode_score_select_noalloc(p, Q, L, sel_idx, sel_score, stream=None):
+    """hils_score_select for N == 1 with the library's fixed scratch: no workspace argument.
+
+    For callers that cannot allocate device memory; see include/hils.h."""
+    _check(_lib.hils_decode_score_select_noalloc(ctypes.byref(p), _ptr(Q), _ptr(L), _ptr(sel_idx),
+                                                 _ptr(sel_score), _stream(stream)),
+           "hils_decode_score_select_noalloc")
 
 
 def problem(B, H, Hkv, N, T, d, C, k, q_offset=0, in_dtype=HILS_BF16, out_dtype=None, scale=0.0):

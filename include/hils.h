@@ -152,6 +152,34 @@ HILS_API hils_status hils_sync_status(void *stream);
  */
 HILS_API hils_status hils_set_wait_limit(long long polls);
 
+/*
+ * Allocation-free decode selection.  The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- plugins whose
+ * host application owns the whole device memory budget, memory-capped
+ * processes that cannot reserve a per-call workspace, and latency-critical
+ * paths that must not enter the driver's allocator.
+ *
+ * Same result as hils_score_select for a single-token decode problem (N == 1),
+ * but the kernel's scratch (per-split candidate lists and completion tickets)
+ * comes from a fixed array of HILS_NOALLOC_SCRATCH_BYTES in the library's own
+ * device memory; the caller still passes Q, L, sel_idx and sel_score.  Every
+ * GPU that loads the library holds that array until the process exits.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Problems whose scratch (hils_score_select_workspace_size) exceeds
+ *     HILS_NOALLOC_SCRATCH_BYTES return HILS_ERR_WORKSPACE; N != 1 returns
+ *     HILS_ERR_UNSUPPORTED.  Nothing is launched in either case.
+ *   - The call allocates and frees nothing.  It clears the tickets it needs
+ *     before its kernel runs.
+ *   - All calls share the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other host threads) race
+ *     and give undefined results.
+ */
+#define HILS_NOALLOC_SCRATCH_BYTES (1u << 20)   /* 1 MiB per device */
+HILS_API hils_status hils_decode_score_select_noalloc(const hils_problem *p, const void *Q, const void *L,
+                                                      int32_t *sel_idx, float *sel_score, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
