@@ -165,8 +165,9 @@ def hils_sync_status(stream=None):
     return _lib.hils_sync_status(_stream(stream))
 
 
-def hils_set_wait_limit(polls):
-    _check(_lib.hils_set_wait_limit(int(polls)), "hils_set_wait_limit")
+def hils_set_wait_limit(ns):
+    """Bounded-wait limit of the kernels in nanoseconds (0 = default, one second)."""
+    _check(_lib.hils_set_wait_limit(int(ns)), "hils_set_wait_limit")
 
 
 def hils_decode_score_select_noalloc(p, Q, L, sel_idx, sel_score, stream=None):

@@ -1,5 +1,7 @@
 // api.cu -- the C ABI of libhils.so: validation, workspace sizing, dispatch.
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 #include <mutex>
 
 #include "internal.h"
@@ -10,9 +12,11 @@ namespace {
 
 __device__ unsigned int g_status;   // device-side status word (one per device)
 
-constexpr long long kDefaultWaitLimit = 1ll << 24;   // polls; roughly a second of spinning
+constexpr long long kDefaultWaitLimit = 1000000000ll;   // ns of the GPU global timer: one second
 long long g_wait_limit = kDefaultWaitLimit;
 std::mutex g_mu;
+
+}  // namespace
 
 hils_status device_ctl(DeviceCtl *ctl)
 {
@@ -30,6 +34,8 @@ hils_status device_ctl(DeviceCtl *ctl)
     ctl->wait_limit = g_wait_limit;
     return HILS_OK;
 }
+
+namespace {
 
 bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
@@ -55,17 +61,18 @@ hils_status resolve(const hils_problem *p, Dims *o)
     o->nL = (p->T + p->C - 1) / p->C;
     o->q_offset = p->q_offset;
     o->scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
-    if (o->N == 1) {
-        const DecodePlan plan = decode_plan(*o);
-        if ((size_t)plan.sort_n * 8 + (size_t)o->d * 4 > 200 * 1024) return HILS_ERR_UNSUPPORTED;
-    }
+    if (o->N == 1 && decode_select_smem_bytes(*o, p->in_dtype) > 200 * 1024) return HILS_ERR_UNSUPPORTED;
     return HILS_OK;
 }
 
 size_t sel_idx_bytes(const Dims &p) { return align_up((size_t)p.B * p.Hkv * p.N * p.k * sizeof(int32_t), 256); }
 size_t sel_score_bytes(const Dims &p) { return align_up((size_t)p.B * p.H * p.N * (p.k + 1) * sizeof(float), 256); }
 size_t select_ws(const Dims &p) { return p.N == 1 ? decode_select_ws_bytes(p) : 0; }
-size_t attend_ws(const Dims &p) { return p.N == 1 ? decode_attend_ws_bytes(p) : 0; }
+size_t attend_ws(const Dims &p, hils_dtype in)
+{
+    if (p.N == 1) return decode_attend_ws_bytes(p);
+    return attend_tc_supported(p, in) ? attend_tc_ws_bytes(p) : 0;
+}
 
 hils_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA; }
 
@@ -80,7 +87,12 @@ hils_status check_ws(void *ws, size_t have, size_t need)
 hils_status do_select(const Dims &p, hils_dtype in, const void *Q, const void *L, int32_t *sel_idx,
                       float *sel_score, void *ws, cudaStream_t s)
 {
-    if (p.N == 1) return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, s));
+    if (p.N == 1) {
+        DeviceCtl ctl;
+        hils_status st = device_ctl(&ctl);
+        if (st != HILS_OK) return st;
+        return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, ctl, s));
+    }
     return from_cuda(launch_select_prefill(p, in, Q, L, sel_idx, sel_score, s));
 }
 
@@ -88,21 +100,25 @@ hils_status do_attend(const Dims &p, hils_dtype in, hils_dtype out, const void *
                       const void *V, const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
                       cudaStream_t s)
 {
-    if (p.N == 1) return from_cuda(launch_attend_decode(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, s));
     DeviceCtl ctl;
     hils_status st = device_ctl(&ctl);
     if (st != HILS_OK) return st;
-    return from_cuda(launch_attend_prefill(p, in, out, Q, K, V, sel_idx, sel_score, O, ctl, s));
+    if (p.N == 1) return from_cuda(launch_attend_decode(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
+    return from_cuda(launch_attend_prefill(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
 }
 
 }  // namespace
 
 // Prefill dispatch: the tensor-core kernel when it covers the shape, else CUDA cores.
+// HILS_PREFILL_KERNEL=simt forces the CUDA-core kernel (used to cross-check the two).
 cudaError_t launch_attend_prefill(const Dims &p, hils_dtype in, hils_dtype out, const void *Q, const void *K,
-                                  const void *V, const int32_t *sel_idx, const float *sel_score, void *O,
+                                  const void *V, const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
                                   const DeviceCtl &ctl, cudaStream_t s)
 {
-    (void)ctl;
+    const char *force = getenv("HILS_PREFILL_KERNEL");
+    const bool simt = force && strcmp(force, "simt") == 0;
+    if (!simt && attend_tc_supported(p, in))
+        return launch_attend_prefill_tc(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s);
     return launch_attend_prefill_simt(p, in, out, Q, K, V, sel_idx, sel_score, O, s);
 }
 
@@ -149,7 +165,7 @@ hils_status hils_chunk_attend_fuse_workspace_size(const hils_problem *p, size_t 
     if (!bytes) return HILS_ERR_INVALID_ARG;
     hils_status st = resolve(p, &d);
     if (st != HILS_OK) return st;
-    *bytes = attend_ws(d);
+    *bytes = attend_ws(d, p->in_dtype);
     return HILS_OK;
 }
 
@@ -159,7 +175,7 @@ hils_status hils_forward_workspace_size(const hils_problem *p, size_t *bytes)
     if (!bytes) return HILS_ERR_INVALID_ARG;
     hils_status st = resolve(p, &d);
     if (st != HILS_OK) return st;
-    const size_t scratch = select_ws(d) > attend_ws(d) ? select_ws(d) : attend_ws(d);
+    const size_t scratch = select_ws(d) > attend_ws(d, p->in_dtype) ? select_ws(d) : attend_ws(d, p->in_dtype);
     *bytes = sel_idx_bytes(d) + sel_score_bytes(d) + scratch;
     return HILS_OK;
 }
@@ -189,7 +205,7 @@ hils_status hils_chunk_attend_fuse(const hils_problem *p, const void *Q, const v
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(sel_score) ||
         (sel_idx && !aligned16(sel_idx)))
         return HILS_ERR_INVALID_ARG;
-    st = check_ws(workspace, workspace_bytes, attend_ws(d));
+    st = check_ws(workspace, workspace_bytes, attend_ws(d, p->in_dtype));
     if (st != HILS_OK) return st;
     return do_attend(d, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, workspace,
                      static_cast<cudaStream_t>(stream));
@@ -234,11 +250,11 @@ hils_status hils_sync_status(void *stream)
     return HILS_OK;
 }
 
-hils_status hils_set_wait_limit(long long polls)
+hils_status hils_set_wait_limit(long long ns)
 {
-    if (polls < 0) return HILS_ERR_INVALID_ARG;
+    if (ns < 0) return HILS_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lk(g_mu);
-    g_wait_limit = polls == 0 ? kDefaultWaitLimit : polls;
+    g_wait_limit = ns == 0 ? kDefaultWaitLimit : ns;
     return HILS_OK;
 }
 

@@ -1,0 +1,553 @@
+// attend_prefill_tc.cu -- chunk attention and fusion on the sm_100a tensor cores (bf16 in, d = 128, C = 64).
+//
+// "Hierarchical Sparse Attention Done Right" (arXiv 2607.02980v1):
+//   Abstract / Sec. 3 "Hierarchical softmax": softmax inside every selected
+//   chunk, chunk outputs fused by a softmax over the retrieval scores;
+//   Sec. 4 "Kernel design": adjacent queries share most of their chunks, so a
+//   block of M queries is processed over the union of their chunks, making the
+//   tensor-core product (M x G, d) x (d, S) and loading each chunk once;
+//   Sec. 4 "Architecture": a GQA group's heads share the retrieved chunks.
+//
+// One CTA owns 128 rows = (128 / G) consecutive queries x the G heads of one
+// kv-group (row r = head * (128 / G) + query).  It walks the union of the
+// chunks its queries selected, in ascending chunk order:
+//   warp 0 (one thread)  TMA loads of Q once and of every union chunk's K and V
+//                        (two 64-column halves each, 128-byte swizzle, no
+//                        multicast) and the tcgen05.mma issue: S = Q K^T (bf16,
+//                        A and B from shared memory) into one of two TMEM
+//                        buffers, then O += P V (f16, P from TMEM, V from shared
+//                        memory) into the TMEM accumulator;
+//   warps 2..9           two groups of four warps, one thread per row; group
+//                        t % 2 handles chunk t: it reads S from TMEM, takes the
+//                        softmax over the chunk's visible keys, scales it by the
+//                        row's fusion weight (0 if the row's query did not
+//                        select this chunk) and writes P (f16) to TMEM.  At the
+//                        end both groups read O from TMEM and store it.
+// Because each chunk's softmax is normalised on its own and the fusion weights
+// are known before the loop, P already carries w_c / l_c and the accumulator
+// needs no rescaling between chunks.  V is read as f16 (converted once per call
+// by a streaming pass), so P can be kept in f16 with a 2^-11 rounding.
+//
+// Every barrier wait is bounded: on expiry the CTA records HILS_ERR_TIMEOUT,
+// stops issuing work, waits (with its own bound) for the copies and MMAs it has
+// in flight, frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace hils {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;     // 10 warps
+constexpr int kRows = 128;        // MMA M
+constexpr int kChunk = 64;        // C
+constexpr int kD = 128;           // d
+constexpr uint32_t kTmemCols = 512;   // S0, S1 (64 each), O (128), P0, P1 (32 each)
+constexpr uint32_t kColO = 128, kColP = 256;
+constexpr unsigned long long kDrainNs = 2000000000ull;
+
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 64, false, false);   // S = Q K^T, bf16, both K-major
+constexpr uint32_t IDESC_PV = idesc_f16_f32(128, 128, false, true);    // O += P V, f16, V MN-major
+
+struct Layout {
+    uint32_t q, kv, pbuf, bar, misc, bitmap, uni, qlist, qcnt, wts, total;
+};
+
+__host__ __device__ inline uint32_t al16(uint32_t x) { return (x + 15u) & ~15u; }
+
+template <int NS>
+__host__ __device__ inline Layout make_layout(int k, int nwords, int BQ)
+{
+    Layout L;
+    const uint32_t ns = (uint32_t)(k + 1);
+    L.q = 0;
+    L.kv = 32768;
+    L.pbuf = L.kv + NS * 32768u;   // (unused: P lives in TMEM)
+    L.bar = L.pbuf;
+    L.misc = L.bar + 32 * 8;
+    L.bitmap = L.misc + 16;
+    L.uni = al16(L.bitmap + 4u * (uint32_t)nwords);
+    L.qlist = al16(L.uni + 4u * ns * (uint32_t)BQ);
+    L.qcnt = al16(L.qlist + 4u * ns * (uint32_t)BQ);
+    L.wts = al16(L.qcnt + 4u * (uint32_t)BQ);
+    L.total = al16(L.wts + 4u * ns * (uint32_t)kRows);
+    return L;
+}
+
+// barrier slots
+template <int NS>
+struct Bars {
+    static constexpr int Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + NS, S_FULL = 1 + 2 * NS, P_FULL = 3 + 2 * NS,
+                         P_EMPTY = 5 + 2 * NS, O_FULL = 7 + 2 * NS, MMA_DONE = 8 + 2 * NS;
+};
+
+__device__ __forceinline__ void store_row32(float *dst, const uint32_t *v)
+{
+#pragma unroll
+    for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4 *>(dst + i) =
+            make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                        __uint_as_float(v[i + 3]));
+}
+
+__device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const uint32_t *v)
+{
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+        uint4 u;
+        __nv_bfloat162 a = __floats2bfloat162_rn(__uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+        __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+        __nv_bfloat162 c = __floats2bfloat162_rn(__uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
+        __nv_bfloat162 d = __floats2bfloat162_rn(__uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
+        u.x = *reinterpret_cast<uint32_t *>(&a);
+        u.y = *reinterpret_cast<uint32_t *>(&b);
+        u.z = *reinterpret_cast<uint32_t *>(&c);
+        u.w = *reinterpret_cast<uint32_t *>(&d);
+        *reinterpret_cast<uint4 *>(dst + i) = u;
+    }
+}
+
+// lane 0 waits, the result is broadcast so the warp decides uniformly
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, unsigned long long lim, volatile int *abort_flag,
+                                          unsigned int *status)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, lim, abort_flag, status) ? 1 : 0;
+    return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
+template <int G, typename Tout, int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, Dims p, const int32_t *__restrict__ sel_idx,
+                     const float *__restrict__ sel_score, Tout *__restrict__ O, unsigned int *status,
+                     unsigned long long limit_ns, int nwords)
+{
+    constexpr int BQ = kRows / G;
+    using BR = Bars<NS>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    const Layout Ly = make_layout<NS>(p.k, nwords, BQ);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q0 = blockIdx.x * BQ, g = blockIdx.y, b = blockIdx.z;
+    const int nq = min(BQ, p.N - q0);
+    const int ns = p.k + 1;
+
+    const uint32_t sQ = smem_addr(base + Ly.q), sKV = smem_addr(base + Ly.kv);
+    const uint32_t bar0 = smem_addr(base + Ly.bar);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + Ly.misc);
+    int *n_union_p = reinterpret_cast<int *>(base + Ly.misc + 4);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 8);
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(base + Ly.bitmap);
+    int *uni = reinterpret_cast<int *>(base + Ly.uni);
+    int *qlist = reinterpret_cast<int *>(base + Ly.qlist);
+    int *qcnt = reinterpret_cast<int *>(base + Ly.qcnt);
+    float *wts = reinterpret_cast<float *>(base + Ly.wts);
+    auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+
+    // ---- set-up: barriers, TMEM, union of the block's selected chunks ------
+    if (tid == 0) {
+        mbar_init(BAR(BR::Q_FULL), 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(BAR(BR::KV_FULL + s), 1);
+            mbar_init(BAR(BR::KV_EMPTY + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(BAR(BR::S_FULL + s), 1);
+            mbar_init(BAR(BR::P_FULL + s), 4);
+            mbar_init(BAR(BR::P_EMPTY + s), 1);
+        }
+        mbar_init(BAR(BR::O_FULL), 1);
+        mbar_init(BAR(BR::MMA_DONE), 1);
+        fence_mbar_init();
+        *abort_flag = 0;
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_holder), kTmemCols);
+        tmem_relinquish();
+    }
+    for (int i = tid; i < nwords; i += kThreads) bitmap[i] = 0u;
+    __syncthreads();
+
+    const int32_t *sel_base = sel_idx + ((((size_t)b * p.Hkv + g) * p.N) + q0) * p.k;
+    for (int e = tid; e < nq * p.k; e += kThreads) {
+        const int c = sel_base[e];
+        if (c >= 0) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+    }
+    for (int qi = tid; qi < nq; qi += kThreads) {
+        const int c = (int)(((long long)p.q_offset + q0 + qi) / kChunk);
+        atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ascending list of the union's chunks
+        int running = 0;
+        for (int w0 = 0; w0 < nwords; w0 += 32) {
+            uint32_t word = (w0 + lane < nwords) ? bitmap[w0 + lane] : 0u;
+            const int cnt = __popc(word);
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int off = running + incl - cnt;
+            while (word) {
+                const int bit = __ffs(word) - 1;
+                uni[off++] = (w0 + lane) * 32 + bit;
+                word &= word - 1;
+            }
+            running += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) *n_union_p = running;
+    } else if (tid >= 32 && tid < 32 + nq) {
+        // each query's chunks (selected + own) in ascending order
+        const int qi = tid - 32;
+        int *lst = qlist + qi * ns;
+        int cnt = 0;
+        for (int j = 0; j <= p.k; ++j) {
+            const int c = (j < p.k) ? sel_base[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
+            if (c < 0) continue;
+            int at = cnt++;
+            while (at > 0 && lst[at - 1] > c) {
+                lst[at] = lst[at - 1];
+                --at;
+            }
+            lst[at] = c;
+        }
+        qcnt[qi] = cnt;
+    }
+    __syncthreads();
+
+    if (tid < kRows) {
+        // fusion weights of each row, stored in the order of its query's chunk list
+        const int r = tid, h = r / BQ, qi = r % BQ;
+        if (qi < nq) {
+            const size_t row_h = (((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi;
+            const float *sc = sel_score + row_h * ns;
+            float M = -INFINITY;
+            for (int j = 0; j < ns; ++j) M = fmaxf(M, sc[j]);
+            float Z = 0.f;
+            for (int j = 0; j < ns; ++j) Z += (sc[j] == -INFINITY) ? 0.f : expf(sc[j] - M);
+            const int *lst = qlist + qi * ns;
+            const int cnt = qcnt[qi];
+            for (int j = 0; j < ns; ++j) {
+                const int c = (j < p.k) ? sel_base[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
+                if (c < 0) continue;
+                int lo = 0, hi = cnt - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (lst[mid] < c) lo = mid + 1; else hi = mid;
+                }
+                wts[r * ns + lo] = (sc[j] == -INFINITY) ? 0.f : expf(sc[j] - M) / Z;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const int n_union = *n_union_p;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA + MMA issue --------------------------------
+            const int kv_row0 = (b * p.Hkv + g) * p.T;
+            int next_load = 0;
+            bool ok = true;
+            mbar_arrive_expect_tx(BAR(BR::Q_FULL), 32768u);
+            tma_load_3d(sQ, &tmQ, BAR(BR::Q_FULL), 0, q0, b * p.H + g * G);
+            tma_load_3d(sQ + 16384u, &tmQ, BAR(BR::Q_FULL), 64, q0, b * p.H + g * G);
+
+            auto issue_pv = [&](int u) -> bool {
+                if (!mbar_wait(BAR(BR::P_FULL + (u & 1)), (u >> 1) & 1, limit_ns, abort_flag, status)) return false;
+                tc_fence_after();
+                const uint32_t st = (uint32_t)(u % NS);
+                const uint32_t pa = tmem + kColP + (uint32_t)(u & 1) * 32u;
+                const uint32_t va = sKV + st * 32768u + 16384u;
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_f16_ts(tmem + kColO, pa + 8u * s, smem_desc_sw128(va + 2048u * s, 8192, 1024), IDESC_PV,
+                               (u > 0 || s > 0) ? 1u : 0u);
+                mma_commit(BAR(BR::KV_EMPTY + (int)st));
+                mma_commit(BAR(BR::P_EMPTY + (u & 1)));
+                return true;
+            };
+
+            for (int t = 0; t < n_union && ok; ++t) {
+                while (next_load < n_union && (next_load < NS || next_load <= t + NS - 2)) {
+                    const int u = next_load, st = u % NS;
+                    if (u >= NS &&
+                        !mbar_wait(BAR(BR::KV_EMPTY + st), ((u / NS) - 1) & 1, limit_ns, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    const int row = kv_row0 + uni[u] * kChunk;
+                    const uint32_t dst = sKV + (uint32_t)st * 32768u;
+                    mbar_arrive_expect_tx(BAR(BR::KV_FULL + st), 32768u);
+                    tma_load_2d(dst, &tmK, BAR(BR::KV_FULL + st), 0, row);
+                    tma_load_2d(dst + 8192u, &tmK, BAR(BR::KV_FULL + st), 64, row);
+                    tma_load_2d(dst + 16384u, &tmV, BAR(BR::KV_FULL + st), 0, row);
+                    tma_load_2d(dst + 24576u, &tmV, BAR(BR::KV_FULL + st), 64, row);
+                    ++next_load;
+                }
+                if (!ok) break;
+                const int st = t % NS;
+                if (!mbar_wait(BAR(BR::KV_FULL + st), (t / NS) & 1, limit_ns, abort_flag, status)) break;
+                if (t == 0 && !mbar_wait(BAR(BR::Q_FULL), 0, limit_ns, abort_flag, status)) break;
+                tc_fence_after();
+                // S buffer t % 2 is free: its previous chunk's P was consumed by a PV issued earlier,
+                // and that group had read S before writing P
+                const uint32_t d_s = tmem + (uint32_t)(t & 1) * 64u;
+                const uint32_t ka = sKV + (uint32_t)st * 32768u;
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16_ss(d_s, smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
+                                smem_desc_sw128(ka + (s >> 2) * 8192u + (s & 3) * 32u, 16, 1024), IDESC_QK,
+                                s > 0 ? 1u : 0u);
+                mma_commit(BAR(BR::S_FULL + (t & 1)));
+                if (t >= 1 && !issue_pv(t - 1)) break;
+                if (t == n_union - 1) {
+                    if (issue_pv(t)) mma_commit(BAR(BR::O_FULL));
+                }
+            }
+            // drain: every issued MMA, then the latest load of every stage and Q
+            mma_commit(BAR(BR::MMA_DONE));
+            mbar_drain(BAR(BR::MMA_DONE), 0, kDrainNs);
+            for (int u = max(0, next_load - NS); u < next_load; ++u)
+                mbar_drain(BAR(BR::KV_FULL + u % NS), (u / NS) & 1, kDrainNs);
+            mbar_drain(BAR(BR::Q_FULL), 0, kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp >= 2) {
+        // ---------------- softmax (two groups, alternate chunks) and epilogue ----
+        const int grp = (warp - 2) >> 2;
+        const int qq = warp & 3;
+        const int r = 32 * qq + lane, h = r / BQ, qi = r % BQ;
+        const bool valid = qi < nq;
+        const long long pos = (long long)p.q_offset + q0 + qi;
+        const int own = (int)(pos / kChunk);
+        const int cnt = valid ? qcnt[qi] : 0;
+        const int *lst = qlist + qi * ns;
+        const float *wr = wts + r * ns;
+        const float sl2 = p.scale * 1.4426950408889634f;
+        const uint32_t lane_off = (uint32_t)(32 * qq) << 16;
+        const uint32_t tS = tmem + lane_off + (uint32_t)grp * 64u;
+        const uint32_t tP = tmem + lane_off + kColP + (uint32_t)grp * 32u;
+        int ptr = 0;
+        bool ok = true;
+        for (int t = grp; t < n_union; t += 2) {
+            const int u = t >> 1;
+            if (!warp_wait(BAR(BR::S_FULL + grp), (uint32_t)(u & 1), limit_ns, abort_flag, status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sv[64];
+            tmem_ld32(tS, sv);
+            tmem_ld32(tS + 32u, sv + 32);
+            tmem_wait_ld();
+
+            const int c = uni[t];
+            while (ptr < cnt && lst[ptr] < c) ++ptr;
+            const float w = (ptr < cnt && lst[ptr] == c) ? wr[ptr] : 0.f;
+            uint32_t pk[32];
+            if (w > 0.f) {
+                const int n_vis = (c == own) ? (int)(pos - (long long)c * kChunk + 1) : kChunk;
+                float mx[8];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
+                if (n_vis == kChunk) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sv[j]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (j < n_vis) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sv[j]));
+                }
+                const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                const float nb = -m * sl2;
+                float ls[8];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) ls[a] = 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const float e = (j < n_vis) ? ex2_approx(fmaf(__uint_as_float(sv[j]), sl2, nb)) : 0.f;
+                    sv[j] = __float_as_uint(e);
+                    ls[j & 7] += e;
+                }
+                const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                const float f = w / l;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    __half2 v2 = __floats2half2_rn(__uint_as_float(sv[2 * j]) * f, __uint_as_float(sv[2 * j + 1]) * f);
+                    pk[j] = *reinterpret_cast<uint32_t *>(&v2);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) pk[j] = 0u;
+            }
+            if (u >= 1 &&
+                !warp_wait(BAR(BR::P_EMPTY + grp), (uint32_t)((u - 1) & 1), limit_ns, abort_flag, status)) {
+                ok = false;
+                break;
+            }
+            tmem_st32(tP, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(BR::P_FULL + grp));
+        }
+        if (ok && warp_wait(BAR(BR::O_FULL), 0, limit_ns, abort_flag, status)) {
+            tc_fence_after();
+            Tout *orow = O + ((((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi) * kD;
+#pragma unroll
+            for (int cg = 0; cg < 2; ++cg) {
+                const int col = grp * 64 + cg * 32;
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + kColO + (uint32_t)col, v);
+                tmem_wait_ld();
+                if (valid) store_row32(orow + col, v);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// The driver's tensor-map encoder, looked up through the runtime so that the
+// library itself does not link against libcuda (it loads on machines without a
+// GPU driver; the lookup happens on the first launch).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+bool encode(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, int rank, const cuuint64_t *dims,
+            const cuuint64_t *strides, const cuuint32_t *box)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void *>(ptr),
+                                        dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+constexpr int kStages = 4;
+
+// V (bf16) -> f16, 8 elements per 16-byte vector; exact for |v| < 65504.
+__global__ void v_to_f16_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, size_t n)
+{
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const uint4 u = __ldg(in + i);
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            __half2 h2 = __floats2half2_rn(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+            w[e] = *reinterpret_cast<uint32_t *>(&h2);
+        }
+        out[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+template <int G, typename Tout>
+cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V, const int32_t *sel_idx,
+                     const float *sel_score, void *O, const DeviceCtl &ctl, cudaStream_t s)
+{
+    constexpr int BQ = kRows / G;
+    CUtensorMap tq, tk, tv;
+    const cuuint64_t qd[3] = {(cuuint64_t)kD, (cuuint64_t)p.N, (cuuint64_t)p.B * p.H};
+    const cuuint64_t qs[2] = {(cuuint64_t)kD * 2, (cuuint64_t)p.N * kD * 2};
+    const cuuint32_t qb[3] = {64, (cuuint32_t)BQ, (cuuint32_t)G};
+    const cuuint64_t kd[2] = {(cuuint64_t)kD, (cuuint64_t)p.B * p.Hkv * p.T};
+    const cuuint64_t ks[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t kb[2] = {64, (cuuint32_t)kChunk};
+    if (!encode(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, 3, qd, qs, qb) ||
+        !encode(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, 2, kd, ks, kb) ||
+        !encode(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, V, 2, kd, ks, kb))
+        return cudaErrorInvalidValue;
+    const int c_max = (int)(((long long)p.q_offset + p.N - 1) / kChunk);
+    const int nwords = c_max / 32 + 1;
+    const Layout Ly = make_layout<kStages>(p.k, nwords, BQ);
+    const size_t smem = Ly.total + 1024;
+    auto kern = attend_tc_kernel<G, Tout, kStages>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
+    kern<<<grid, kThreads, smem, s>>>(tq, tk, tv, p, sel_idx, sel_score, static_cast<Tout *>(O), ctl.status,
+                                      (unsigned long long)ctl.wait_limit, nwords);
+    return cudaGetLastError();
+}
+
+template <typename Tout>
+cudaError_t launch_o(const Dims &p, const void *Q, const void *K, const void *V, const int32_t *sel_idx,
+                     const float *sel_score, void *O, const DeviceCtl &ctl, cudaStream_t s)
+{
+    switch (p.G) {
+    case 1: return launch_g<1, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
+    case 2: return launch_g<2, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
+    case 4: return launch_g<4, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
+    case 8: return launch_g<8, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
+    default: return launch_g<16, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
+    }
+}
+
+}  // namespace
+
+// Whether the tensor-core kernel covers this problem.
+bool attend_tc_supported(const Dims &p, hils_dtype in)
+{
+    if (in != HILS_BF16 || p.d != kD || p.C != kChunk || p.N < 2) return false;
+    if (p.G != 1 && p.G != 2 && p.G != 4 && p.G != 8 && p.G != 16) return false;
+    const int c_max = (int)(((long long)p.q_offset + p.N - 1) / kChunk);
+    const Layout Ly = make_layout<kStages>(p.k, c_max / 32 + 1, kRows / p.G);
+    return Ly.total + 1024 <= 227 * 1024;
+}
+
+size_t attend_tc_ws_bytes(const Dims &p)
+{
+    return align_up((size_t)p.B * p.Hkv * p.T * kD * 2, 256);   // V as f16
+}
+
+cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
+                                     const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
+                                     const DeviceCtl &ctl, cudaStream_t s)
+{
+    const size_t n16 = (size_t)p.B * p.Hkv * p.T * kD / 8;
+    v_to_f16_kernel<<<148 * 8, 256, 0, s>>>(static_cast<const uint4 *>(V), static_cast<uint4 *>(ws), n16);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (out == HILS_F32) return launch_o<float>(p, Q, K, ws, sel_idx, sel_score, O, ctl, s);
+    return launch_o<__nv_bfloat16>(p, Q, K, ws, sel_idx, sel_score, O, ctl, s);
+}
+
+}  // namespace hils

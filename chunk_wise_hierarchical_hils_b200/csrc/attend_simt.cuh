@@ -19,6 +19,7 @@ __device__ __forceinline__ void stage_rows(Tin *dst, const Tin *src, int n_rows)
     const int n_vec = n_rows * D / VEC;
     const uint4 *s = reinterpret_cast<const uint4 *>(src);
     uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll 8
     for (int e = threadIdx.x; e < n_vec; e += blockDim.x) d[e] = __ldg(s + e);
 }
 

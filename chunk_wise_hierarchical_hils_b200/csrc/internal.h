@@ -41,17 +41,28 @@ size_t decode_attend_ws_bytes(const Dims &p);
 cudaError_t launch_select_prefill(const Dims &p, hils_dtype in, const void *Q, const void *L,
                                   int32_t *sel_idx, float *sel_score, cudaStream_t s);
 cudaError_t launch_select_decode(const Dims &p, hils_dtype in, const void *Q, const void *L,
-                                 int32_t *sel_idx, float *sel_score, void *ws, cudaStream_t s);
+                                 int32_t *sel_idx, float *sel_score, void *ws, const DeviceCtl &ctl,
+                                 cudaStream_t s);
+size_t decode_select_smem_bytes(const Dims &p, hils_dtype in);
 cudaError_t launch_attend_prefill(const Dims &p, hils_dtype in, hils_dtype out, const void *Q,
                                   const void *K, const void *V, const int32_t *sel_idx,
-                                  const float *sel_score, void *O, const DeviceCtl &ctl,
+                                  const float *sel_score, void *O, void *ws, const DeviceCtl &ctl,
                                   cudaStream_t s);
 cudaError_t launch_attend_prefill_simt(const Dims &p, hils_dtype in, hils_dtype out, const void *Q,
                                        const void *K, const void *V, const int32_t *sel_idx,
                                        const float *sel_score, void *O, cudaStream_t s);
+bool attend_tc_supported(const Dims &p, hils_dtype in);
+size_t attend_tc_ws_bytes(const Dims &p);
+cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
+                                     const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
+                                     const DeviceCtl &ctl, cudaStream_t s);
 cudaError_t launch_attend_decode(const Dims &p, hils_dtype in, hils_dtype out, const void *Q,
                                  const void *K, const void *V, const int32_t *sel_idx,
-                                 const float *sel_score, void *O, void *ws, cudaStream_t s);
+                                 const float *sel_score, void *O, void *ws, const DeviceCtl &ctl,
+                                 cudaStream_t s);
+
+// Device status word and wait limit of the current device (looked up once per device).
+hils_status device_ctl(DeviceCtl *ctl);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

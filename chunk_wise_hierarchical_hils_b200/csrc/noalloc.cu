@@ -77,8 +77,11 @@ extern "C" hils_status hils_decode_score_select_noalloc(const hils_problem *p, c
     d.nL = (p->T + p->C - 1) / p->C;
     d.q_offset = p->q_offset;
     d.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+    DeviceCtl ctl;
+    st = device_ctl(&ctl);
+    if (st != HILS_OK) return st;
     // the launcher clears the completion tickets in the scratch before the kernel runs
-    cudaError_t e = launch_select_decode(d, p->in_dtype, Q, L, sel_idx, sel_score, scratch,
+    cudaError_t e = launch_select_decode(d, p->in_dtype, Q, L, sel_idx, sel_score, scratch, ctl,
                                          static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
 }

@@ -6,32 +6,43 @@
 //
 // With one query per (b, g) and up to 65,536 candidate chunks, the scan is split
 // over `nsplit` CTAs per (b, g) so that the landmark cache streams through all
-// SMs.  Each split scores its range of chunks (half a warp, or a quarter for
-// d = 64, reads one 16-byte piece per lane of each landmark row), sorts its keys
-// in shared memory and publishes its local top-k to the workspace.  The last
-// split CTA to finish for a (b, g) (atomic ticket) merges the nsplit local lists:
-// the global top-k is contained in their union.  It then writes the selection and
-// the per-head scores of the k slots plus the own chunk.
+// SMs at HBM rate.  Each split streams its contiguous range of landmark rows
+// into a ring of shared-memory stages with bulk asynchronous copies (one copy
+// per stage, several stages in flight), scores them (one 16-byte piece per lane,
+// a row per half warp), sorts its keys in shared memory and publishes its local
+// top-k.  The last split CTA of a (b, g) (atomic ticket) merges the nsplit
+// local lists -- the global top-k lies in their union -- and writes the
+// selection and the per-head scores of the k slots plus the own chunk.
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace hils {
 namespace {
 
-constexpr int NT = 256;   // threads per CTA
+using namespace sm100;
+
+constexpr int NT = 256;          // threads per CTA
+constexpr int RING = 4;          // stages in flight
+constexpr int RPS = 32;          // landmark rows per stage
+constexpr unsigned long long kDrainNs = 2000000000ull;
 
 template <typename Tin, int D>
-__global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan plan,
-                                                           const Tin *__restrict__ Q,
-                                                           const Tin *__restrict__ L,
-                                                           uint64_t *__restrict__ cand,
+__global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan plan, const Tin *__restrict__ Q,
+                                                           const Tin *__restrict__ L, uint64_t *__restrict__ cand,
                                                            unsigned int *__restrict__ tickets,
                                                            int32_t *__restrict__ sel_idx,
-                                                           float *__restrict__ sel_score)
+                                                           float *__restrict__ sel_score, unsigned int *status,
+                                                           unsigned long long limit_ns)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    float *qs = reinterpret_cast<float *>(smem_raw);                    // [D]
-    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw + D * sizeof(float));  // [sort_n]
+    constexpr uint32_t STAGE_BYTES = RPS * D * sizeof(Tin);
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    float *qs = reinterpret_cast<float *>(smem_raw);                              // [D]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + D * sizeof(float));  // [RING]
+    unsigned char *ring = smem_raw + D * sizeof(float) + 128;                      // [RING][STAGE_BYTES]
+    uint64_t *keys = reinterpret_cast<uint64_t *>(ring + RING * STAGE_BYTES);      // [spl]
+    uint64_t *mkeys = reinterpret_cast<uint64_t *>(ring);                          // merge reuses the ring
     __shared__ int s_last;
+    __shared__ int s_abort;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bg = blockIdx.y, b = bg / p.Hkv, g = bg % p.Hkv;
@@ -41,8 +52,25 @@ __global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan pl
     const int n_past = p.k > 0 ? ci : 0;   // k == 0: only the own chunk is used
     const int c0 = split * plan.spl;
     const int c1 = min(c0 + plan.spl, n_past);
+    const int n_local = max(c1 - c0, 0);
+    const int n_stages = (n_local + RPS - 1) / RPS;
     const Tin *Lbg = L + (size_t)bg * p.nL * D;
+    const uint32_t bar0 = smem_addr(bars), ring0 = smem_addr(ring);
 
+    auto issue = [&](int s) {
+        const int r0 = c0 + s * RPS, nr = min(RPS, c1 - r0);
+        const uint32_t bytes = (uint32_t)nr * D * sizeof(Tin);
+        const uint32_t bar = bar0 + 8u * (uint32_t)(s % RING);
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load(ring0 + (uint32_t)(s % RING) * STAGE_BYTES, Lbg + (size_t)r0 * D, bytes, bar);
+    };
+
+    if (tid == 0) {
+        for (int s = 0; s < RING; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
+        s_abort = 0;
+        for (int s = 0; s < min(RING, n_stages); ++s) issue(s);
+    }
     if (tid < D) {
         float a = 0.f;
         for (int h = 0; h < p.G; ++h) a += to_float(Q[((size_t)b * p.H + (size_t)g * p.G + h) * D + tid]);
@@ -57,33 +85,42 @@ __global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan pl
     float qv[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) qv[u] = qs[sub * 8 + u];
-    constexpr int UNR = 4;
-    const int step = (NT / 32) * RPW;
-    // the loop bound is warp-uniform so that every lane reaches the shuffles
-    for (int cw = c0 + warp * RPW; cw < c1; cw += step * UNR) {
-        float lv[UNR][8];
+    int s_done = 0;   // stages consumed
+    for (int s = 0; s < n_stages; ++s) {
+        const int slot = s % RING;
+        if (!mbar_wait(bar0 + 8u * slot, (uint32_t)((s / RING) & 1), limit_ns, &s_abort, status)) s_abort = 1;
+        if (!s_abort) {
+            const int r0 = s * RPS, nr = min(RPS, n_local - r0);
+            const Tin *st = reinterpret_cast<const Tin *>(ring + (size_t)slot * STAGE_BYTES);
+            // the loop bound is warp-uniform so that every lane reaches the shuffles
+            for (int rw = warp * RPW; rw < nr; rw += (NT / 32) * RPW) {
+                const int rr = rw + lane / LPC;
+                float lv[8];
+                if (rr < nr) {
+                    lds8(st + (size_t)rr * D + sub * 8, lv);
+                } else {
 #pragma unroll
-        for (int r = 0; r < UNR; ++r) {
-            const int c = cw + lane / LPC + r * step;
-            if (c < c1) {
-                load8(Lbg + (size_t)c * D + sub * 8, lv[r]);
-            } else {
+                    for (int u = 0; u < 8; ++u) lv[u] = 0.f;
+                }
+                float a = 0.f;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) lv[r][u] = 0.f;
+                for (int u = 0; u < 8; ++u) a = fmaf(qv[u], lv[u], a);
+#pragma unroll
+                for (int o = LPC / 2; o; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+                if (sub == 0 && rr < nr) keys[r0 + rr] = make_key(a, c0 + r0 + rr);
             }
         }
-#pragma unroll
-        for (int r = 0; r < UNR; ++r) {
-            float a = 0.f;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) a = fmaf(qv[u], lv[r][u], a);
-#pragma unroll
-            for (int o = LPC / 2; o; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
-            const int c = cw + lane / LPC + r * step;
-            if (sub == 0 && c < c1) keys[c - c0] = make_key(a, c);
-        }
+        __syncthreads();
+        if (s_abort) break;
+        s_done = s + 1;
+        if (tid == 0 && s + RING < n_stages) issue(s + RING);
     }
-    const int n_local = max(c1 - c0, 0);
+    if (tid == 0 && s_abort) {
+        // after an abort: the copies of stages issued but not consumed must land before exit
+        const int issued = min(n_stages, s_done + RING);
+        for (int u = s_done; u < issued; ++u)
+            mbar_drain(bar0 + 8u * (u % RING), (uint32_t)((u / RING) & 1), kDrainNs);
+    }
     int local_n = 1;
     while (local_n < n_local) local_n <<= 1;
     for (int e = n_local + tid; e < local_n; e += NT) keys[e] = 0ull;
@@ -105,33 +142,47 @@ __global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan pl
     int merge_n = 1;
     while (merge_n < nm) merge_n <<= 1;
     const uint64_t *all = cand + (size_t)bg * plan.nsplit * p.k;
-    for (int e = tid; e < merge_n; e += NT) keys[e] = (e < nm) ? __ldcg(all + e) : 0ull;
-    if (merge_n > 1) bitonic_sort_desc(keys, merge_n);
+    for (int e = tid; e < merge_n; e += NT) mkeys[e] = (e < nm) ? __ldcg(all + e) : 0ull;
+    if (merge_n > 1) bitonic_sort_desc(mkeys, merge_n);
     else __syncthreads();
 
     int32_t *si = sel_idx + (size_t)bg * p.k;
-    for (int j = tid; j < p.k; j += NT) si[j] = key_index(keys[j]);
+    for (int j = tid; j < p.k; j += NT) si[j] = key_index(mkeys[j]);
 
-    // per-head scores of the k slots and the own chunk: one warp per (head, slot)
+    // per-head scores of the k slots and the own chunk: LPC lanes per (head, slot)
     const int ns = p.k + 1;
-    for (int task = warp; task < p.G * ns; task += NT / 32) {
-        const int h = task / ns, j = task % ns;
-        const int c = (j < p.k) ? key_index(keys[j]) : ci;
+    constexpr int TPW = 32 / LPC;   // tasks per warp step
+    for (int t0 = warp * TPW; t0 < p.G * ns; t0 += (NT / 32) * TPW) {
+        const int task = t0 + lane / LPC;
+        const bool live = task < p.G * ns;
+        const int h = live ? task / ns : 0, j = live ? task % ns : 0;
+        const int c = !live ? -1 : (j < p.k) ? key_index(mkeys[j]) : ci;
         float acc = 0.f;
         if (c >= 0) {
-            const Tin *qrow = Q + ((size_t)b * p.H + (size_t)g * p.G + h) * D;
-            const Tin *lrow = Lbg + (size_t)c * D;
-            for (int x = lane; x < D; x += 32) acc = fmaf(to_float(qrow[x]), to_float(lrow[x]), acc);
-            acc = warp_sum(acc);
+            float qv8[8], lv8[8];
+            load8(Q + ((size_t)b * p.H + (size_t)g * p.G + h) * D + sub * 8, qv8);
+            load8(Lbg + (size_t)c * D + sub * 8, lv8);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc = fmaf(qv8[u], lv8[u], acc);
         }
-        if (lane == 0)
+#pragma unroll
+        for (int o = LPC / 2; o; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+        if (live && sub == 0)
             sel_score[((size_t)b * p.H + (size_t)g * p.G + h) * ns + j] = (c >= 0) ? acc * p.scale : -INFINITY;
     }
 }
 
 template <typename Tin, int D>
-cudaError_t launch_t(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
-                     void *ws, cudaStream_t s)
+size_t smem_bytes(const DecodePlan &plan)
+{
+    const size_t scan = D * sizeof(float) + 128 + (size_t)RING * RPS * D * sizeof(Tin) + (size_t)plan.spl * 8;
+    const size_t merge = D * sizeof(float) + 128 + (size_t)plan.sort_n * 8;
+    return scan > merge ? scan : merge;
+}
+
+template <typename Tin, int D>
+cudaError_t launch_t(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score, void *ws,
+                     const DeviceCtl &ctl, cudaStream_t s)
 {
     const DecodePlan plan = decode_plan(p);
     uint64_t *cand = static_cast<uint64_t *>(ws);
@@ -139,13 +190,13 @@ cudaError_t launch_t(const Dims &p, const void *Q, const void *L, int32_t *sel_i
         static_cast<char *>(ws) + align_up((size_t)p.B * p.Hkv * plan.nsplit * p.k * sizeof(uint64_t), 256));
     cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)p.B * p.Hkv * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
-    const size_t smem = D * sizeof(float) + (size_t)plan.sort_n * sizeof(uint64_t);
+    const size_t smem = smem_bytes<Tin, D>(plan);
     auto kern = select_decode_kernel<Tin, D>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(plan.nsplit, p.B * p.Hkv);
-    kern<<<grid, NT, smem, s>>>(p, plan, static_cast<const Tin *>(Q), static_cast<const Tin *>(L), cand,
-                                tickets, sel_idx, sel_score);
+    kern<<<grid, NT, smem, s>>>(p, plan, static_cast<const Tin *>(Q), static_cast<const Tin *>(L), cand, tickets,
+                                sel_idx, sel_score, ctl.status, (unsigned long long)ctl.wait_limit);
     return cudaGetLastError();
 }
 
@@ -166,12 +217,11 @@ DecodePlan decode_plan(const Dims &p)
     int m = 1;
     while (m < plan.nsplit * p.k) m <<= 1;
     plan.sort_n = m > spl ? m : spl;
-    // attention: one CTA per group of selected chunks, about four CTAs per SM
+    // attention: two selected chunks per CTA when both fit in 64 KB of shared memory
     const int ns = p.k + 1;
-    int per = 1;
-    while (per < ns && (long long)bg * ((ns + per - 1) / per) > 8 * 148) ++per;
-    plan.slots_per_cta = per;
-    plan.nsplit2 = (ns + per - 1) / per;
+    const size_t chunk_bytes = 2ull * p.C * p.d * 2;   // K and V rows of one chunk, bf16
+    plan.slots_per_cta = chunk_bytes <= 32768 ? 2 : 1;
+    plan.nsplit2 = (ns + plan.slots_per_cta - 1) / plan.slots_per_cta;
     return plan;
 }
 
@@ -182,14 +232,21 @@ size_t decode_select_ws_bytes(const Dims &p)
            align_up((size_t)p.B * p.Hkv * sizeof(unsigned int), 256);
 }
 
-cudaError_t launch_select_decode(const Dims &p, hils_dtype in, const void *Q, const void *L,
-                                 int32_t *sel_idx, float *sel_score, void *ws, cudaStream_t s)
+size_t decode_select_smem_bytes(const Dims &p, hils_dtype in)
+{
+    const DecodePlan plan = decode_plan(p);
+    if (in == HILS_F32) return p.d == 64 ? smem_bytes<float, 64>(plan) : smem_bytes<float, 128>(plan);
+    return p.d == 64 ? smem_bytes<__nv_bfloat16, 64>(plan) : smem_bytes<__nv_bfloat16, 128>(plan);
+}
+
+cudaError_t launch_select_decode(const Dims &p, hils_dtype in, const void *Q, const void *L, int32_t *sel_idx,
+                                 float *sel_score, void *ws, const DeviceCtl &ctl, cudaStream_t s)
 {
     if (in == HILS_F32)
-        return p.d == 64 ? launch_t<float, 64>(p, Q, L, sel_idx, sel_score, ws, s)
-                         : launch_t<float, 128>(p, Q, L, sel_idx, sel_score, ws, s);
-    return p.d == 64 ? launch_t<__nv_bfloat16, 64>(p, Q, L, sel_idx, sel_score, ws, s)
-                     : launch_t<__nv_bfloat16, 128>(p, Q, L, sel_idx, sel_score, ws, s);
+        return p.d == 64 ? launch_t<float, 64>(p, Q, L, sel_idx, sel_score, ws, ctl, s)
+                         : launch_t<float, 128>(p, Q, L, sel_idx, sel_score, ws, ctl, s);
+    return p.d == 64 ? launch_t<__nv_bfloat16, 64>(p, Q, L, sel_idx, sel_score, ws, ctl, s)
+                     : launch_t<__nv_bfloat16, 128>(p, Q, L, sel_idx, sel_score, ws, ctl, s);
 }
 
 }  // namespace hils

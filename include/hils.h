@@ -142,15 +142,19 @@ HILS_API hils_status hils_forward(const hils_problem *p, const void *Q, const vo
  * HILS_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the kernel then
  * skipped its remaining work and released its resources), HILS_ERR_CUDA if
  * the synchronisation failed, else HILS_OK.  Clears the recorded status.
+ * A recorded timeout is sticky until read here: kernels launched meanwhile
+ * give up at their first slow wait, so one failure ends quickly everywhere.
  */
 HILS_API hils_status hils_sync_status(void *stream);
 
 /*
- * Debug/test control of the bounded waits: the number of polls a kernel makes
- * on a barrier before it records HILS_ERR_TIMEOUT and gives up.  0 restores the
- * default (about one second).  Affects kernels launched afterwards.
+ * Debug/test control of the bounded waits: how long (nanoseconds of the GPU's
+ * global timer) a kernel waits on a barrier before it records HILS_ERR_TIMEOUT
+ * and gives up.  0 restores the default of one second.  Affects kernels
+ * launched afterwards; a kernel that gives up still waits for its own copies
+ * and MMAs in flight and frees its tensor memory before it exits.
  */
-HILS_API hils_status hils_set_wait_limit(long long polls);
+HILS_API hils_status hils_set_wait_limit(long long ns);
 
 /*
  * Allocation-free decode selection.  The paper has no counterpart: this entry

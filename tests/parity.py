@@ -14,7 +14,11 @@ from oracle import oracle as orc
 from synth import workloads as W
 
 EPS_TIE = 1e-3          # near-tie band on group scores (selection may differ inside it)
-TOL_O = {"f32": 1e-4, "bf16": 1e-2}   # max-abs output error
+TOL_O = {"f32": 1e-4, "bf16": 1e-2}   # max-abs output error of the float32 result
+# A bf16 output adds its own rounding, up to half a bf16 ulp of the value (2^-8 relative below the
+# next power of two): compared against the float64 result, a bf16 output may differ by the
+# computation's tolerance plus that half ulp.  (For |o| >= 4 the half ulp alone is >= 0.0078, so a
+# flat 1e-2 cannot hold for bf16 outputs even from an exact computation.)
 TOL_S = 1e-4            # max-abs error of the per-head slot scores
 
 
@@ -79,8 +83,6 @@ def compare(w, items, answers, sel, s, o, tol_o=None, tol_s=TOL_S, out_dtype="f3
     """Check every sampled query group; returns a stats dict (failures listed in stats['fail'])."""
     if tol_o is None:
         tol_o = TOL_O[w.dtype]
-        if out_dtype == "bf16":
-            tol_o = max(tol_o, 1e-2)
     st = {"n": len(items), "near_tie": 0, "overflow": 0, "max_err_O": 0.0, "max_err_s": 0.0, "fail": []}
     for n, (it, ans) in enumerate(zip(items, answers)):
         pos = ans["pos"]
@@ -128,10 +130,13 @@ def compare(w, items, answers, sel, s, o, tol_o=None, tol_s=TOL_S, out_dtype="f3
                 st["max_err_s"] = max(st["max_err_s"], e)
                 if not e <= tol_s:
                     st["fail"].append((it, "slot score", j, h, gs, os_[h, jo]))
-        e = float(np.max(np.abs(o[n] - oo)))
-        st["max_err_O"] = max(st["max_err_O"], e)
-        if not e <= tol_o:
-            st["fail"].append((it, "output err %.3g" % e))
+        allowed = tol_o
+        if out_dtype == "bf16":
+            allowed = tol_o + np.ldexp(1.0, np.frexp(np.abs(oo))[1] - 9)   # half ulp of bf16 at |o|
+        e = np.abs(o[n] - oo)
+        st["max_err_O"] = max(st["max_err_O"], float(np.max(e)))
+        if not np.all(e <= allowed):
+            st["fail"].append((it, "output err %.3g" % float(np.max(e - allowed + tol_o))))
     return st
 
 

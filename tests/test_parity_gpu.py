@@ -58,6 +58,14 @@ def test_parity_small(w):
     _check(st)
 
 
+@pytest.mark.parametrize("w", [CASES[1], CASES[7], CASES[8], CASES[10]], ids=lambda w: w.name)
+def test_cuda_core_kernel_too(w, monkeypatch):
+    """The CUDA-core prefill kernel, forced, on shapes the tensor-core kernel normally takes."""
+    monkeypatch.setenv("HILS_PREFILL_KERNEL", "simt")
+    st, _ = parity.run_small(w)
+    _check(st)
+
+
 @pytest.mark.parametrize("w", [CASES[1], DECODE[0]], ids=lambda w: w.name)
 def test_bf16_output(w):
     st, _ = parity.run_small(w, out_dtype="bf16")
