@@ -76,6 +76,13 @@ size_t attend_ws(const Dims &p, hils_dtype in)
 
 hils_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA; }
 
+// HILS_PREFILL_KERNEL=simt forces the CUDA-core prefill kernels (used to cross-check the two paths).
+bool force_cuda_cores()
+{
+    const char *force = getenv("HILS_PREFILL_KERNEL");
+    return force && strcmp(force, "simt") == 0;
+}
+
 hils_status check_ws(void *ws, size_t have, size_t need)
 {
     if (need == 0) return HILS_OK;
@@ -87,12 +94,12 @@ hils_status check_ws(void *ws, size_t have, size_t need)
 hils_status do_select(const Dims &p, hils_dtype in, const void *Q, const void *L, int32_t *sel_idx,
                       float *sel_score, void *ws, cudaStream_t s)
 {
-    if (p.N == 1) {
-        DeviceCtl ctl;
-        hils_status st = device_ctl(&ctl);
-        if (st != HILS_OK) return st;
-        return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, ctl, s));
-    }
+    DeviceCtl ctl;
+    hils_status st = device_ctl(&ctl);
+    if (st != HILS_OK) return st;
+    if (p.N == 1) return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, ctl, s));
+    if (!force_cuda_cores() && select_tc_supported(p, in))
+        return from_cuda(launch_select_prefill_tc(p, Q, L, sel_idx, sel_score, ctl, s));
     return from_cuda(launch_select_prefill(p, in, Q, L, sel_idx, sel_score, s));
 }
 
@@ -110,14 +117,11 @@ hils_status do_attend(const Dims &p, hils_dtype in, hils_dtype out, const void *
 }  // namespace
 
 // Prefill dispatch: the tensor-core kernel when it covers the shape, else CUDA cores.
-// HILS_PREFILL_KERNEL=simt forces the CUDA-core kernel (used to cross-check the two).
 cudaError_t launch_attend_prefill(const Dims &p, hils_dtype in, hils_dtype out, const void *Q, const void *K,
                                   const void *V, const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
                                   const DeviceCtl &ctl, cudaStream_t s)
 {
-    const char *force = getenv("HILS_PREFILL_KERNEL");
-    const bool simt = force && strcmp(force, "simt") == 0;
-    if (!simt && attend_tc_supported(p, in))
+    if (!force_cuda_cores() && attend_tc_supported(p, in))
         return launch_attend_prefill_tc(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s);
     return launch_attend_prefill_simt(p, in, out, Q, K, V, sel_idx, sel_score, O, s);
 }

@@ -49,6 +49,7 @@ constexpr int kD = 128;           // d
 constexpr uint32_t kTmemCols = 512;   // S0, S1 (64 each), O (128), P0, P1 (32 each)
 constexpr uint32_t kColO = 128, kColP = 256;
 constexpr unsigned long long kDrainNs = 2000000000ull;
+constexpr int kPolyEvery = 4;     // share of exponentials computed by exp2_poly: 1 in kPolyEvery
 
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 64, false, false);   // S = Q K^T, bf16, both K-major
 constexpr uint32_t IDESC_PV = idesc_f16_f32(128, 128, false, true);    // O += P V, f16, V MN-major
@@ -380,9 +381,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float ls[8];
 #pragma unroll
                 for (int a = 0; a < 8; ++a) ls[a] = 0.f;
+                // one exponential in kPolyEvery on the FMA pipe, the rest on the special-function unit
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
-                    const float e = (j < n_vis) ? ex2_approx(fmaf(__uint_as_float(sv[j]), sl2, nb)) : 0.f;
+                    const float x = fmaf(__uint_as_float(sv[j]), sl2, nb);
+                    const float ex = (j % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x) : ex2_approx(x);
+                    const float e = (j < n_vis) ? ex : 0.f;
                     sv[j] = __float_as_uint(e);
                     ls[j & 7] += e;
                 }

@@ -1,0 +1,327 @@
+// select_prefill_tc.cu -- landmark scoring and top-k chunk selection on the sm_100a tensor cores
+// (bf16 in, d = 128).
+//
+// "Hierarchical Sparse Attention Done Right" (arXiv 2607.02980v1), Sec. 3
+// Methodology, "Sparse training": every query scores all chunk summaries and
+// keeps the top-K; Sec. 4, "Architecture": under GQA the group's heads share one
+// selection.
+//
+// One CTA owns 128 rows = (128 / G) queries x the G heads of one kv-group, laid
+// out query-major (row r = query * G + head) so that a query's heads sit in G
+// adjacent lanes of one warp.  It streams the landmarks of chunks 0 .. c_hi in
+// tiles of 64 through shared memory (TMA, 128-byte swizzle, no multicast) and
+// computes every per-head score with one tcgen05.mma per tile:
+//   S[row, c] = q_{query, head} . L_c      (bf16 products, f32 accumulation)
+// into a double-buffered TMEM tile.  Four epilogue warps (one thread per row)
+// read S, form the group score mean_h(scale * S) with a butterfly over the G
+// lanes, and keep a per-row binary min-heap of the k best (group score, chunk)
+// keys; each row carries its own head's score as the heap payload, so the
+// per-head slot scores come out of the same pass.  Ties go to the lower chunk
+// index through the key order.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace hils {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 192;
+constexpr int kRows = 128;
+constexpr int kD = 128;
+constexpr int kTile = 64;                 // landmarks per tile
+constexpr uint32_t kTileBytes = kTile * kD * 2;
+constexpr uint32_t kTmemCols = 128;       // two 64-column score buffers
+constexpr unsigned long long kDrainNs = 2000000000ull;
+constexpr uint32_t IDESC = idesc_bf16_f32(128, kTile, false, false);
+
+struct Layout {
+    uint32_t q, l, bar, misc, keys, pay, own, total;
+};
+
+__host__ __device__ inline Layout make_layout(int k, int nsl)
+{
+    Layout L;
+    L.q = 0;
+    L.l = 32768;
+    L.bar = L.l + (uint32_t)nsl * kTileBytes;
+    L.misc = L.bar + 32 * 8;
+    L.keys = L.misc + 16;                                   // 8-byte aligned
+    L.pay = L.keys + 8u * (uint32_t)k * kRows;
+    L.own = L.pay + 4u * (uint32_t)k * kRows;
+    L.total = L.own + 4u * kRows;
+    return L;
+}
+
+__device__ __noinline__ void sift_down_p(uint64_t *h, float *pl, int n, uint64_t x, float xp)
+{
+    int e = 0;
+    for (;;) {
+        const int l = 2 * e + 1;
+        if (l >= n) break;
+        const int r = l + 1;
+        const int m = (r < n && h[r * kRows] < h[l * kRows]) ? r : l;
+        const uint64_t hm = h[m * kRows];
+        if (hm >= x) break;
+        h[e * kRows] = hm;
+        pl[e * kRows] = pl[m * kRows];
+        e = m;
+    }
+    h[e * kRows] = x;
+    pl[e * kRows] = xp;
+}
+
+template <int G, int NSL>
+__global__ void __launch_bounds__(kThreads, 1)
+    select_tc_kernel(const __grid_constant__ CUtensorMap tmL, Dims p, const __nv_bfloat16 *__restrict__ Q,
+                     int32_t *__restrict__ sel_idx, float *__restrict__ sel_score, unsigned int *status,
+                     unsigned long long limit_ns)
+{
+    constexpr int BQ = kRows / G;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    const Layout Ly = make_layout(p.k, NSL);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q0 = blockIdx.x * BQ, g = blockIdx.y, b = blockIdx.z;
+    const int nq = min(BQ, p.N - q0);
+    const int c_hi = (int)(((long long)p.q_offset + q0 + nq - 1) / p.C);   // own chunk of the last query
+    const int n_tiles = c_hi / kTile + 1;
+
+    const uint32_t sQ = smem_addr(base + Ly.q), sL = smem_addr(base + Ly.l), bar0 = smem_addr(base + Ly.bar);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + Ly.misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 8);
+    uint64_t *keys = reinterpret_cast<uint64_t *>(base + Ly.keys);
+    float *pay = reinterpret_cast<float *>(base + Ly.pay);
+    float *own_s = reinterpret_cast<float *>(base + Ly.own);
+    auto L_FULL = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+    auto L_EMPTY = [&](int s) { return bar0 + 8u * (uint32_t)(NSL + s); };
+    auto S_FULL = [&](int s) { return bar0 + 8u * (uint32_t)(2 * NSL + s); };
+    auto S_FREE = [&](int s) { return bar0 + 8u * (uint32_t)(2 * NSL + 2 + s); };
+    const uint32_t MMA_DONE = bar0 + 8u * (uint32_t)(2 * NSL + 4);
+
+    if (tid == 0) {
+        for (int s = 0; s < NSL; ++s) {
+            mbar_init(L_FULL(s), 1);
+            mbar_init(L_EMPTY(s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(S_FULL(s), 1);
+            mbar_init(S_FREE(s), 4);
+        }
+        mbar_init(MMA_DONE, 1);
+        fence_mbar_init();
+        *abort_flag = 0;
+        prefetch_tensormap(&tmL);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_holder), kTmemCols);
+        tmem_relinquish();
+    }
+    for (int e = tid; e < p.k * kRows; e += kThreads) keys[e] = 0ull;
+    // stage Q query-major in the 128-byte-swizzled K-major layout the MMA reads:
+    // row r = query * G + head, two 64-column halves of 128 rows x 128 bytes
+    for (int e = tid; e < kRows * 16; e += kThreads) {
+        const int r = e >> 4, half = (e >> 3) & 1, j = e & 7;
+        const int qi = r / G, h = r % G;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (qi < nq)
+            v = __ldg(reinterpret_cast<const uint4 *>(
+                Q + ((((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi) * kD + half * 64 + j * 8));
+        *reinterpret_cast<uint4 *>(base + Ly.q + half * 16384u + (uint32_t)r * 128u + ((j ^ (r & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const int row0 = (b * p.Hkv + g) * p.nL;
+            int next = 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                bool ok = true;
+                while (next < n_tiles && (next < NSL || next <= t + NSL - 1)) {
+                    const int st = next % NSL;
+                    if (next >= NSL &&
+                        !mbar_wait(L_EMPTY(st), (uint32_t)(((next / NSL) - 1) & 1), limit_ns, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t dst = sL + (uint32_t)st * kTileBytes;
+                    mbar_arrive_expect_tx(L_FULL(st), kTileBytes);
+                    tma_load_2d(dst, &tmL, L_FULL(st), 0, row0 + next * kTile);
+                    tma_load_2d(dst + kTileBytes / 2, &tmL, L_FULL(st), 64, row0 + next * kTile);
+                    ++next;
+                }
+                if (!ok) break;
+                const int st = t % NSL;
+                if (!mbar_wait(L_FULL(st), (uint32_t)((t / NSL) & 1), limit_ns, abort_flag, status)) break;
+                if (t >= 2 && !mbar_wait(S_FREE(t & 1), (uint32_t)(((t >> 1) - 1) & 1), limit_ns, abort_flag, status))
+                    break;
+                tc_fence_after();
+                const uint32_t la = sL + (uint32_t)st * kTileBytes;
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16_ss(tmem + (uint32_t)(t & 1) * kTile,
+                                smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
+                                smem_desc_sw128(la + (s >> 2) * (kTileBytes / 2) + (s & 3) * 32u, 16, 1024), IDESC,
+                                s > 0 ? 1u : 0u);
+                mma_commit(S_FULL(t & 1));
+                mma_commit(L_EMPTY(st));
+            }
+            mma_commit(MMA_DONE);
+            mbar_drain(MMA_DONE, 0, kDrainNs);
+            for (int u = max(0, next - NSL); u < next; ++u)
+                mbar_drain(L_FULL(u % NSL), (uint32_t)((u / NSL) & 1), kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp >= 2) {
+        const int qq = warp & 3;
+        const int r = 32 * qq + lane, qi = r / G, h = r % G;
+        const bool valid = qi < nq;
+        const long long pos = (long long)p.q_offset + q0 + qi;
+        const int ci = (int)(pos / p.C);
+        const float sc_g = p.scale / (float)G;
+        const uint32_t trow = tmem + ((uint32_t)(32 * qq) << 16);
+        uint64_t *hk = keys + r;
+        float *hp = pay + r;
+        float own = -INFINITY;
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            int w_ok = 1;
+            if (lane == 0) w_ok = mbar_wait(S_FULL(t & 1), (uint32_t)((t >> 1) & 1), limit_ns, abort_flag, status);
+            if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sv[64];
+            tmem_ld32(trow + (uint32_t)(t & 1) * kTile, sv);
+            tmem_ld32(trow + (uint32_t)(t & 1) * kTile + 32u, sv + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(S_FREE(t & 1));
+            const int c0 = t * kTile;
+#pragma unroll
+            for (int j = 0; j < kTile; ++j) {
+                const float s = __uint_as_float(sv[j]);
+                float gs = s;
+#pragma unroll
+                for (int o = 1; o < G; o <<= 1) gs += __shfl_xor_sync(0xFFFFFFFFu, gs, o);
+                const int c = c0 + j;
+                if (valid && c < ci && p.k > 0) {
+                    const uint64_t key = make_key(gs * sc_g, c);
+                    if (key > hk[0]) sift_down_p(hk, hp, p.k, key, s * p.scale);
+                }
+                if (c == ci) own = s * p.scale;
+            }
+        }
+        if (ok && valid) {
+            // heap sort: slots 0..k-1 end in descending key order
+            for (int n = p.k; n > 1; --n) {
+                const uint64_t top = hk[0];
+                const float topp = hp[0];
+                sift_down_p(hk, hp, n - 1, hk[(n - 1) * kRows], hp[(n - 1) * kRows]);
+                hk[(n - 1) * kRows] = top;
+                hp[(n - 1) * kRows] = topp;
+            }
+            const size_t row_g = (((size_t)b * p.Hkv + g) * p.N) + q0 + qi;
+            const size_t row_h = (((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi;
+            const int ns = p.k + 1;
+            if (h == 0)
+                for (int j = 0; j < p.k; ++j) sel_idx[row_g * p.k + j] = key_index(hk[j * kRows]);
+            for (int j = 0; j < p.k; ++j) sel_score[row_h * ns + j] = hk[j * kRows] ? hp[j * kRows] : -INFINITY;
+            sel_score[row_h * ns + p.k] = own;
+        }
+        (void)own_s;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+int stages_for(int k) { return k <= 32 ? 2 : 4; }
+
+template <int G>
+cudaError_t launch_g(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
+                     const DeviceCtl &ctl, cudaStream_t s)
+{
+    constexpr int BQ = kRows / G;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    CUtensorMap tl;
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)p.B * p.Hkv * p.nL};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+    const cuuint32_t es[2] = {1, 1};
+    if (fn(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(L), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const int nsl = stages_for(p.k);
+    const size_t smem = make_layout(p.k, nsl).total + 1024;
+    dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
+    cudaError_t e;
+    if (nsl == 2) {
+        auto kern = select_tc_kernel<G, 2>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kThreads, smem, s>>>(tl, p, static_cast<const __nv_bfloat16 *>(Q), sel_idx, sel_score,
+                                          ctl.status, (unsigned long long)ctl.wait_limit);
+    } else {
+        auto kern = select_tc_kernel<G, 4>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kThreads, smem, s>>>(tl, p, static_cast<const __nv_bfloat16 *>(Q), sel_idx, sel_score,
+                                          ctl.status, (unsigned long long)ctl.wait_limit);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool select_tc_supported(const Dims &p, hils_dtype in)
+{
+    if (in != HILS_BF16 || p.d != kD || p.N < 2) return false;
+    if (p.G != 1 && p.G != 2 && p.G != 4 && p.G != 8 && p.G != 16) return false;
+    return make_layout(p.k, stages_for(p.k)).total + 1024 <= 227 * 1024;
+}
+
+cudaError_t launch_select_prefill_tc(const Dims &p, const void *Q, const void *L, int32_t *sel_idx,
+                                     float *sel_score, const DeviceCtl &ctl, cudaStream_t s)
+{
+    switch (p.G) {
+    case 1: return launch_g<1>(p, Q, L, sel_idx, sel_score, ctl, s);
+    case 2: return launch_g<2>(p, Q, L, sel_idx, sel_score, ctl, s);
+    case 4: return launch_g<4>(p, Q, L, sel_idx, sel_score, ctl, s);
+    case 8: return launch_g<8>(p, Q, L, sel_idx, sel_score, ctl, s);
+    default: return launch_g<16>(p, Q, L, sel_idx, sel_score, ctl, s);
+    }
+}
+
+}  // namespace hils

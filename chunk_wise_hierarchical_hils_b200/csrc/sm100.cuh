@@ -58,6 +58,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Same test, but the thread may sleep up to hint_ns while the phase is pending
+// (it wakes when the phase completes), so waiting threads do not spin on the
+// issue slots the working warps need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: returns false (and raises the CTA's abort flag and the device
 // status) when the phase has not completed within limit_ns.  It also returns
 // false once another role of the CTA aborted, or once any CTA recorded a
@@ -69,16 +85,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
     for (unsigned int poll = 0;; ++poll) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
         if (*abort_flag) return false;
-        if ((poll & 255u) == 255u && *reinterpret_cast<volatile unsigned int *>(status) != 0u) {
-            *abort_flag = 1;
-            return false;
-        }
-        if (global_timer_ns() - t0 > limit_ns) {
-            *abort_flag = 1;
-            atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
-            return false;
+        if ((poll & 7u) == 7u) {
+            if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
+                *abort_flag = 1;
+                return false;
+            }
+            if (global_timer_ns() - t0 > limit_ns) {
+                *abort_flag = 1;
+                atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
+                return false;
+            }
         }
     }
 }
@@ -208,6 +226,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
 }
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x for x <= 0 on the FMA and integer pipes: x = n + f with n = rint(x) (the
+// 1.5 * 2^23 rounding trick), 2^f from a degree-4 polynomial on [-1/2, 1/2]
+// (coefficients fitted for this library by weighted least squares on Chebyshev
+// nodes; relative error 3.1e-6 in float32), 2^n added to the exponent bits.
+// Inputs below -125 are clamped there (the result, < 3e-38, is then rounded
+// away by the f16 probabilities anyway).
+__device__ __forceinline__ float exp2_poly(float x)
+{
+    x = fmaxf(x, -125.0f);
+    const float magic = 12582912.0f;
+    const float t = x + magic;
+    const float f = x - (t - magic);
+    const int n = __float_as_int(t) - __float_as_int(magic);
+    const float p = fmaf(fmaf(fmaf(fmaf(0.0096003953f, f, 0.055916894f), f, 0.24023719f), f, 0.69312197f), f, 1.0f);
+    return __int_as_float(__float_as_int(p) + (n << 23));
+}
 
 // 2^x on the special-function unit (flushes subnormal results to zero)
 __device__ __forceinline__ float ex2_approx(float x)

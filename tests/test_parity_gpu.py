@@ -33,6 +33,8 @@ CASES = [
     wl("g16", H=16, Hkv=1, N=200, T=200, k=3, seed=108),
     wl("k64_max", H=2, Hkv=1, N=300, T=4200, q_offset=3900, C=32, k=64, seed=109, l_mode="iid"),
     wl("needles", B=1, H=8, Hkv=2, N=2048, T=2048, k=4, seed=110, l_mode="iid", n_needles=8, needle_period=128),
+    wl("g1_d128_long", B=1, H=2, Hkv=2, N=1200, T=9000, q_offset=7800, k=12, seed=111),
+    wl("g2_k32_c128", B=2, H=4, Hkv=2, N=700, T=4400, q_offset=3700, C=128, k=32, seed=112, l_mode="iid"),
 ]
 DECODE = [
     wl("decode_ragged_T", B=3, H=8, Hkv=2, N=1, T=1000, q_offset=999, k=4, seed=120),
@@ -58,7 +60,7 @@ def test_parity_small(w):
     _check(st)
 
 
-@pytest.mark.parametrize("w", [CASES[1], CASES[7], CASES[8], CASES[10]], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [CASES[1], CASES[7], CASES[8], CASES[10], CASES[11]], ids=lambda w: w.name)
 def test_cuda_core_kernel_too(w, monkeypatch):
     """The CUDA-core prefill kernel, forced, on shapes the tensor-core kernel normally takes."""
     monkeypatch.setenv("HILS_PREFILL_KERNEL", "simt")
