@@ -27,7 +27,7 @@ HILS_MAX_GROUP = 16
 EXPORTS = ("hils_status_string", "hils_version", "hils_validate", "hils_score_select_workspace_size",
            "hils_chunk_attend_fuse_workspace_size", "hils_forward_workspace_size", "hils_score_select",
            "hils_chunk_attend_fuse", "hils_forward", "hils_sync_status", "hils_set_wait_limit",
-           "hils_decode_score_select_noalloc")
+           "hils_decode_score_select_noalloc", "hils_debug_inject_stall")
 HILS_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -67,6 +67,7 @@ def _load():
     lib.hils_sync_status.argtypes = [vp]
     lib.hils_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.hils_decode_score_select_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
+    lib.hils_debug_inject_stall.argtypes = [ctypes.c_int]
     for n in EXPORTS[2:]:
         if n not in ("hils_status_string", "hils_version"):
             getattr(lib, n).restype = ctypes.c_int
@@ -170,13 +171,18 @@ def hils_set_wait_limit(ns):
     _check(_lib.hils_set_wait_limit(int(ns)), "hils_set_wait_limit")
 
 
+def hils_debug_inject_stall(on):
+    """Test control: tensor-core kernels wait once on a barrier nothing signals (their bounded wait expires)."""
+    _check(_lib.hils_debug_inject_stall(int(bool(on))), "hils_debug_inject_stall")
+
+
 def hils_decode_score_select_noalloc(p, Q, L, sel_idx, sel_score, stream=None):
     """hils_score_select for N == 1 with the library's fixed scratch: no workspace argument.
 
     For callers that cannot allocate device memory; see include/hils.h."""
     _check(_lib.hils_decode_score_select_noalloc(ctypes.byref(p), _ptr(Q), _ptr(L), _ptr(sel_idx),
                                                  _ptr(sel_score), _stream(stream)),
-           "hils_decode_score_select_noalloc")
+           "hils_decode_score_select_noalloc", "hils_debug_inject_stall")
 
 
 def problem(B, H, Hkv, N, T, d, C, k, q_offset=0, in_dtype=HILS_BF16, out_dtype=None, scale=0.0):

@@ -14,6 +14,7 @@ __device__ unsigned int g_status;   // device-side status word (one per device)
 
 constexpr long long kDefaultWaitLimit = 1000000000ll;   // ns of the GPU global timer: one second
 long long g_wait_limit = kDefaultWaitLimit;
+int g_inject_stall = 0;
 std::mutex g_mu;
 
 }  // namespace
@@ -32,6 +33,7 @@ hils_status device_ctl(DeviceCtl *ctl)
     }
     ctl->status = addr[dev];
     ctl->wait_limit = g_wait_limit;
+    ctl->inject_stall = g_inject_stall;
     return HILS_OK;
 }
 
@@ -259,6 +261,13 @@ hils_status hils_set_wait_limit(long long ns)
     if (ns < 0) return HILS_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lk(g_mu);
     g_wait_limit = ns == 0 ? kDefaultWaitLimit : ns;
+    return HILS_OK;
+}
+
+hils_status hils_debug_inject_stall(int on)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_inject_stall = on ? 1 : 0;
     return HILS_OK;
 }
 

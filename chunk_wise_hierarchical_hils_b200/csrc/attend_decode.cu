@@ -97,7 +97,7 @@ __global__ void attend_decode_kernel(Dims p, DecodePlan plan, const Tin *__restr
 
     float *mine = partial + (((size_t)bg * plan.nsplit2 + split) * p.G + warp) * D;
 #pragma unroll
-    for (int x = 0; x < D / 32; ++x) mine[lane + 32 * x] = acc[x];
+    for (int x = 0; x < D / 32; ++x) mine[lane * (D / 32) + x] = acc[x];
 
     __threadfence();
     __syncthreads();

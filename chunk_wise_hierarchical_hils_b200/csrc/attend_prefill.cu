@@ -60,7 +60,7 @@ __global__ void attend_prefill_simt_kernel(Dims p, const Tin *__restrict__ Q, co
         warp_attend_chunk<Tin, D>(qsm + warp * D, Ks, Vs, n_vis, wsm[warp * ns + j], acc);
     }
 #pragma unroll
-    for (int x = 0; x < D / 32; ++x) store_out(O + row_h * D + lane + 32 * x, acc[x]);
+    for (int x = 0; x < D / 32; ++x) store_out(O + row_h * D + lane * (D / 32) + x, acc[x]);
 }
 
 template <typename Tin, typename Tout, int D>

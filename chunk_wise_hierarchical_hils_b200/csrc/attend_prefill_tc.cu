@@ -46,8 +46,10 @@ constexpr int kThreads = 320;     // 10 warps
 constexpr int kRows = 128;        // MMA M
 constexpr int kChunk = 64;        // C
 constexpr int kD = 128;           // d
-constexpr uint32_t kTmemCols = 512;   // S0, S1 (64 each), O (128), P0, P1 (32 each)
-constexpr uint32_t kColO = 128, kColP = 256;
+constexpr int kSB = 4;                // S and P buffers: QK may run up to kSB chunks ahead of PV
+constexpr int kGroups = 2;            // softmax warp groups; group t % kGroups handles chunk t
+constexpr uint32_t kTmemCols = 512;   // S0..S3 (64 columns each), O (128), P0..P3 (32 each)
+constexpr uint32_t kColO = 256, kColP = 384;
 constexpr unsigned long long kDrainNs = 2000000000ull;
 constexpr int kPolyEvery = 4;     // share of exponentials computed by exp2_poly: 1 in kPolyEvery
 
@@ -82,8 +84,9 @@ __host__ __device__ inline Layout make_layout(int k, int nwords, int BQ)
 // barrier slots
 template <int NS>
 struct Bars {
-    static constexpr int Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + NS, S_FULL = 1 + 2 * NS, P_FULL = 3 + 2 * NS,
-                         P_EMPTY = 5 + 2 * NS, O_FULL = 7 + 2 * NS, MMA_DONE = 8 + 2 * NS;
+    static constexpr int Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + NS, S_FULL = 1 + 2 * NS,
+                         P_FULL = 1 + 2 * NS + kSB, P_EMPTY = 1 + 2 * NS + 2 * kSB, O_FULL = 1 + 2 * NS + 3 * kSB,
+                         MMA_DONE = 2 + 2 * NS + 3 * kSB;
 };
 
 __device__ __forceinline__ void store_row32(float *dst, const uint32_t *v)
@@ -126,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, Dims p, const int32_t *__restrict__ sel_idx,
                      const float *__restrict__ sel_score, Tout *__restrict__ O, unsigned int *status,
-                     unsigned long long limit_ns, int nwords)
+                     unsigned long long limit_ns, int nwords, int inject_stall)
 {
     constexpr int BQ = kRows / G;
     using BR = Bars<NS>;
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(BAR(BR::KV_FULL + s), 1);
             mbar_init(BAR(BR::KV_EMPTY + s), 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kSB; ++s) {
             mbar_init(BAR(BR::S_FULL + s), 1);
             mbar_init(BAR(BR::P_FULL + s), 4);
             mbar_init(BAR(BR::P_EMPTY + s), 1);
@@ -262,75 +265,98 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA + MMA issue --------------------------------
+            // One thread drives both async engines.  It never blocks on one event while
+            // another could proceed: each pass tests (without waiting) whether a load, a QK
+            // product or a PV product can be issued, and issues it.  QK runs up to kSB
+            // chunks ahead of PV, loads up to NS chunks ahead.
             const int kv_row0 = (b * p.Hkv + g) * p.T;
-            int next_load = 0;
-            bool ok = true;
+            int next_load = 0, next_qk = 0, next_pv = 0;
+            bool q_ready = false;
             mbar_arrive_expect_tx(BAR(BR::Q_FULL), 32768u);
             tma_load_3d(sQ, &tmQ, BAR(BR::Q_FULL), 0, q0, b * p.H + g * G);
             tma_load_3d(sQ + 16384u, &tmQ, BAR(BR::Q_FULL), 64, q0, b * p.H + g * G);
-
-            auto issue_pv = [&](int u) -> bool {
-                if (!mbar_wait(BAR(BR::P_FULL + (u & 1)), (u >> 1) & 1, limit_ns, abort_flag, status)) return false;
-                tc_fence_after();
-                const uint32_t st = (uint32_t)(u % NS);
-                const uint32_t pa = tmem + kColP + (uint32_t)(u & 1) * 32u;
-                const uint32_t va = sKV + st * 32768u + 16384u;
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_f16_ts(tmem + kColO, pa + 8u * s, smem_desc_sw128(va + 2048u * s, 8192, 1024), IDESC_PV,
-                               (u > 0 || s > 0) ? 1u : 0u);
-                mma_commit(BAR(BR::KV_EMPTY + (int)st));
-                mma_commit(BAR(BR::P_EMPTY + (u & 1)));
-                return true;
-            };
-
-            for (int t = 0; t < n_union && ok; ++t) {
-                while (next_load < n_union && (next_load < NS || next_load <= t + NS - 2)) {
+            if (inject_stall) {
+                // test control: wait once on a barrier nothing signals, so the bounded wait expires
+                mbar_wait(BAR(BR::MMA_DONE), 0, limit_ns, abort_flag, status);
+            }
+            unsigned long long idle_since = 0ull;
+            while (next_pv < n_union && !*abort_flag) {
+                bool prog = false;
+                if (next_load < n_union && next_load < next_pv + NS) {
                     const int u = next_load, st = u % NS;
-                    if (u >= NS &&
-                        !mbar_wait(BAR(BR::KV_EMPTY + st), ((u / NS) - 1) & 1, limit_ns, abort_flag, status)) {
-                        ok = false;
-                        break;
+                    if (u < NS || mbar_test(BAR(BR::KV_EMPTY + st), (uint32_t)(((u / NS) - 1) & 1))) {
+                        const int row = kv_row0 + uni[u] * kChunk;
+                        const uint32_t dst = sKV + (uint32_t)st * 32768u;
+                        mbar_arrive_expect_tx(BAR(BR::KV_FULL + st), 32768u);
+                        tma_load_2d(dst, &tmK, BAR(BR::KV_FULL + st), 0, row);
+                        tma_load_2d(dst + 8192u, &tmK, BAR(BR::KV_FULL + st), 64, row);
+                        tma_load_2d(dst + 16384u, &tmV, BAR(BR::KV_FULL + st), 0, row);
+                        tma_load_2d(dst + 24576u, &tmV, BAR(BR::KV_FULL + st), 64, row);
+                        ++next_load;
+                        prog = true;
                     }
-                    const int row = kv_row0 + uni[u] * kChunk;
-                    const uint32_t dst = sKV + (uint32_t)st * 32768u;
-                    mbar_arrive_expect_tx(BAR(BR::KV_FULL + st), 32768u);
-                    tma_load_2d(dst, &tmK, BAR(BR::KV_FULL + st), 0, row);
-                    tma_load_2d(dst + 8192u, &tmK, BAR(BR::KV_FULL + st), 64, row);
-                    tma_load_2d(dst + 16384u, &tmV, BAR(BR::KV_FULL + st), 0, row);
-                    tma_load_2d(dst + 24576u, &tmV, BAR(BR::KV_FULL + st), 64, row);
-                    ++next_load;
                 }
-                if (!ok) break;
-                const int st = t % NS;
-                if (!mbar_wait(BAR(BR::KV_FULL + st), (t / NS) & 1, limit_ns, abort_flag, status)) break;
-                if (t == 0 && !mbar_wait(BAR(BR::Q_FULL), 0, limit_ns, abort_flag, status)) break;
-                tc_fence_after();
-                // S buffer t % 2 is free: its previous chunk's P was consumed by a PV issued earlier,
-                // and that group had read S before writing P
-                const uint32_t d_s = tmem + (uint32_t)(t & 1) * 64u;
-                const uint32_t ka = sKV + (uint32_t)st * 32768u;
+                if (next_qk < next_load && next_qk < next_pv + kSB) {
+                    if (!q_ready) q_ready = mbar_test(BAR(BR::Q_FULL), 0);
+                    const int t = next_qk, st = t % NS;
+                    if (q_ready && mbar_test(BAR(BR::KV_FULL + st), (uint32_t)((t / NS) & 1))) {
+                        tc_fence_after();
+                        // S buffer t % kSB is free: QK(t - kSB)'s chunk was softmaxed before its PV,
+                        // which was issued before this point (next_pv > t - kSB)
+                        const uint32_t d_s = tmem + (uint32_t)(t % kSB) * 64u;
+                        const uint32_t ka = sKV + (uint32_t)st * 32768u;
 #pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16_ss(d_s, smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
-                                smem_desc_sw128(ka + (s >> 2) * 8192u + (s & 3) * 32u, 16, 1024), IDESC_QK,
-                                s > 0 ? 1u : 0u);
-                mma_commit(BAR(BR::S_FULL + (t & 1)));
-                if (t >= 1 && !issue_pv(t - 1)) break;
-                if (t == n_union - 1) {
-                    if (issue_pv(t)) mma_commit(BAR(BR::O_FULL));
+                        for (int s = 0; s < 8; ++s)
+                            mma_bf16_ss(d_s, smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
+                                        smem_desc_sw128(ka + (s >> 2) * 8192u + (s & 3) * 32u, 16, 1024), IDESC_QK,
+                                        s > 0 ? 1u : 0u);
+                        mma_commit(BAR(BR::S_FULL + t % kSB));
+                        ++next_qk;
+                        prog = true;
+                    }
+                }
+                if (next_pv < next_qk) {
+                    const int u = next_pv;
+                    if (mbar_test(BAR(BR::P_FULL + u % kSB), (uint32_t)((u / kSB) & 1))) {
+                        tc_fence_after();
+                        const uint32_t st = (uint32_t)(u % NS);
+                        const uint32_t pa = tmem + kColP + (uint32_t)(u % kSB) * 32u;
+                        const uint32_t va = sKV + st * 32768u + 16384u;
+#pragma unroll
+                        for (int s = 0; s < 4; ++s)
+                            mma_f16_ts(tmem + kColO, pa + 8u * s, smem_desc_sw128(va + 2048u * s, 8192, 1024),
+                                       IDESC_PV, (u > 0 || s > 0) ? 1u : 0u);
+                        mma_commit(BAR(BR::KV_EMPTY + (int)st));
+                        mma_commit(BAR(BR::P_EMPTY + u % kSB));
+                        ++next_pv;
+                        prog = true;
+                    }
+                }
+                if (prog) {
+                    idle_since = 0ull;
+                } else {
+                    const unsigned long long now = global_timer_ns();
+                    if (!idle_since) idle_since = now;
+                    if (now - idle_since > limit_ns) {
+                        *abort_flag = 1;
+                        atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
+                    } else if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
+                        *abort_flag = 1;
+                    }
+                    __nanosleep(32);
                 }
             }
+            if (!*abort_flag) mma_commit(BAR(BR::O_FULL));
             // drain: every issued MMA, then the latest load of every stage and Q
             mma_commit(BAR(BR::MMA_DONE));
             mbar_drain(BAR(BR::MMA_DONE), 0, kDrainNs);
             for (int u = max(0, next_load - NS); u < next_load; ++u)
-                mbar_drain(BAR(BR::KV_FULL + u % NS), (u / NS) & 1, kDrainNs);
+                mbar_drain(BAR(BR::KV_FULL + u % NS), (uint32_t)((u / NS) & 1), kDrainNs);
             mbar_drain(BAR(BR::Q_FULL), 0, kDrainNs);
         }
         __syncwarp();
     } else if (warp >= 2) {
-        // ---------------- softmax (two groups, alternate chunks) and epilogue ----
+        // ---------------- softmax (kGroups groups, alternate chunks) and epilogue ----
         const int grp = (warp - 2) >> 2;
         const int qq = warp & 3;
         const int r = 32 * qq + lane, h = r / BQ, qi = r % BQ;
@@ -342,18 +368,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float *wr = wts + r * ns;
         const float sl2 = p.scale * 1.4426950408889634f;
         const uint32_t lane_off = (uint32_t)(32 * qq) << 16;
-        const uint32_t tS = tmem + lane_off + (uint32_t)grp * 64u;
-        const uint32_t tP = tmem + lane_off + kColP + (uint32_t)grp * 32u;
         int ptr = 0;
         bool ok = true;
-        for (int t = grp; t < n_union; t += 2) {
-            const int u = t >> 1;
-            if (!warp_wait(BAR(BR::S_FULL + grp), (uint32_t)(u & 1), limit_ns, abort_flag, status)) {
+        for (int t = grp; t < n_union; t += kGroups) {
+            const int bsel = t % kSB, u = t / kSB;
+            if (!warp_wait(BAR(BR::S_FULL + bsel), (uint32_t)(u & 1), limit_ns, abort_flag, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             uint32_t sv[64];
+            const uint32_t tS = tmem + lane_off + (uint32_t)bsel * 64u;
             tmem_ld32(tS, sv);
             tmem_ld32(tS + 32u, sv + 32);
             tmem_wait_ld();
@@ -364,29 +389,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[32];
             if (w > 0.f) {
                 const int n_vis = (c == own) ? (int)(pos - (long long)c * kChunk + 1) : kChunk;
-                float mx[8];
-#pragma unroll
-                for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
-                if (n_vis == kChunk) {
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sv[j]));
-                } else {
+                if (n_vis < kChunk) {
 #pragma unroll
                     for (int j = 0; j < 64; ++j)
-                        if (j < n_vis) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sv[j]));
+                        if (j >= n_vis) sv[j] = __float_as_uint(-INFINITY);
                 }
+                float mx[8];
+#pragma unroll
+                for (int a = 0; a < 8; ++a) mx[a] = __uint_as_float(sv[a]);
+#pragma unroll
+                for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sv[j]));
                 const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
                 const float nb = -m * sl2;
                 float ls[8];
 #pragma unroll
                 for (int a = 0; a < 8; ++a) ls[a] = 0.f;
-                // one exponential in kPolyEvery on the FMA pipe, the rest on the special-function unit
+                // one exponential in kPolyEvery on the FMA pipe, the rest on the special-function unit;
+                // masked keys hold -inf and give 0 either way
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     const float x = fmaf(__uint_as_float(sv[j]), sl2, nb);
-                    const float ex = (j % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x) : ex2_approx(x);
-                    const float e = (j < n_vis) ? ex : 0.f;
+                    const float e = (j % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x) : ex2_approx(x);
                     sv[j] = __float_as_uint(e);
                     ls[j & 7] += e;
                 }
@@ -401,16 +425,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) pk[j] = 0u;
             }
-            if (u >= 1 &&
-                !warp_wait(BAR(BR::P_EMPTY + grp), (uint32_t)((u - 1) & 1), limit_ns, abort_flag, status)) {
+            if (t >= kSB &&
+                !warp_wait(BAR(BR::P_EMPTY + bsel), (uint32_t)((u - 1) & 1), limit_ns, abort_flag, status)) {
                 ok = false;
                 break;
             }
-            tmem_st32(tP, pk);
+            tmem_st32(tmem + lane_off + kColP + (uint32_t)bsel * 32u, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(BR::P_FULL + grp));
+            if (lane == 0) mbar_arrive(BAR(BR::P_FULL + bsel));
         }
         if (ok && warp_wait(BAR(BR::O_FULL), 0, limit_ns, abort_flag, status)) {
             tc_fence_after();
@@ -508,7 +532,7 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V,
     if (e != cudaSuccess) return e;
     dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
     kern<<<grid, kThreads, smem, s>>>(tq, tk, tv, p, sel_idx, sel_score, static_cast<Tout *>(O), ctl.status,
-                                      (unsigned long long)ctl.wait_limit, nwords);
+                                      (unsigned long long)ctl.wait_limit, nwords, ctl.inject_stall);
     return cudaGetLastError();
 }
 

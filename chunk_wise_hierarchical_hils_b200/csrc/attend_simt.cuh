@@ -46,13 +46,40 @@ __device__ __forceinline__ float dot_rotated(const float *qsm, const Tin *krow, 
     return a0 + a1;
 }
 
-// acc[x] (element lane + 32 x of the head's output) += coef * o_c, where o_c is
-// the softmax-weighted mean of the staged value rows over the n_vis visible
+// Load EPL = D/32 consecutive elements of a staged row as float (8 or 16 bytes per lane).
+template <int EPL>
+__device__ __forceinline__ void lds_epl(const __nv_bfloat16 *p, float *o)
+{
+    if constexpr (EPL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        o[0] = __uint_as_float(u.x << 16); o[1] = __uint_as_float(u.x & 0xFFFF0000u);
+        o[2] = __uint_as_float(u.y << 16); o[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+        o[0] = __uint_as_float(u << 16); o[1] = __uint_as_float(u & 0xFFFF0000u);
+    }
+}
+
+template <int EPL>
+__device__ __forceinline__ void lds_epl(const float *p, float *o)
+{
+    if constexpr (EPL == 4) {
+        const float4 u = *reinterpret_cast<const float4 *>(p);
+        o[0] = u.x; o[1] = u.y; o[2] = u.z; o[3] = u.w;
+    } else {
+        const float2 u = *reinterpret_cast<const float2 *>(p);
+        o[0] = u.x; o[1] = u.y;
+    }
+}
+
+// acc[x] (element lane * D/32 + x of the head's output) += coef * o_c, where o_c
+// is the softmax-weighted mean of the staged value rows over the n_vis visible
 // tokens (n_vis <= 128).
 template <typename Tin, int D>
 __device__ __forceinline__ void warp_attend_chunk(const float *qsm, const Tin *Ks, const Tin *Vs, int n_vis,
                                                   float coef, float *acc)
 {
+    constexpr int EPL = D / 32;
     const int lane = threadIdx.x & 31;
     float lg[4];
 #pragma unroll
@@ -68,9 +95,9 @@ __device__ __forceinline__ void warp_attend_chunk(const float *qsm, const Tin *K
         sum += e[m];
     }
     sum = warp_sum(sum);
-    float oc[D / 32];
+    float oc[EPL];
 #pragma unroll
-    for (int x = 0; x < D / 32; ++x) oc[x] = 0.f;
+    for (int x = 0; x < EPL; ++x) oc[x] = 0.f;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         if (32 * m >= n_vis) break;
@@ -79,15 +106,16 @@ __device__ __forceinline__ void warp_attend_chunk(const float *qsm, const Tin *K
             const int t = 32 * m + tt;
             const float pt = __shfl_sync(0xFFFFFFFFu, e[m], tt);
             if (t < n_vis) {
-                const Tin *vr = Vs + (size_t)t * D;
+                float v[EPL];
+                lds_epl<EPL>(Vs + (size_t)t * D + lane * EPL, v);
 #pragma unroll
-                for (int x = 0; x < D / 32; ++x) oc[x] = fmaf(pt, to_float(vr[lane + 32 * x]), oc[x]);
+                for (int x = 0; x < EPL; ++x) oc[x] = fmaf(pt, v[x], oc[x]);
             }
         }
     }
     const float c = coef / sum;
 #pragma unroll
-    for (int x = 0; x < D / 32; ++x) acc[x] = fmaf(c, oc[x], acc[x]);
+    for (int x = 0; x < EPL; ++x) acc[x] = fmaf(c, oc[x], acc[x]);
 }
 
 // Fusion weights of the slots [j0, j1) for one head: softmax over all ns slot

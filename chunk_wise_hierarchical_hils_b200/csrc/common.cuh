@@ -110,4 +110,93 @@ __device__ __forceinline__ void bitonic_sort_desc(uint64_t *a, int n)
     __syncthreads();
 }
 
+// ---- block-wide top-m of 64-bit keys ---------------------------------------
+// Writes the m largest of keys[0..n) to out[0..m) in descending order (out is
+// padded with 0 when fewer than m keys are real).  Real keys are distinct and
+// non-zero; zeros are padding.  MSB-first radix select over 8-bit digits: each
+// pass histograms the keys that share the current prefix, keeps the digit at
+// which the count from the top reaches the number still to take, and stops as
+// soon as that digit's whole group is taken.  The m survivors are then sorted.
+// Every thread of the block must call it.  hist: 256 unsigned; ctrl: 4 words.
+__device__ __forceinline__ void block_topk_desc(const uint64_t *keys, int n, int m, uint64_t *out,
+                                                unsigned int *hist, unsigned long long *ctrl)
+{
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
+    if (m <= 0) {
+        __syncthreads();
+        return;
+    }
+    int m_pow2 = 1;
+    while (m_pow2 < m) m_pow2 <<= 1;
+    // number of real keys
+    if (tid == 0) ctrl[3] = 0ull;
+    __syncthreads();
+    unsigned int real = 0;
+    for (int i = tid; i < n; i += nt) real += keys[i] != 0ull;
+    real = (unsigned)__reduce_add_sync(0xFFFFFFFFu, real);
+    if (lane == 0 && real) atomicAdd(&ctrl[3], (unsigned long long)real);
+    __syncthreads();
+    const int n_real = (int)ctrl[3];
+    unsigned long long prefix = 0ull, mask = 0ull;
+    if (n_real > m) {
+        unsigned int remaining = (unsigned)m;
+        for (int shift = 56; shift >= 0; shift -= 8) {
+            for (int i = tid; i < 256; i += nt) hist[i] = 0u;
+            __syncthreads();
+            for (int i = tid; i < n; i += nt) {
+                const uint64_t key = keys[i];
+                if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (tid < 32) {
+                // lane l owns digits 255-8l .. 248-8l (highest digits first)
+                unsigned int c[8], tot = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    c[e] = hist[255 - 8 * lane - e];
+                    tot += c[e];
+                }
+                unsigned int incl = tot;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                const unsigned int excl = incl - tot;   // keys in higher digits than this lane's
+                const unsigned int hit = __ballot_sync(0xFFFFFFFFu, excl < remaining && incl >= remaining);
+                if (lane == __ffs(hit) - 1) {
+                    unsigned int above = excl;
+                    int e = 0;
+                    while (above + c[e] < remaining) above += c[e++];
+                    const unsigned int d = 255u - 8u * lane - (unsigned)e;
+                    ctrl[0] = prefix | ((unsigned long long)d << shift);
+                    ctrl[1] = mask | (255ull << shift);
+                    ctrl[2] = ((unsigned long long)(remaining - above) << 32) | (unsigned long long)(c[e] == remaining - above);
+                }
+            }
+            __syncthreads();
+            prefix = ctrl[0];
+            mask = ctrl[1];
+            remaining = (unsigned)(ctrl[2] >> 32);
+            const bool done = (ctrl[2] & 1ull) != 0ull;
+            __syncthreads();
+            if (done) break;
+        }
+    }
+    // collect: higher prefix, or the boundary group (all of it when the loop stopped early,
+    // otherwise the single key equal to the full prefix)
+    if (tid == 0) ctrl[3] = 0ull;
+    for (int i = tid; i < m_pow2; i += nt) out[i] = 0ull;
+    __syncthreads();
+    for (int i = tid; i < n; i += nt) {
+        const uint64_t key = keys[i];
+        if (key != 0ull && (key & mask) >= prefix) {
+            const unsigned long long slot = atomicAdd(&ctrl[3], 1ull);
+            if (slot < (unsigned long long)m) out[slot] = key;
+        }
+    }
+    if (m_pow2 > 1) bitonic_sort_desc(out, m_pow2);
+    else __syncthreads();
+}
+
 }  // namespace hils

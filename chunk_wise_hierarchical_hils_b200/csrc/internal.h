@@ -21,7 +21,8 @@ struct Dims {
 // Device-side status shared by all kernels of the library.
 struct DeviceCtl {
     unsigned int *status;   // HILS_OK or HILS_ERR_TIMEOUT, sticky until read
-    long long wait_limit;   // polls before a bounded wait gives up
+    long long wait_limit;   // ns a bounded wait may take before it gives up
+    int inject_stall;       // test control: tensor-core kernels wait once on a barrier nothing signals
 };
 
 // Decode selection layout in the workspace.

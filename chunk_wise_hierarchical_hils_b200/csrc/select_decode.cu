@@ -38,9 +38,14 @@ __global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan pl
     extern __shared__ __align__(128) unsigned char smem_raw[];
     float *qs = reinterpret_cast<float *>(smem_raw);                              // [D]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + D * sizeof(float));  // [RING]
-    unsigned char *ring = smem_raw + D * sizeof(float) + 128;                      // [RING][STAGE_BYTES]
+    unsigned char *big = smem_raw + D * sizeof(float) + 128;
+    unsigned char *ring = big;                                                     // [RING][STAGE_BYTES]
     uint64_t *keys = reinterpret_cast<uint64_t *>(ring + RING * STAGE_BYTES);      // [spl]
-    uint64_t *mkeys = reinterpret_cast<uint64_t *>(ring);                          // merge reuses the ring
+    uint64_t *mkeys = reinterpret_cast<uint64_t *>(big);                           // merge reuses the ring
+    float *rows = reinterpret_cast<float *>(big);                                  // then: staged q and L rows
+    __shared__ unsigned int s_hist[256];
+    __shared__ unsigned long long s_ctrl[4];
+    __shared__ uint64_t s_top[HILS_MAX_K];
     __shared__ int s_last;
     __shared__ int s_abort;
 
@@ -121,14 +126,10 @@ __global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan pl
         for (int u = s_done; u < issued; ++u)
             mbar_drain(bar0 + 8u * (u % RING), (uint32_t)((u / RING) & 1), kDrainNs);
     }
-    int local_n = 1;
-    while (local_n < n_local) local_n <<= 1;
-    for (int e = n_local + tid; e < local_n; e += NT) keys[e] = 0ull;
-    if (n_local > 1) bitonic_sort_desc(keys, local_n);
-    else __syncthreads();
+    block_topk_desc(keys, n_local, min(p.k, max(n_local, 1)), s_top, s_hist, s_ctrl);
 
     uint64_t *mine = cand + ((size_t)bg * plan.nsplit + split) * p.k;
-    for (int j = tid; j < p.k; j += NT) mine[j] = (j < n_local) ? keys[j] : 0ull;
+    for (int j = tid; j < p.k; j += NT) mine[j] = (j < n_local) ? s_top[j] : 0ull;
 
     // ---- last split of this (b, g) merges --------------------------------
     __threadfence();
@@ -139,45 +140,59 @@ __global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan pl
     __threadfence();
 
     const int nm = plan.nsplit * p.k;
-    int merge_n = 1;
-    while (merge_n < nm) merge_n <<= 1;
     const uint64_t *all = cand + (size_t)bg * plan.nsplit * p.k;
-    for (int e = tid; e < merge_n; e += NT) mkeys[e] = (e < nm) ? __ldcg(all + e) : 0ull;
-    if (merge_n > 1) bitonic_sort_desc(mkeys, merge_n);
-    else __syncthreads();
+    for (int e = tid; e < nm; e += NT) mkeys[e] = __ldcg(all + e);
+    __syncthreads();
+    if (p.k > 0) block_topk_desc(mkeys, nm, p.k, s_top, s_hist, s_ctrl);
 
     int32_t *si = sel_idx + (size_t)bg * p.k;
-    for (int j = tid; j < p.k; j += NT) si[j] = key_index(mkeys[j]);
+    for (int j = tid; j < p.k; j += NT) si[j] = key_index(s_top[j]);
 
-    // per-head scores of the k slots and the own chunk: LPC lanes per (head, slot)
+    // per-head scores of the k slots and the own chunk: stage the group's query rows and the
+    // k+1 landmark rows in shared memory (all loads in flight at once), then one dot per thread
     const int ns = p.k + 1;
-    constexpr int TPW = 32 / LPC;   // tasks per warp step
-    for (int t0 = warp * TPW; t0 < p.G * ns; t0 += (NT / 32) * TPW) {
-        const int task = t0 + lane / LPC;
-        const bool live = task < p.G * ns;
-        const int h = live ? task / ns : 0, j = live ? task % ns : 0;
-        const int c = !live ? -1 : (j < p.k) ? key_index(mkeys[j]) : ci;
-        float acc = 0.f;
-        if (c >= 0) {
-            float qv8[8], lv8[8];
-            load8(Q + ((size_t)b * p.H + (size_t)g * p.G + h) * D + sub * 8, qv8);
-            load8(Lbg + (size_t)c * D + sub * 8, lv8);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) acc = fmaf(qv8[u], lv8[u], acc);
+    float *qrows = rows;                       // [G][D]
+    float *lrows = rows + (size_t)p.G * D;     // [ns][D]
+    for (int e = tid; e < (p.G + ns) * (D / 8); e += NT) {
+        const int rr = e / (D / 8), seg = e % (D / 8);
+        const Tin *src;
+        if (rr < p.G) {
+            src = Q + ((size_t)b * p.H + (size_t)g * p.G + rr) * D;
+        } else {
+            const int j = rr - p.G;
+            const int c = (j < p.k) ? key_index(s_top[j]) : ci;
+            src = Lbg + (size_t)(c >= 0 ? c : 0) * D;
         }
-#pragma unroll
-        for (int o = LPC / 2; o; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-        if (live && sub == 0)
-            sel_score[((size_t)b * p.H + (size_t)g * p.G + h) * ns + j] = (c >= 0) ? acc * p.scale : -INFINITY;
+        float v[8];
+        load8(src + seg * 8, v);
+        float4 *dst = reinterpret_cast<float4 *>(rows + (size_t)rr * D + seg * 8);
+        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    __syncthreads();
+    for (int task = tid; task < p.G * ns; task += NT) {
+        const int h = task / ns, j = task % ns;
+        const int c = (j < p.k) ? key_index(s_top[j]) : ci;
+        const float *qr = qrows + (size_t)h * D, *lr = lrows + (size_t)j * D;
+        float a0 = 0.f, a1 = 0.f;
+        for (int x = 0; x < D; x += 2) {
+            const int i0 = (x + tid) & (D - 1), i1 = (x + 1 + tid) & (D - 1);   // rotated: no bank conflicts
+            a0 = fmaf(qr[i0], lr[i0], a0);
+            a1 = fmaf(qr[i1], lr[i1], a1);
+        }
+        sel_score[((size_t)b * p.H + (size_t)g * p.G + h) * ns + j] = (c >= 0) ? (a0 + a1) * p.scale : -INFINITY;
     }
 }
 
 template <typename Tin, int D>
-size_t smem_bytes(const DecodePlan &plan)
+size_t smem_bytes(const Dims &p, const DecodePlan &plan)
 {
-    const size_t scan = D * sizeof(float) + 128 + (size_t)RING * RPS * D * sizeof(Tin) + (size_t)plan.spl * 8;
-    const size_t merge = D * sizeof(float) + 128 + (size_t)plan.sort_n * 8;
-    return scan > merge ? scan : merge;
+    const size_t scan = (size_t)RING * RPS * D * sizeof(Tin) + (size_t)plan.spl * 8;
+    const size_t merge = (size_t)plan.nsplit * p.k * 8;
+    const size_t score = (size_t)(p.G + p.k + 1) * D * sizeof(float);
+    size_t big = scan > merge ? scan : merge;
+    big = big > score ? big : score;
+    return D * sizeof(float) + 128 + big;
 }
 
 template <typename Tin, int D>
@@ -190,7 +205,7 @@ cudaError_t launch_t(const Dims &p, const void *Q, const void *L, int32_t *sel_i
         static_cast<char *>(ws) + align_up((size_t)p.B * p.Hkv * plan.nsplit * p.k * sizeof(uint64_t), 256));
     cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)p.B * p.Hkv * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
-    const size_t smem = smem_bytes<Tin, D>(plan);
+    const size_t smem = smem_bytes<Tin, D>(p, plan);
     auto kern = select_decode_kernel<Tin, D>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -235,8 +250,8 @@ size_t decode_select_ws_bytes(const Dims &p)
 size_t decode_select_smem_bytes(const Dims &p, hils_dtype in)
 {
     const DecodePlan plan = decode_plan(p);
-    if (in == HILS_F32) return p.d == 64 ? smem_bytes<float, 64>(plan) : smem_bytes<float, 128>(plan);
-    return p.d == 64 ? smem_bytes<__nv_bfloat16, 64>(plan) : smem_bytes<__nv_bfloat16, 128>(plan);
+    if (in == HILS_F32) return p.d == 64 ? smem_bytes<float, 64>(p, plan) : smem_bytes<float, 128>(p, plan);
+    return p.d == 64 ? smem_bytes<__nv_bfloat16, 64>(p, plan) : smem_bytes<__nv_bfloat16, 128>(p, plan);
 }
 
 cudaError_t launch_select_decode(const Dims &p, hils_dtype in, const void *Q, const void *L, int32_t *sel_idx,

@@ -58,6 +58,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking test of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Same test, but the thread may sleep up to hint_ns while the phase is pending
 // (it wakes when the phase completes), so waiting threads do not spin on the
 // issue slots the working warps need.
@@ -84,20 +98,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
-    for (unsigned int poll = 0;; ++poll) {
-        if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
+    for (;;) {
         if (*abort_flag) return false;
-        if ((poll & 7u) == 7u) {
-            if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
-                *abort_flag = 1;
-                return false;
-            }
-            if (global_timer_ns() - t0 > limit_ns) {
-                *abort_flag = 1;
-                atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
-                return false;
-            }
+        if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
+            *abort_flag = 1;
+            return false;
         }
+        if (global_timer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
+            return false;
+        }
+        if (mbar_try_wait_sleep(bar, parity, 500u)) return true;
     }
 }
 

@@ -157,6 +157,14 @@ HILS_API hils_status hils_sync_status(void *stream);
 HILS_API hils_status hils_set_wait_limit(long long ns);
 
 /*
+ * Test control of the failure path: when `on` is non-zero, tensor-core kernels
+ * launched afterwards first wait on a barrier that nothing signals, so that
+ * bounded wait expires after the wait limit; the kernel then records
+ * HILS_ERR_TIMEOUT, drains and exits.  No GPU fault is involved.  Off by default.
+ */
+HILS_API hils_status hils_debug_inject_stall(int on);
+
+/*
  * Allocation-free decode selection.  The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- plugins whose
  * host application owns the whole device memory budget, memory-capped
