@@ -182,7 +182,7 @@ def hils_decode_score_select_noalloc(p, Q, L, sel_idx, sel_score, stream=None):
     For callers that cannot allocate device memory; see include/hils.h."""
     _check(_lib.hils_decode_score_select_noalloc(ctypes.byref(p), _ptr(Q), _ptr(L), _ptr(sel_idx),
                                                  _ptr(sel_score), _stream(stream)),
-           "hils_decode_score_select_noalloc", "hils_debug_inject_stall")
+           "hils_decode_score_select_noalloc")
 
 
 def problem(B, H, Hkv, N, T, d, C, k, q_offset=0, in_dtype=HILS_BF16, out_dtype=None, scale=0.0):
