@@ -57,24 +57,29 @@ constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 64, false, false);   // S = Q 
 constexpr uint32_t IDESC_PV = idesc_f16_f32(128, 128, false, true);    // O += P V, f16, V MN-major
 
 struct Layout {
-    uint32_t q, kv, pbuf, bar, misc, bitmap, uni, qlist, qcnt, wts, total;
+    uint32_t q, k, v, bar, misc, bitmap, uni, selbuf, scbuf, qlist, qcnt, wts, total;
 };
 
 __host__ __device__ inline uint32_t al16(uint32_t x) { return (x + 15u) & ~15u; }
 
-template <int NS>
-__host__ __device__ inline Layout make_layout(int k, int nwords, int BQ)
+constexpr int kMaxBars = 64;
+
+// Shared memory: Q (32 KB), a ring of NSK key tiles and a ring of NSV value tiles (16 KB each),
+// barriers, then the block's selection bookkeeping.
+__host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nwords, int BQ)
 {
     Layout L;
     const uint32_t ns = (uint32_t)(k + 1);
     L.q = 0;
-    L.kv = 32768;
-    L.pbuf = L.kv + NS * 32768u;   // (unused: P lives in TMEM)
-    L.bar = L.pbuf;
-    L.misc = L.bar + 32 * 8;
+    L.k = 32768;
+    L.v = L.k + (uint32_t)nsk * 16384u;
+    L.bar = L.v + (uint32_t)nsv * 16384u;
+    L.misc = L.bar + kMaxBars * 8;
     L.bitmap = L.misc + 16;
     L.uni = al16(L.bitmap + 4u * (uint32_t)nwords);
-    L.qlist = al16(L.uni + 4u * ns * (uint32_t)BQ);
+    L.selbuf = al16(L.uni + 4u * ns * (uint32_t)BQ);               // the block's sel_idx rows
+    L.scbuf = al16(L.selbuf + 4u * (uint32_t)k * (uint32_t)BQ);    // the rows' sel_score values
+    L.qlist = al16(L.scbuf + 4u * ns * (uint32_t)kRows);
     L.qcnt = al16(L.qlist + 4u * ns * (uint32_t)BQ);
     L.wts = al16(L.qcnt + 4u * (uint32_t)BQ);
     L.total = al16(L.wts + 4u * ns * (uint32_t)kRows);
@@ -82,11 +87,12 @@ __host__ __device__ inline Layout make_layout(int k, int nwords, int BQ)
 }
 
 // barrier slots
-template <int NS>
+template <int NSK, int NSV>
 struct Bars {
-    static constexpr int Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + NS, S_FULL = 1 + 2 * NS,
-                         P_FULL = 1 + 2 * NS + kSB, P_EMPTY = 1 + 2 * NS + 2 * kSB, O_FULL = 1 + 2 * NS + 3 * kSB,
-                         MMA_DONE = 2 + 2 * NS + 3 * kSB;
+    static constexpr int Q_FULL = 0, K_FULL = 1, K_EMPTY = 1 + NSK, V_FULL = 1 + 2 * NSK,
+                         V_EMPTY = 1 + 2 * NSK + NSV, S_FULL = 1 + 2 * NSK + 2 * NSV, P_FULL = S_FULL + kSB,
+                         P_EMPTY = P_FULL + kSB, O_FULL = P_EMPTY + kSB, MMA_DONE = O_FULL + 1;
+    static_assert(MMA_DONE < kMaxBars, "barrier slots");
 };
 
 __device__ __forceinline__ void store_row32(float *dst, const uint32_t *v)
@@ -124,7 +130,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, unsigne
     return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
-template <int G, typename Tout, int NS>
+template <int G, typename Tout, int NSK, int NSV>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, Dims p, const int32_t *__restrict__ sel_idx,
@@ -132,34 +138,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                      unsigned long long limit_ns, int nwords, int inject_stall)
 {
     constexpr int BQ = kRows / G;
-    using BR = Bars<NS>;
+    using BR = Bars<NSK, NSV>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    const Layout Ly = make_layout<NS>(p.k, nwords, BQ);
+    const Layout Ly = make_layout(NSK, NSV, p.k, nwords, BQ);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q0 = blockIdx.x * BQ, g = blockIdx.y, b = blockIdx.z;
     const int nq = min(BQ, p.N - q0);
     const int ns = p.k + 1;
 
-    const uint32_t sQ = smem_addr(base + Ly.q), sKV = smem_addr(base + Ly.kv);
+    const uint32_t sQ = smem_addr(base + Ly.q), sK = smem_addr(base + Ly.k), sV = smem_addr(base + Ly.v);
     const uint32_t bar0 = smem_addr(base + Ly.bar);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + Ly.misc);
     int *n_union_p = reinterpret_cast<int *>(base + Ly.misc + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 8);
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(base + Ly.bitmap);
     int *uni = reinterpret_cast<int *>(base + Ly.uni);
+    int *selbuf = reinterpret_cast<int *>(base + Ly.selbuf);
+    float *scbuf = reinterpret_cast<float *>(base + Ly.scbuf);
     int *qlist = reinterpret_cast<int *>(base + Ly.qlist);
     int *qcnt = reinterpret_cast<int *>(base + Ly.qcnt);
     float *wts = reinterpret_cast<float *>(base + Ly.wts);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
 
-    // ---- set-up: barriers, TMEM, union of the block's selected chunks ------
+    // ---- set-up --------------------------------------------------------------
+    // Q's load starts at once; the selection rows are copied to shared memory with
+    // coalesced loads, and the block's chunk union, per-query chunk lists and per-row
+    // fusion weights are built from there.
     if (tid == 0) {
         mbar_init(BAR(BR::Q_FULL), 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(BAR(BR::KV_FULL + s), 1);
-            mbar_init(BAR(BR::KV_EMPTY + s), 1);
+        for (int s = 0; s < NSK; ++s) {
+            mbar_init(BAR(BR::K_FULL + s), 1);
+            mbar_init(BAR(BR::K_EMPTY + s), 1);
+        }
+        for (int s = 0; s < NSV; ++s) {
+            mbar_init(BAR(BR::V_FULL + s), 1);
+            mbar_init(BAR(BR::V_EMPTY + s), 1);
         }
         for (int s = 0; s < kSB; ++s) {
             mbar_init(BAR(BR::S_FULL + s), 1);
@@ -173,17 +188,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
+        mbar_arrive_expect_tx(BAR(BR::Q_FULL), 32768u);
+        tma_load_3d(sQ, &tmQ, BAR(BR::Q_FULL), 0, q0, b * p.H + g * G);
+        tma_load_3d(sQ + 16384u, &tmQ, BAR(BR::Q_FULL), 64, q0, b * p.H + g * G);
     }
     if (warp == 1) {
         tmem_alloc(smem_addr(tmem_holder), kTmemCols);
         tmem_relinquish();
     }
     for (int i = tid; i < nwords; i += kThreads) bitmap[i] = 0u;
+    const int32_t *sel_base = sel_idx + ((((size_t)b * p.Hkv + g) * p.N) + q0) * p.k;
+    for (int e = tid; e < nq * p.k; e += kThreads) selbuf[e] = __ldg(sel_base + e);
+    for (int e = tid; e < G * nq * ns; e += kThreads) {
+        const int h = e / (nq * ns), rem = e % (nq * ns);
+        const size_t row0 = (((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0;
+        scbuf[(h * BQ + rem / ns) * ns + rem % ns] = __ldg(sel_score + row0 * ns + rem);
+    }
     __syncthreads();
 
-    const int32_t *sel_base = sel_idx + ((((size_t)b * p.Hkv + g) * p.N) + q0) * p.k;
     for (int e = tid; e < nq * p.k; e += kThreads) {
-        const int c = sel_base[e];
+        const int c = selbuf[e];
         if (c >= 0) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
     }
     for (int qi = tid; qi < nq; qi += kThreads) {
@@ -219,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int *lst = qlist + qi * ns;
         int cnt = 0;
         for (int j = 0; j <= p.k; ++j) {
-            const int c = (j < p.k) ? sel_base[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
+            const int c = (j < p.k) ? selbuf[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
             if (c < 0) continue;
             int at = cnt++;
             while (at > 0 && lst[at - 1] > c) {
@@ -234,10 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid < kRows) {
         // fusion weights of each row, stored in the order of its query's chunk list
-        const int r = tid, h = r / BQ, qi = r % BQ;
+        const int r = tid, qi = r % BQ;
         if (qi < nq) {
-            const size_t row_h = (((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi;
-            const float *sc = sel_score + row_h * ns;
+            const float *sc = scbuf + r * ns;
             float M = -INFINITY;
             for (int j = 0; j < ns; ++j) M = fmaxf(M, sc[j]);
             float Z = 0.f;
@@ -245,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int *lst = qlist + qi * ns;
             const int cnt = qcnt[qi];
             for (int j = 0; j < ns; ++j) {
-                const int c = (j < p.k) ? sel_base[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
+                const int c = (j < p.k) ? selbuf[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
                 if (c < 0) continue;
                 int lo = 0, hi = cnt - 1;
                 while (lo < hi) {
@@ -265,16 +288,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA + MMA issue --------------------------------
-            // One thread drives both async engines.  It never blocks on one event while
-            // another could proceed: each pass tests (without waiting) whether a load, a QK
-            // product or a PV product can be issued, and issues it.  QK runs up to kSB
-            // chunks ahead of PV, loads up to NS chunks ahead.
+            // One thread drives both async engines and never blocks on one event while another
+            // could proceed.  Each pass, in priority order: a key-tile load (up to NSK chunks ahead
+            // of QK; a key slot frees when its QK completes), a value-tile load (up to NSV ahead of
+            // PV), the next PV product, the next QK product (up to kSB chunks ahead of PV).
             const int kv_row0 = (b * p.Hkv + g) * p.T;
-            int next_load = 0, next_qk = 0, next_pv = 0;
+            int next_k = 0, next_v = 0, next_qk = 0, next_pv = 0;
             bool q_ready = false;
-            mbar_arrive_expect_tx(BAR(BR::Q_FULL), 32768u);
-            tma_load_3d(sQ, &tmQ, BAR(BR::Q_FULL), 0, q0, b * p.H + g * G);
-            tma_load_3d(sQ + 16384u, &tmQ, BAR(BR::Q_FULL), 64, q0, b * p.H + g * G);
             if (inject_stall) {
                 // test control: wait once on a barrier nothing signals, so the bounded wait expires
                 mbar_wait(BAR(BR::MMA_DONE), 0, limit_ns, abort_flag, status);
@@ -282,53 +302,64 @@ __global__ void __launch_bounds__(kThreads, 1)
             unsigned long long idle_since = 0ull;
             while (next_pv < n_union && !*abort_flag) {
                 bool prog = false;
-                if (next_load < n_union && next_load < next_pv + NS) {
-                    const int u = next_load, st = u % NS;
-                    if (u < NS || mbar_test(BAR(BR::KV_EMPTY + st), (uint32_t)(((u / NS) - 1) & 1))) {
+                if (next_k < n_union && next_k < next_qk + NSK) {
+                    const int u = next_k, st = u % NSK;
+                    if (u < NSK || mbar_test(BAR(BR::K_EMPTY + st), (uint32_t)(((u / NSK) - 1) & 1))) {
                         const int row = kv_row0 + uni[u] * kChunk;
-                        const uint32_t dst = sKV + (uint32_t)st * 32768u;
-                        mbar_arrive_expect_tx(BAR(BR::KV_FULL + st), 32768u);
-                        tma_load_2d(dst, &tmK, BAR(BR::KV_FULL + st), 0, row);
-                        tma_load_2d(dst + 8192u, &tmK, BAR(BR::KV_FULL + st), 64, row);
-                        tma_load_2d(dst + 16384u, &tmV, BAR(BR::KV_FULL + st), 0, row);
-                        tma_load_2d(dst + 24576u, &tmV, BAR(BR::KV_FULL + st), 64, row);
-                        ++next_load;
+                        const uint32_t dst = sK + (uint32_t)st * 16384u;
+                        mbar_arrive_expect_tx(BAR(BR::K_FULL + st), 16384u);
+                        tma_load_2d(dst, &tmK, BAR(BR::K_FULL + st), 0, row);
+                        tma_load_2d(dst + 8192u, &tmK, BAR(BR::K_FULL + st), 64, row);
+                        ++next_k;
                         prog = true;
                     }
                 }
-                if (next_qk < next_load && next_qk < next_pv + kSB) {
-                    if (!q_ready) q_ready = mbar_test(BAR(BR::Q_FULL), 0);
-                    const int t = next_qk, st = t % NS;
-                    if (q_ready && mbar_test(BAR(BR::KV_FULL + st), (uint32_t)((t / NS) & 1))) {
+                if (next_v < n_union && next_v < next_pv + NSV) {
+                    const int u = next_v, st = u % NSV;
+                    if (u < NSV || mbar_test(BAR(BR::V_EMPTY + st), (uint32_t)(((u / NSV) - 1) & 1))) {
+                        const int row = kv_row0 + uni[u] * kChunk;
+                        const uint32_t dst = sV + (uint32_t)st * 16384u;
+                        mbar_arrive_expect_tx(BAR(BR::V_FULL + st), 16384u);
+                        tma_load_2d(dst, &tmV, BAR(BR::V_FULL + st), 0, row);
+                        tma_load_2d(dst + 8192u, &tmV, BAR(BR::V_FULL + st), 64, row);
+                        ++next_v;
+                        prog = true;
+                    }
+                }
+                if (next_pv < next_qk && next_pv < next_v) {
+                    const int u = next_pv, vst = u % NSV;
+                    if (mbar_test(BAR(BR::P_FULL + u % kSB), (uint32_t)((u / kSB) & 1)) &&
+                        mbar_test(BAR(BR::V_FULL + vst), (uint32_t)((u / NSV) & 1))) {
                         tc_fence_after();
-                        // S buffer t % kSB is free: QK(t - kSB)'s chunk was softmaxed before its PV,
-                        // which was issued before this point (next_pv > t - kSB)
+                        const uint32_t pa = tmem + kColP + (uint32_t)(u % kSB) * 32u;
+                        const uint32_t va = sV + (uint32_t)vst * 16384u;
+#pragma unroll
+                        for (int s = 0; s < 4; ++s)
+                            mma_f16_ts(tmem + kColO, pa + 8u * s, smem_desc_sw128(va + 2048u * s, 8192, 1024),
+                                       IDESC_PV, (u > 0 || s > 0) ? 1u : 0u);
+                        mma_commit(BAR(BR::V_EMPTY + vst));
+                        mma_commit(BAR(BR::P_EMPTY + u % kSB));
+                        ++next_pv;
+                        prog = true;
+                    }
+                }
+                if (next_qk < next_k && next_qk < next_pv + kSB) {
+                    if (!q_ready) q_ready = mbar_test(BAR(BR::Q_FULL), 0);
+                    const int t = next_qk, kst = t % NSK;
+                    if (q_ready && mbar_test(BAR(BR::K_FULL + kst), (uint32_t)((t / NSK) & 1))) {
+                        tc_fence_after();
+                        // S buffer t % kSB is free: chunk t - kSB was softmaxed before its PV, which was
+                        // issued before this point (next_pv > t - kSB)
                         const uint32_t d_s = tmem + (uint32_t)(t % kSB) * 64u;
-                        const uint32_t ka = sKV + (uint32_t)st * 32768u;
+                        const uint32_t ka = sK + (uint32_t)kst * 16384u;
 #pragma unroll
                         for (int s = 0; s < 8; ++s)
                             mma_bf16_ss(d_s, smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
                                         smem_desc_sw128(ka + (s >> 2) * 8192u + (s & 3) * 32u, 16, 1024), IDESC_QK,
                                         s > 0 ? 1u : 0u);
                         mma_commit(BAR(BR::S_FULL + t % kSB));
+                        mma_commit(BAR(BR::K_EMPTY + kst));
                         ++next_qk;
-                        prog = true;
-                    }
-                }
-                if (next_pv < next_qk) {
-                    const int u = next_pv;
-                    if (mbar_test(BAR(BR::P_FULL + u % kSB), (uint32_t)((u / kSB) & 1))) {
-                        tc_fence_after();
-                        const uint32_t st = (uint32_t)(u % NS);
-                        const uint32_t pa = tmem + kColP + (uint32_t)(u % kSB) * 32u;
-                        const uint32_t va = sKV + st * 32768u + 16384u;
-#pragma unroll
-                        for (int s = 0; s < 4; ++s)
-                            mma_f16_ts(tmem + kColO, pa + 8u * s, smem_desc_sw128(va + 2048u * s, 8192, 1024),
-                                       IDESC_PV, (u > 0 || s > 0) ? 1u : 0u);
-                        mma_commit(BAR(BR::KV_EMPTY + (int)st));
-                        mma_commit(BAR(BR::P_EMPTY + u % kSB));
-                        ++next_pv;
                         prog = true;
                     }
                 }
@@ -343,15 +374,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
                         *abort_flag = 1;
                     }
-                    __nanosleep(32);
+                    __nanosleep(20);
                 }
             }
             if (!*abort_flag) mma_commit(BAR(BR::O_FULL));
-            // drain: every issued MMA, then the latest load of every stage and Q
+            // drain: every issued MMA, then the latest load of every slot and Q
             mma_commit(BAR(BR::MMA_DONE));
             mbar_drain(BAR(BR::MMA_DONE), 0, kDrainNs);
-            for (int u = max(0, next_load - NS); u < next_load; ++u)
-                mbar_drain(BAR(BR::KV_FULL + u % NS), (uint32_t)((u / NS) & 1), kDrainNs);
+            for (int u = max(0, next_k - NSK); u < next_k; ++u)
+                mbar_drain(BAR(BR::K_FULL + u % NSK), (uint32_t)((u / NSK) & 1), kDrainNs);
+            for (int u = max(0, next_v - NSV); u < next_v; ++u)
+                mbar_drain(BAR(BR::V_FULL + u % NSV), (uint32_t)((u / NSV) & 1), kDrainNs);
             mbar_drain(BAR(BR::Q_FULL), 0, kDrainNs);
         }
         __syncwarp();
@@ -490,8 +523,6 @@ bool encode(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, int rank, c
     return r == CUDA_SUCCESS;
 }
 
-constexpr int kStages = 4;
-
 // V (bf16) -> f16, 8 elements per 16-byte vector; exact for |v| < 65504.
 __global__ void v_to_f16_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, size_t n)
 {
@@ -505,6 +536,17 @@ __global__ void v_to_f16_kernel(const uint4 *__restrict__ in, uint4 *__restrict_
         }
         out[i] = make_uint4(w[0], w[1], w[2], w[3]);
     }
+}
+
+constexpr int kSmemLimit = 227 * 1024;
+
+// Deepest key/value rings that fit: 0 = (6, 4), 1 = (4, 3), 2 = (2, 2), -1 = none.
+int ring_config(int k, int nwords, int BQ)
+{
+    if (make_layout(6, 4, k, nwords, BQ).total + 1024 <= kSmemLimit) return 0;
+    if (make_layout(4, 3, k, nwords, BQ).total + 1024 <= kSmemLimit) return 1;
+    if (make_layout(2, 2, k, nwords, BQ).total + 1024 <= kSmemLimit) return 2;
+    return -1;
 }
 
 template <int G, typename Tout>
@@ -525,14 +567,23 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V,
         return cudaErrorInvalidValue;
     const int c_max = (int)(((long long)p.q_offset + p.N - 1) / kChunk);
     const int nwords = c_max / 32 + 1;
-    const Layout Ly = make_layout<kStages>(p.k, nwords, BQ);
-    const size_t smem = Ly.total + 1024;
-    auto kern = attend_tc_kernel<G, Tout, kStages>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
-    kern<<<grid, kThreads, smem, s>>>(tq, tk, tv, p, sel_idx, sel_score, static_cast<Tout *>(O), ctl.status,
-                                      (unsigned long long)ctl.wait_limit, nwords, ctl.inject_stall);
+    const int cfg = ring_config(p.k, nwords, BQ);
+    cudaError_t e = cudaErrorInvalidValue;
+#define HILS_LAUNCH_TC(NK, NV)                                                                              \
+    {                                                                                                        \
+        const size_t smem = make_layout(NK, NV, p.k, nwords, BQ).total + 1024;                              \
+        auto kern = attend_tc_kernel<G, Tout, NK, NV>;                                                      \
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);              \
+        if (e != cudaSuccess) return e;                                                                      \
+        kern<<<grid, kThreads, smem, s>>>(tq, tk, tv, p, sel_idx, sel_score, static_cast<Tout *>(O),         \
+                                          ctl.status, (unsigned long long)ctl.wait_limit, nwords,            \
+                                          ctl.inject_stall);                                                 \
+    }
+    if (cfg == 0) HILS_LAUNCH_TC(6, 4)
+    else if (cfg == 1) HILS_LAUNCH_TC(4, 3)
+    else HILS_LAUNCH_TC(2, 2)
+#undef HILS_LAUNCH_TC
     return cudaGetLastError();
 }
 
@@ -557,8 +608,7 @@ bool attend_tc_supported(const Dims &p, hils_dtype in)
     if (in != HILS_BF16 || p.d != kD || p.C != kChunk || p.N < 2) return false;
     if (p.G != 1 && p.G != 2 && p.G != 4 && p.G != 8 && p.G != 16) return false;
     const int c_max = (int)(((long long)p.q_offset + p.N - 1) / kChunk);
-    const Layout Ly = make_layout<kStages>(p.k, c_max / 32 + 1, kRows / p.G);
-    return Ly.total + 1024 <= 227 * 1024;
+    return ring_config(p.k, c_max / 32 + 1, kRows / p.G) >= 0;
 }
 
 size_t attend_tc_ws_bytes(const Dims &p)
