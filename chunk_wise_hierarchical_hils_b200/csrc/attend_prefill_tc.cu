@@ -42,12 +42,13 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;     // 10 warps
+constexpr int kThreads = 384;     // 12 warps: K loads, V loads + TMEM, MMA, spare, 2 x 4 softmax
 constexpr int kRows = 128;        // MMA M
 constexpr int kChunk = 64;        // C
 constexpr int kD = 128;           // d
 constexpr int kSB = 4;                // S and P buffers: QK may run up to kSB chunks ahead of PV
 constexpr int kGroups = 2;            // softmax warp groups; group t % kGroups handles chunk t
+constexpr int kLookahead = 3;         // QK products issued ahead of the PV being waited for (< kSB)
 constexpr uint32_t kTmemCols = 512;   // S0..S3 (64 columns each), O (128), P0..P3 (32 each)
 constexpr uint32_t kColO = 256, kColP = 384;
 constexpr unsigned long long kDrainNs = 2000000000ull;
@@ -57,7 +58,7 @@ constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 64, false, false);   // S = Q 
 constexpr uint32_t IDESC_PV = idesc_f16_f32(128, 128, false, true);    // O += P V, f16, V MN-major
 
 struct Layout {
-    uint32_t q, k, v, bar, misc, bitmap, uni, selbuf, scbuf, qlist, qcnt, wts, total;
+    uint32_t q, k, v, bar, misc, bitmap, uni, selbuf, scbuf, qlist, qslot, qcnt, wts, total;
 };
 
 __host__ __device__ inline uint32_t al16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -80,7 +81,8 @@ __host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nword
     L.selbuf = al16(L.uni + 4u * ns * (uint32_t)BQ);               // the block's sel_idx rows
     L.scbuf = al16(L.selbuf + 4u * (uint32_t)k * (uint32_t)BQ);    // the rows' sel_score values
     L.qlist = al16(L.scbuf + 4u * ns * (uint32_t)kRows);
-    L.qcnt = al16(L.qlist + 4u * ns * (uint32_t)BQ);
+    L.qslot = al16(L.qlist + 4u * ns * (uint32_t)BQ);
+    L.qcnt = al16(L.qslot + 4u * ns * (uint32_t)BQ);
     L.wts = al16(L.qcnt + 4u * (uint32_t)BQ);
     L.total = al16(L.wts + 4u * ns * (uint32_t)kRows);
     return L;
@@ -158,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *selbuf = reinterpret_cast<int *>(base + Ly.selbuf);
     float *scbuf = reinterpret_cast<float *>(base + Ly.scbuf);
     int *qlist = reinterpret_cast<int *>(base + Ly.qlist);
+    int *qslot = reinterpret_cast<int *>(base + Ly.qslot);
     int *qcnt = reinterpret_cast<int *>(base + Ly.qcnt);
     float *wts = reinterpret_cast<float *>(base + Ly.wts);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -206,13 +209,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
-    for (int e = tid; e < nq * p.k; e += kThreads) {
-        const int c = selbuf[e];
-        if (c >= 0) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
-    }
-    for (int qi = tid; qi < nq; qi += kThreads) {
-        const int c = (int)(((long long)p.q_offset + q0 + qi) / kChunk);
-        atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+    // mark the selected and own chunks; with few bitmap words the bits are OR-reduced across the
+    // warp first, so that the shared-memory atomics do not all land on the same words
+    const int n_marks = nq * p.k + nq;
+    for (int e0 = warp * 32; e0 < n_marks; e0 += kThreads) {
+        const int e = e0 + lane;
+        int c = -1;
+        if (e < nq * p.k) c = selbuf[e];
+        else if (e < n_marks) c = (int)(((long long)p.q_offset + q0 + (e - nq * p.k)) / kChunk);
+        if (nwords <= 8) {
+            for (int wd = 0; wd < nwords; ++wd) {
+                const unsigned int bits =
+                    __reduce_or_sync(0xFFFFFFFFu, (c >= 0 && (c >> 5) == wd) ? (1u << (c & 31)) : 0u);
+                if (lane == 0 && bits) atomicOr(&bitmap[wd], bits);
+            }
+        } else if (c >= 0) {
+            atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+        }
     }
     __syncthreads();
 
@@ -241,6 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // each query's chunks (selected + own) in ascending order
         const int qi = tid - 32;
         int *lst = qlist + qi * ns;
+        int *slt = qslot + qi * ns;
         int cnt = 0;
         for (int j = 0; j <= p.k; ++j) {
             const int c = (j < p.k) ? selbuf[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
@@ -248,34 +262,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             int at = cnt++;
             while (at > 0 && lst[at - 1] > c) {
                 lst[at] = lst[at - 1];
+                slt[at] = slt[at - 1];
                 --at;
             }
             lst[at] = c;
+            slt[at] = j;    // the slot this chunk came from
         }
         qcnt[qi] = cnt;
     }
     __syncthreads();
 
     if (tid < kRows) {
-        // fusion weights of each row, stored in the order of its query's chunk list
+        // fusion weights of each row, in the order of its query's chunk list
         const int r = tid, qi = r % BQ;
         if (qi < nq) {
             const float *sc = scbuf + r * ns;
             float M = -INFINITY;
             for (int j = 0; j < ns; ++j) M = fmaxf(M, sc[j]);
             float Z = 0.f;
-            for (int j = 0; j < ns; ++j) Z += (sc[j] == -INFINITY) ? 0.f : expf(sc[j] - M);
-            const int *lst = qlist + qi * ns;
+            for (int j = 0; j < ns; ++j) Z += (sc[j] == -INFINITY) ? 0.f : __expf(sc[j] - M);
+            const float iz = 1.0f / Z;
+            const int *slt = qslot + qi * ns;
             const int cnt = qcnt[qi];
-            for (int j = 0; j < ns; ++j) {
-                const int c = (j < p.k) ? selbuf[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
-                if (c < 0) continue;
-                int lo = 0, hi = cnt - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (lst[mid] < c) lo = mid + 1; else hi = mid;
-                }
-                wts[r * ns + lo] = (sc[j] == -INFINITY) ? 0.f : expf(sc[j] - M) / Z;
+            for (int pos = 0; pos < cnt; ++pos) {
+                const float sj = sc[slt[pos]];
+                wts[r * ns + pos] = (sj == -INFINITY) ? 0.f : __expf(sj - M) * iz;
             }
         }
     }
@@ -285,112 +296,104 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_holder;
     const int n_union = *n_union_p;
 
+    const int kv_row0 = (b * p.Hkv + g) * p.T;
     if (warp == 0) {
+        // ---------------- key tiles: up to NSK chunks ahead; a slot frees when its QK completes
         if (lane == 0) {
-            // ---------------- TMA + MMA issue --------------------------------
-            // One thread drives both async engines and never blocks on one event while another
-            // could proceed.  Each pass, in priority order: a key-tile load (up to NSK chunks ahead
-            // of QK; a key slot frees when its QK completes), a value-tile load (up to NSV ahead of
-            // PV), the next PV product, the next QK product (up to kSB chunks ahead of PV).
-            const int kv_row0 = (b * p.Hkv + g) * p.T;
-            int next_k = 0, next_v = 0, next_qk = 0, next_pv = 0;
-            bool q_ready = false;
-            if (inject_stall) {
-                // test control: wait once on a barrier nothing signals, so the bounded wait expires
-                mbar_wait(BAR(BR::MMA_DONE), 0, limit_ns, abort_flag, status);
+            int u = 0;
+            for (; u < n_union; ++u) {
+                const int st = u % NSK;
+                if (u >= NSK &&
+                    !mbar_wait(BAR(BR::K_EMPTY + st), (uint32_t)(((u / NSK) - 1) & 1), limit_ns, abort_flag, status))
+                    break;
+                const int row = kv_row0 + uni[u] * kChunk;
+                const uint32_t dst = sK + (uint32_t)st * 16384u;
+                mbar_arrive_expect_tx(BAR(BR::K_FULL + st), 16384u);
+                tma_load_2d(dst, &tmK, BAR(BR::K_FULL + st), 0, row);
+                tma_load_2d(dst + 8192u, &tmK, BAR(BR::K_FULL + st), 64, row);
             }
-            unsigned long long idle_since = 0ull;
-            while (next_pv < n_union && !*abort_flag) {
-                bool prog = false;
-                if (next_k < n_union && next_k < next_qk + NSK) {
-                    const int u = next_k, st = u % NSK;
-                    if (u < NSK || mbar_test(BAR(BR::K_EMPTY + st), (uint32_t)(((u / NSK) - 1) & 1))) {
-                        const int row = kv_row0 + uni[u] * kChunk;
-                        const uint32_t dst = sK + (uint32_t)st * 16384u;
-                        mbar_arrive_expect_tx(BAR(BR::K_FULL + st), 16384u);
-                        tma_load_2d(dst, &tmK, BAR(BR::K_FULL + st), 0, row);
-                        tma_load_2d(dst + 8192u, &tmK, BAR(BR::K_FULL + st), 64, row);
-                        ++next_k;
-                        prog = true;
-                    }
-                }
-                if (next_v < n_union && next_v < next_pv + NSV) {
-                    const int u = next_v, st = u % NSV;
-                    if (u < NSV || mbar_test(BAR(BR::V_EMPTY + st), (uint32_t)(((u / NSV) - 1) & 1))) {
-                        const int row = kv_row0 + uni[u] * kChunk;
-                        const uint32_t dst = sV + (uint32_t)st * 16384u;
-                        mbar_arrive_expect_tx(BAR(BR::V_FULL + st), 16384u);
-                        tma_load_2d(dst, &tmV, BAR(BR::V_FULL + st), 0, row);
-                        tma_load_2d(dst + 8192u, &tmV, BAR(BR::V_FULL + st), 64, row);
-                        ++next_v;
-                        prog = true;
-                    }
-                }
-                if (next_pv < next_qk && next_pv < next_v) {
-                    const int u = next_pv, vst = u % NSV;
-                    if (mbar_test(BAR(BR::P_FULL + u % kSB), (uint32_t)((u / kSB) & 1)) &&
-                        mbar_test(BAR(BR::V_FULL + vst), (uint32_t)((u / NSV) & 1))) {
-                        tc_fence_after();
-                        const uint32_t pa = tmem + kColP + (uint32_t)(u % kSB) * 32u;
-                        const uint32_t va = sV + (uint32_t)vst * 16384u;
-#pragma unroll
-                        for (int s = 0; s < 4; ++s)
-                            mma_f16_ts(tmem + kColO, pa + 8u * s, smem_desc_sw128(va + 2048u * s, 8192, 1024),
-                                       IDESC_PV, (u > 0 || s > 0) ? 1u : 0u);
-                        mma_commit(BAR(BR::V_EMPTY + vst));
-                        mma_commit(BAR(BR::P_EMPTY + u % kSB));
-                        ++next_pv;
-                        prog = true;
-                    }
-                }
-                if (next_qk < next_k && next_qk < next_pv + kSB) {
-                    if (!q_ready) q_ready = mbar_test(BAR(BR::Q_FULL), 0);
-                    const int t = next_qk, kst = t % NSK;
-                    if (q_ready && mbar_test(BAR(BR::K_FULL + kst), (uint32_t)((t / NSK) & 1))) {
-                        tc_fence_after();
-                        // S buffer t % kSB is free: chunk t - kSB was softmaxed before its PV, which was
-                        // issued before this point (next_pv > t - kSB)
-                        const uint32_t d_s = tmem + (uint32_t)(t % kSB) * 64u;
-                        const uint32_t ka = sK + (uint32_t)kst * 16384u;
-#pragma unroll
-                        for (int s = 0; s < 8; ++s)
-                            mma_bf16_ss(d_s, smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
-                                        smem_desc_sw128(ka + (s >> 2) * 8192u + (s & 3) * 32u, 16, 1024), IDESC_QK,
-                                        s > 0 ? 1u : 0u);
-                        mma_commit(BAR(BR::S_FULL + t % kSB));
-                        mma_commit(BAR(BR::K_EMPTY + kst));
-                        ++next_qk;
-                        prog = true;
-                    }
-                }
-                if (prog) {
-                    idle_since = 0ull;
-                } else {
-                    const unsigned long long now = global_timer_ns();
-                    if (!idle_since) idle_since = now;
-                    if (now - idle_since > limit_ns) {
-                        *abort_flag = 1;
-                        atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
-                    } else if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
-                        *abort_flag = 1;
-                    }
-                    __nanosleep(20);
-                }
-            }
-            if (!*abort_flag) mma_commit(BAR(BR::O_FULL));
-            // drain: every issued MMA, then the latest load of every slot and Q
-            mma_commit(BAR(BR::MMA_DONE));
-            mbar_drain(BAR(BR::MMA_DONE), 0, kDrainNs);
-            for (int u = max(0, next_k - NSK); u < next_k; ++u)
-                mbar_drain(BAR(BR::K_FULL + u % NSK), (uint32_t)((u / NSK) & 1), kDrainNs);
-            for (int u = max(0, next_v - NSV); u < next_v; ++u)
-                mbar_drain(BAR(BR::V_FULL + u % NSV), (uint32_t)((u / NSV) & 1), kDrainNs);
+            // the copies must land before the CTA exits (only outstanding after an abort)
+            for (int v = max(0, u - NSK); v < u; ++v)
+                mbar_drain(BAR(BR::K_FULL + v % NSK), (uint32_t)((v / NSK) & 1), kDrainNs);
             mbar_drain(BAR(BR::Q_FULL), 0, kDrainNs);
         }
         __syncwarp();
-    } else if (warp >= 2) {
+    } else if (warp == 1) {
+        // ---------------- value tiles: up to NSV chunks ahead; a slot frees when its PV completes
+        if (lane == 0) {
+            int u = 0;
+            for (; u < n_union; ++u) {
+                const int st = u % NSV;
+                if (u >= NSV &&
+                    !mbar_wait(BAR(BR::V_EMPTY + st), (uint32_t)(((u / NSV) - 1) & 1), limit_ns, abort_flag, status))
+                    break;
+                const int row = kv_row0 + uni[u] * kChunk;
+                const uint32_t dst = sV + (uint32_t)st * 16384u;
+                mbar_arrive_expect_tx(BAR(BR::V_FULL + st), 16384u);
+                tma_load_2d(dst, &tmV, BAR(BR::V_FULL + st), 0, row);
+                tma_load_2d(dst + 8192u, &tmV, BAR(BR::V_FULL + st), 64, row);
+            }
+            for (int v = max(0, u - NSV); v < u; ++v)
+                mbar_drain(BAR(BR::V_FULL + v % NSV), (uint32_t)((v / NSV) & 1), kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ---------------- MMA issue: QK runs kLookahead chunks ahead of PV -----------------
+        // Schedule: QK(0..L-1), then for each u: PV(u), QK(u+L).  QK(t) reuses the S buffer of
+        // chunk t - kSB, whose PV (and so its softmax) came earlier in this order (L < kSB).
+        if (lane == 0) {
+            bool ok = true;
+            if (inject_stall) {
+                // test control: wait once on a barrier nothing signals, so the bounded wait expires
+                ok = mbar_wait(BAR(BR::MMA_DONE), 0, limit_ns, abort_flag, status);
+            }
+            ok = ok && mbar_wait(BAR(BR::Q_FULL), 0, limit_ns, abort_flag, status);
+            auto issue_qk = [&](int t) -> bool {
+                const int kst = t % NSK;
+                if (!mbar_wait(BAR(BR::K_FULL + kst), (uint32_t)((t / NSK) & 1), limit_ns, abort_flag, status))
+                    return false;
+                tc_fence_after();
+                const uint32_t d_s = tmem + (uint32_t)(t % kSB) * 64u;
+                const uint32_t ka = sK + (uint32_t)kst * 16384u;
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16_ss(d_s, smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
+                                smem_desc_sw128(ka + (s >> 2) * 8192u + (s & 3) * 32u, 16, 1024), IDESC_QK,
+                                s > 0 ? 1u : 0u);
+                mma_commit(BAR(BR::S_FULL + t % kSB));
+                mma_commit(BAR(BR::K_EMPTY + kst));
+                return true;
+            };
+            auto issue_pv = [&](int u) -> bool {
+                const int vst = u % NSV;
+                if (!mbar_wait(BAR(BR::P_FULL + u % kSB), (uint32_t)((u / kSB) & 1), limit_ns, abort_flag, status) ||
+                    !mbar_wait(BAR(BR::V_FULL + vst), (uint32_t)((u / NSV) & 1), limit_ns, abort_flag, status))
+                    return false;
+                tc_fence_after();
+                const uint32_t pa = tmem + kColP + (uint32_t)(u % kSB) * 32u;
+                const uint32_t va = sV + (uint32_t)vst * 16384u;
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_f16_ts(tmem + kColO, pa + 8u * s, smem_desc_sw128(va + 2048u * s, 8192, 1024), IDESC_PV,
+                               (u > 0 || s > 0) ? 1u : 0u);
+                mma_commit(BAR(BR::V_EMPTY + vst));
+                mma_commit(BAR(BR::P_EMPTY + u % kSB));
+                return true;
+            };
+            for (int t = 0; ok && t < min(kLookahead, n_union); ++t) ok = issue_qk(t);
+            for (int u = 0; ok && u < n_union; ++u) {
+                ok = issue_pv(u);
+                if (ok && u + kLookahead < n_union) ok = issue_qk(u + kLookahead);
+            }
+            if (ok) mma_commit(BAR(BR::O_FULL));
+            // drain: every issued MMA completes before TMEM is released
+            mma_commit(BAR(BR::MMA_DONE));
+            mbar_drain(BAR(BR::MMA_DONE), 0, kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
         // ---------------- softmax (kGroups groups, alternate chunks) and epilogue ----
-        const int grp = (warp - 2) >> 2;
+        const int grp = (warp - 4) >> 2;
         const int qq = warp & 3;
         const int r = 32 * qq + lane, h = r / BQ, qi = r % BQ;
         const bool valid = qi < nq;
