@@ -10,19 +10,26 @@
 //
 // One CTA owns 128 rows = (128 / G) consecutive queries x the G heads of one
 // kv-group (row r = head * (128 / G) + query).  It walks the union of the
-// chunks its queries selected, in ascending chunk order:
-//   warp 0 (one thread)  TMA loads of Q once and of every union chunk's K and V
-//                        (two 64-column halves each, 128-byte swizzle, no
-//                        multicast) and the tcgen05.mma issue: S = Q K^T (bf16,
-//                        A and B from shared memory) into one of two TMEM
-//                        buffers, then O += P V (f16, P from TMEM, V from shared
-//                        memory) into the TMEM accumulator;
-//   warps 2..9           two groups of four warps, one thread per row; group
-//                        t % 2 handles chunk t: it reads S from TMEM, takes the
-//                        softmax over the chunk's visible keys, scales it by the
-//                        row's fusion weight (0 if the row's query did not
-//                        select this chunk) and writes P (f16) to TMEM.  At the
-//                        end both groups read O from TMEM and store it.
+// chunks its queries selected, in ascending chunk order, with warp-specialised
+// roles that meet on mbarriers:
+//   warp 0 (one thread)  TMA loads of Q once and of the union's K tiles, two
+//                        chunks per ring slot (128-byte swizzle, no multicast);
+//   warp 1 (one thread)  TMA loads of the V tiles, one chunk per ring slot;
+//                        the warp also owns the TMEM allocation;
+//   warp 2 (one thread)  tcgen05.mma issue.  S = Q K^T (bf16, A and B from
+//                        shared memory) runs on two chunks at once (N = 128,
+//                        the tensor core's efficient width) into one of two
+//                        TMEM S buffers; O += P V (f16, P from TMEM, V from
+//                        shared memory) per chunk.  The issuer polls which of
+//                        the two is ready, key products first, so the softmax
+//                        warps never wait behind a value product;
+//   warps 4..11          two groups of four warps, one thread per row; group
+//                        t % 2 handles chunk t: it reads S from TMEM (and frees
+//                        the S buffer at once), takes the softmax over the
+//                        chunk's visible keys, scales it by the row's fusion
+//                        weight (0 if the row's query did not select the chunk)
+//                        and writes P (f16) to one of four TMEM P buffers.  At
+//                        the end both groups read O from TMEM and store it.
 // Because each chunk's softmax is normalised on its own and the fusion weights
 // are known before the loop, P already carries w_c / l_c and the accumulator
 // needs no rescaling between chunks.  V is read as f16 (converted once per call
@@ -34,6 +41,7 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 
+#include "chunk_softmax.cuh"
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -42,19 +50,20 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;     // 12 warps: K loads, V loads + TMEM, MMA, spare, 2 x 4 softmax
+constexpr int kThreads = 384;     // 12 warps: K loads, V loads + TMEM, MMA issue, spare, 2 x 4 softmax
 constexpr int kRows = 128;        // MMA M
 constexpr int kChunk = 64;        // C
 constexpr int kD = 128;           // d
-constexpr int kSB = 4;                // S and P buffers: QK may run up to kSB chunks ahead of PV
+constexpr int kSP = 2;                // S buffers (a pair of chunks, 128 columns each) = key ring slots
 constexpr int kGroups = 2;            // softmax warp groups; group t % kGroups handles chunk t
-constexpr int kLookahead = 3;         // QK products issued ahead of the PV being waited for (< kSB)
-constexpr uint32_t kTmemCols = 512;   // S0..S3 (64 columns each), O (128), P0..P3 (32 each)
+constexpr uint32_t kTmemCols = 512;   // S pair buffers (2 x 128 columns), O (128), up to 4 P buffers (32 each)
 constexpr uint32_t kColO = 256, kColP = 384;
+constexpr uint32_t kPairBytes = 32768;   // K ring slot: [c0 d0-63 | c1 d0-63 | c0 d64-127 | c1 d64-127]
 constexpr unsigned long long kDrainNs = 2000000000ull;
-constexpr int kPolyEvery = 4;     // share of exponentials computed by exp2_poly: 1 in kPolyEvery
+constexpr int kPolyPairEvery = 4; // exponential pairs computed by exp2_poly_x2: 1 in kPolyPairEvery
 
-constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 64, false, false);   // S = Q K^T, bf16, both K-major
+constexpr uint32_t IDESC_QK2 = idesc_bf16_f32(128, 128, false, false);  // S = Q K^T over two chunks, K-major
+constexpr uint32_t IDESC_QK1 = idesc_bf16_f32(128, 64, false, false);   // the same for a lone last chunk
 constexpr uint32_t IDESC_PV = idesc_f16_f32(128, 128, false, true);    // O += P V, f16, V MN-major
 
 struct Layout {
@@ -65,15 +74,15 @@ __host__ __device__ inline uint32_t al16(uint32_t x) { return (x + 15u) & ~15u; 
 
 constexpr int kMaxBars = 64;
 
-// Shared memory: Q (32 KB), a ring of NSK key tiles and a ring of NSV value tiles (16 KB each),
-// barriers, then the block's selection bookkeeping.
+// Shared memory: Q (32 KB), kSP key slots (two chunks, 32 KB each) and a ring of NSV
+// value tiles (16 KB each), barriers, then the block's selection bookkeeping.
 __host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nwords, int BQ)
 {
     Layout L;
     const uint32_t ns = (uint32_t)(k + 1);
     L.q = 0;
     L.k = 32768;
-    L.v = L.k + (uint32_t)nsk * 16384u;
+    L.v = L.k + (uint32_t)nsk * kPairBytes;
     L.bar = L.v + (uint32_t)nsv * 16384u;
     L.misc = L.bar + kMaxBars * 8;
     L.bitmap = L.misc + 16;
@@ -88,12 +97,19 @@ __host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nword
     return L;
 }
 
-// barrier slots
-template <int NSK, int NSV>
+// Barrier slots.  Key slot / S buffer b (pair p uses b = p % 2) and value slot / P buffer s (chunk u
+// uses s = u % NSV):
+//   K_LAND[b]    the pair's key tiles have landed (TMA transaction count)
+//   QK_READY[b]  S buffer b may take pair p: its key tiles are in (the key loader's arrival) and all
+//                eight softmax warps have read pair p - 2 out of it
+//   QK_DONE[b]   the key product of pair p is complete: S is ready and the key slot is free
+//   V_LAND[s], PV_READY[s] (the value loader + the four softmax warps that wrote P), PV_DONE[s] alike
+// so the MMA issuer tests one barrier per product and commits to one.
+template <int NSV>
 struct Bars {
-    static constexpr int Q_FULL = 0, K_FULL = 1, K_EMPTY = 1 + NSK, V_FULL = 1 + 2 * NSK,
-                         V_EMPTY = 1 + 2 * NSK + NSV, S_FULL = 1 + 2 * NSK + 2 * NSV, P_FULL = S_FULL + kSB,
-                         P_EMPTY = P_FULL + kSB, O_FULL = P_EMPTY + kSB, MMA_DONE = O_FULL + 1;
+    static constexpr int Q_FULL = 0, K_LAND = 1, QK_READY = K_LAND + kSP, QK_DONE = QK_READY + kSP,
+                         V_LAND = QK_DONE + kSP, PV_READY = V_LAND + NSV, PV_DONE = PV_READY + NSV,
+                         O_FULL = PV_DONE + NSV, MMA_DONE = O_FULL + 1;
     static_assert(MMA_DONE < kMaxBars, "barrier slots");
 };
 
@@ -132,7 +148,60 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, unsigne
     return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
-template <int G, typename Tout, int NSK, int NSV>
+// One loader thread streams n tiles through a ring of `slots` buffers: tile i goes to slot i % slots
+// once the consumer has finished tile i - slots (its `done` barrier), lands on `land`, and is then
+// announced on `ready` (which other arrivals may share).  Up to `slots` tiles are in flight.  On an
+// abort the thread waits, with its own bound, for the copies it started.  Returns the tiles announced.
+template <typename Issue>
+__device__ __forceinline__ int stream_tiles(int n, int slots, uint32_t done0, uint32_t land0, uint32_t ready0,
+                                            Issue &&issue, unsigned long long limit_ns, volatile int *abort_flag,
+                                            unsigned int *status)
+{
+    int issued = 0, landed = 0;
+    long long t_prog = cycle_now();
+    bool ok = true;
+    while (landed < n) {
+        if (issued < n && issued < landed + slots &&
+            (issued < slots ||
+             mbar_test(done0 + 8u * (uint32_t)(issued % slots), (uint32_t)(((issued / slots) - 1) & 1)))) {
+            issue(issued);
+            ++issued;
+            t_prog = cycle_now();
+            continue;
+        }
+        const uint32_t lbar = land0 + 8u * (uint32_t)(landed % slots);
+        const uint32_t lphase = (uint32_t)((landed / slots) & 1);
+        if (landed < issued && mbar_test(lbar, lphase)) {
+            mbar_arrive(ready0 + 8u * (uint32_t)(landed % slots));
+            ++landed;
+            t_prog = cycle_now();
+            continue;
+        }
+        if (*abort_flag) {
+            ok = false;
+            break;
+        }
+        if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+        }
+        if (past_limit(t_prog, limit_ns)) {
+            *abort_flag = 1;
+            atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
+            ok = false;
+            break;
+        }
+        if (landed < issued) mbar_try_wait_sleep(lbar, lphase, 200u);
+        else mbar_try_wait_sleep(done0 + 8u * (uint32_t)(issued % slots), (uint32_t)(((issued / slots) - 1) & 1), 200u);
+    }
+    if (!ok)   // the copies must land before the CTA exits
+        for (int v = landed; v < issued; ++v)
+            mbar_drain(land0 + 8u * (uint32_t)(v % slots), (uint32_t)((v / slots) & 1), kDrainNs);
+    return landed;
+}
+
+template <int G, typename Tout, int NSV>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, Dims p, const int32_t *__restrict__ sel_idx,
@@ -140,13 +209,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                      unsigned long long limit_ns, int nwords, int inject_stall)
 {
     constexpr int BQ = kRows / G;
-    using BR = Bars<NSK, NSV>;
+    using BR = Bars<NSV>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    const Layout Ly = make_layout(NSK, NSV, p.k, nwords, BQ);
+    const Layout Ly = make_layout(kSP, NSV, p.k, nwords, BQ);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q0 = blockIdx.x * BQ, g = blockIdx.y, b = blockIdx.z;
+    // later query tiles select from more chunks and take longer: they are dispatched first, so that
+    // the grid ends on short blocks
+    const int q0 = (int)(gridDim.x - 1 - blockIdx.x) * BQ, g = blockIdx.y, b = blockIdx.z;
     const int nq = min(BQ, p.N - q0);
     const int ns = p.k + 1;
 
@@ -171,18 +242,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // fusion weights are built from there.
     if (tid == 0) {
         mbar_init(BAR(BR::Q_FULL), 1);
-        for (int s = 0; s < NSK; ++s) {
-            mbar_init(BAR(BR::K_FULL + s), 1);
-            mbar_init(BAR(BR::K_EMPTY + s), 1);
+        for (int s = 0; s < kSP; ++s) {
+            mbar_init(BAR(BR::K_LAND + s), 1);
+            mbar_init(BAR(BR::QK_READY + s), 1 + 4 * kGroups);
+            mbar_init(BAR(BR::QK_DONE + s), 1);
+            for (int a = 0; a < 4 * kGroups; ++a) mbar_arrive(BAR(BR::QK_READY + s));   // pairs 0, 1: S free
         }
         for (int s = 0; s < NSV; ++s) {
-            mbar_init(BAR(BR::V_FULL + s), 1);
-            mbar_init(BAR(BR::V_EMPTY + s), 1);
-        }
-        for (int s = 0; s < kSB; ++s) {
-            mbar_init(BAR(BR::S_FULL + s), 1);
-            mbar_init(BAR(BR::P_FULL + s), 4);
-            mbar_init(BAR(BR::P_EMPTY + s), 1);
+            mbar_init(BAR(BR::V_LAND + s), 1);
+            mbar_init(BAR(BR::PV_READY + s), 1 + 4);
+            mbar_init(BAR(BR::PV_DONE + s), 1);
         }
         mbar_init(BAR(BR::O_FULL), 1);
         mbar_init(BAR(BR::MMA_DONE), 1);
@@ -250,25 +319,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             running += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
         if (lane == 0) *n_union_p = running;
-    } else if (tid >= 32 && tid < 32 + nq) {
-        // each query's chunks (selected + own) in ascending order
-        const int qi = tid - 32;
-        int *lst = qlist + qi * ns;
-        int *slt = qslot + qi * ns;
-        int cnt = 0;
-        for (int j = 0; j <= p.k; ++j) {
-            const int c = (j < p.k) ? selbuf[qi * p.k + j] : (int)(((long long)p.q_offset + q0 + qi) / kChunk);
+    }
+    {
+        // each query's chunks (selected + own) in ascending order, with the slot each came from:
+        // one thread per (query, slot) counts the query's smaller chunks (chunks are distinct)
+        for (int e = tid - 32; e >= 0 && e < nq * ns; e += kThreads - 32) {
+            const int qi = e / ns, j = e % ns;
+            const int own_c = (int)(((long long)p.q_offset + q0 + qi) / kChunk);
+            const int *sl = selbuf + qi * p.k;
+            const int c = (j < p.k) ? sl[j] : own_c;
             if (c < 0) continue;
-            int at = cnt++;
-            while (at > 0 && lst[at - 1] > c) {
-                lst[at] = lst[at - 1];
-                slt[at] = slt[at - 1];
-                --at;
-            }
-            lst[at] = c;
-            slt[at] = j;    // the slot this chunk came from
+            int rank = 0;
+            for (int j2 = 0; j2 < p.k; ++j2) rank += (unsigned)sl[j2] < (unsigned)c;   // -1 never counts
+            rank += own_c < c;
+            qlist[qi * ns + rank] = c;
+            qslot[qi * ns + rank] = j;
+            if (j == p.k) qcnt[qi] = rank + 1;   // the own chunk is the largest
         }
-        qcnt[qi] = cnt;
     }
     __syncthreads();
 
@@ -298,49 +365,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int kv_row0 = (b * p.Hkv + g) * p.T;
     if (warp == 0) {
-        // ---------------- key tiles: up to NSK chunks ahead; a slot frees when its QK completes
+        // ---------------- key tiles, two chunks per slot; a slot frees when its key product completes
         if (lane == 0) {
-            int u = 0;
-            for (; u < n_union; ++u) {
-                const int st = u % NSK;
-                if (u >= NSK &&
-                    !mbar_wait(BAR(BR::K_EMPTY + st), (uint32_t)(((u / NSK) - 1) & 1), limit_ns, abort_flag, status))
-                    break;
-                const int row = kv_row0 + uni[u] * kChunk;
-                const uint32_t dst = sK + (uint32_t)st * 16384u;
-                mbar_arrive_expect_tx(BAR(BR::K_FULL + st), 16384u);
-                tma_load_2d(dst, &tmK, BAR(BR::K_FULL + st), 0, row);
-                tma_load_2d(dst + 8192u, &tmK, BAR(BR::K_FULL + st), 64, row);
-            }
-            // the copies must land before the CTA exits (only outstanding after an abort)
-            for (int v = max(0, u - NSK); v < u; ++v)
-                mbar_drain(BAR(BR::K_FULL + v % NSK), (uint32_t)((v / NSK) & 1), kDrainNs);
+            const int n_pairs = (n_union + 1) >> 1;
+            auto issue = [&](int pr) {
+                const int st = pr % kSP;
+                const bool two = 2 * pr + 1 < n_union;
+                const uint32_t dst = sK + (uint32_t)st * kPairBytes;
+                mbar_arrive_expect_tx(BAR(BR::K_LAND + st), two ? 32768u : 16384u);
+                const int row0 = kv_row0 + uni[2 * pr] * kChunk;
+                tma_load_2d(dst, &tmK, BAR(BR::K_LAND + st), 0, row0);
+                tma_load_2d(dst + 16384u, &tmK, BAR(BR::K_LAND + st), 64, row0);
+                if (two) {
+                    const int row1 = kv_row0 + uni[2 * pr + 1] * kChunk;
+                    tma_load_2d(dst + 8192u, &tmK, BAR(BR::K_LAND + st), 0, row1);
+                    tma_load_2d(dst + 24576u, &tmK, BAR(BR::K_LAND + st), 64, row1);
+                }
+            };
+            const int landed = stream_tiles(n_pairs, kSP, BAR(BR::QK_DONE), BAR(BR::K_LAND), BAR(BR::QK_READY), issue,
+                                            limit_ns, abort_flag, status);
+            (void)landed;
             mbar_drain(BAR(BR::Q_FULL), 0, kDrainNs);
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- value tiles: up to NSV chunks ahead; a slot frees when its PV completes
+        // ---------------- value tiles, one chunk per slot; a slot frees when its value product completes
         if (lane == 0) {
-            int u = 0;
-            for (; u < n_union; ++u) {
+            auto issue = [&](int u) {
                 const int st = u % NSV;
-                if (u >= NSV &&
-                    !mbar_wait(BAR(BR::V_EMPTY + st), (uint32_t)(((u / NSV) - 1) & 1), limit_ns, abort_flag, status))
-                    break;
                 const int row = kv_row0 + uni[u] * kChunk;
                 const uint32_t dst = sV + (uint32_t)st * 16384u;
-                mbar_arrive_expect_tx(BAR(BR::V_FULL + st), 16384u);
-                tma_load_2d(dst, &tmV, BAR(BR::V_FULL + st), 0, row);
-                tma_load_2d(dst + 8192u, &tmV, BAR(BR::V_FULL + st), 64, row);
-            }
-            for (int v = max(0, u - NSV); v < u; ++v)
-                mbar_drain(BAR(BR::V_FULL + v % NSV), (uint32_t)((v / NSV) & 1), kDrainNs);
+                mbar_arrive_expect_tx(BAR(BR::V_LAND + st), 16384u);
+                tma_load_2d(dst, &tmV, BAR(BR::V_LAND + st), 0, row);
+                tma_load_2d(dst + 8192u, &tmV, BAR(BR::V_LAND + st), 64, row);
+            };
+            stream_tiles(n_union, NSV, BAR(BR::PV_DONE), BAR(BR::V_LAND), BAR(BR::PV_READY), issue, limit_ns,
+                         abort_flag, status);
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ---------------- MMA issue: QK runs kLookahead chunks ahead of PV -----------------
-        // Schedule: QK(0..L-1), then for each u: PV(u), QK(u+L).  QK(t) reuses the S buffer of
-        // chunk t - kSB, whose PV (and so its softmax) came earlier in this order (L < kSB).
+        // ---------------- MMA issue -------------------------------------------------------------
+        // The tensor core takes one MMA at a time from this thread (the issue returns about when the
+        // previous one is done), so the thread polls: the next key product whenever its keys are in and
+        // its S buffer has been read, else the next value product whenever its P and V are ready.
         if (lane == 0) {
             bool ok = true;
             if (inject_stall) {
@@ -348,42 +415,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = mbar_wait(BAR(BR::MMA_DONE), 0, limit_ns, abort_flag, status);
             }
             ok = ok && mbar_wait(BAR(BR::Q_FULL), 0, limit_ns, abort_flag, status);
-            auto issue_qk = [&](int t) -> bool {
-                const int kst = t % NSK;
-                if (!mbar_wait(BAR(BR::K_FULL + kst), (uint32_t)((t / NSK) & 1), limit_ns, abort_flag, status))
-                    return false;
-                tc_fence_after();
-                const uint32_t d_s = tmem + (uint32_t)(t % kSB) * 64u;
-                const uint32_t ka = sK + (uint32_t)kst * 16384u;
+            const int n_pairs = (n_union + 1) >> 1;
+            // descriptors: Q's eight K-steps, and the two key slots' and NSV value slots' bases
+            uint64_t dq[8];
 #pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16_ss(d_s, smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
-                                smem_desc_sw128(ka + (s >> 2) * 8192u + (s & 3) * 32u, 16, 1024), IDESC_QK,
-                                s > 0 ? 1u : 0u);
-                mma_commit(BAR(BR::S_FULL + t % kSB));
-                mma_commit(BAR(BR::K_EMPTY + kst));
-                return true;
-            };
-            auto issue_pv = [&](int u) -> bool {
-                const int vst = u % NSV;
-                if (!mbar_wait(BAR(BR::P_FULL + u % kSB), (uint32_t)((u / kSB) & 1), limit_ns, abort_flag, status) ||
-                    !mbar_wait(BAR(BR::V_FULL + vst), (uint32_t)((u / NSV) & 1), limit_ns, abort_flag, status))
-                    return false;
-                tc_fence_after();
-                const uint32_t pa = tmem + kColP + (uint32_t)(u % kSB) * 32u;
-                const uint32_t va = sV + (uint32_t)vst * 16384u;
+            for (int s = 0; s < 8; ++s) dq[s] = smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024);
+            int qp = 0, pu = 0;
+            long long t_prog = cycle_now();
+            while (ok && pu < n_union) {
+                if (qp < n_pairs && mbar_test(BAR(BR::QK_READY + qp % kSP), (uint32_t)((qp / kSP) & 1))) {
+                    tc_fence_after();
+                    const uint32_t d_s = tmem + (uint32_t)(qp % kSP) * 128u;
+                    const uint64_t dk = smem_desc_sw128(sK + (uint32_t)(qp % kSP) * kPairBytes, 16, 1024);
+                    const uint32_t idesc = (2 * qp + 1 < n_union) ? IDESC_QK2 : IDESC_QK1;
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_f16_ts(tmem + kColO, pa + 8u * s, smem_desc_sw128(va + 2048u * s, 8192, 1024), IDESC_PV,
-                               (u > 0 || s > 0) ? 1u : 0u);
-                mma_commit(BAR(BR::V_EMPTY + vst));
-                mma_commit(BAR(BR::P_EMPTY + u % kSB));
-                return true;
-            };
-            for (int t = 0; ok && t < min(kLookahead, n_union); ++t) ok = issue_qk(t);
-            for (int u = 0; ok && u < n_union; ++u) {
-                ok = issue_pv(u);
-                if (ok && u + kLookahead < n_union) ok = issue_qk(u + kLookahead);
+                    for (int s = 0; s < 8; ++s)
+                        mma_bf16_ss(d_s, dq[s], dk + (uint64_t)(((s >> 2) * 16384u + (s & 3) * 32u) >> 4), idesc,
+                                    s > 0 ? 1u : 0u);
+                    mma_commit(BAR(BR::QK_DONE + qp % kSP));
+                    ++qp;
+                    t_prog = cycle_now();
+                    continue;
+                }
+                const uint32_t pbar = BAR(BR::PV_READY + pu % NSV);
+                const uint32_t pphase = (uint32_t)((pu / NSV) & 1);
+                if (mbar_test(pbar, pphase)) {
+                    tc_fence_after();
+                    const uint32_t pa = tmem + kColP + (uint32_t)(pu % NSV) * 32u;
+                    const uint64_t dv = smem_desc_sw128(sV + (uint32_t)(pu % NSV) * 16384u, 8192, 1024);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_f16_ts(tmem + kColO, pa + 8u * s, dv + (uint64_t)((2048u * s) >> 4), IDESC_PV,
+                                   (pu > 0 || s > 0) ? 1u : 0u);
+                    mma_commit(BAR(BR::PV_DONE + pu % NSV));
+                    ++pu;
+                    t_prog = cycle_now();
+                    continue;
+                }
+                // nothing ready: bounded, sleeping wait for the next P (the usual next event)
+                if (*abort_flag) {
+                    ok = false;
+                    break;
+                }
+                if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                if (past_limit(t_prog, limit_ns)) {
+                    *abort_flag = 1;
+                    atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
+                    ok = false;
+                    break;
+                }
+                mbar_try_wait_sleep(pbar, pphase, 100u);
             }
             if (ok) mma_commit(BAR(BR::O_FULL));
             // drain: every issued MMA completes before TMEM is released
@@ -407,17 +492,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         int ptr = 0;
         bool ok = true;
         for (int t = grp; t < n_union; t += kGroups) {
-            const int bsel = t % kSB, u = t / kSB;
-            if (!warp_wait(BAR(BR::S_FULL + bsel), (uint32_t)(u & 1), limit_ns, abort_flag, status)) {
+            const int pr = t >> 1, sb = pr % kSP, pb = t % NSV;
+            if (!warp_wait(BAR(BR::QK_DONE + sb), (uint32_t)((pr / kSP) & 1), limit_ns, abort_flag, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             uint32_t sv[64];
-            const uint32_t tS = tmem + lane_off + (uint32_t)bsel * 64u;
+            const uint32_t tS = tmem + lane_off + (uint32_t)sb * 128u + (uint32_t)(t & 1) * 64u;
             tmem_ld32(tS, sv);
             tmem_ld32(tS + 32u, sv + 32);
             tmem_wait_ld();
+            // the scores are in registers: the S buffer may take the pair after next
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(BR::QK_READY + sb));
 
             const int c = uni[t];
             while (ptr < cnt && lst[ptr] < c) ++ptr;
@@ -425,52 +514,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[32];
             if (w > 0.f) {
                 const int n_vis = (c == own) ? (int)(pos - (long long)c * kChunk + 1) : kChunk;
-                if (n_vis < kChunk) {
-#pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        if (j >= n_vis) sv[j] = __float_as_uint(-INFINITY);
-                }
-                float mx[8];
-#pragma unroll
-                for (int a = 0; a < 8; ++a) mx[a] = __uint_as_float(sv[a]);
-#pragma unroll
-                for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sv[j]));
-                const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                const float nb = -m * sl2;
-                float ls[8];
-#pragma unroll
-                for (int a = 0; a < 8; ++a) ls[a] = 0.f;
-                // one exponential in kPolyEvery on the FMA pipe, the rest on the special-function unit;
-                // masked keys hold -inf and give 0 either way
-#pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const float x = fmaf(__uint_as_float(sv[j]), sl2, nb);
-                    const float e = (j % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x) : ex2_approx(x);
-                    sv[j] = __float_as_uint(e);
-                    ls[j & 7] += e;
-                }
-                const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-                const float f = w / l;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    __half2 v2 = __floats2half2_rn(__uint_as_float(sv[2 * j]) * f, __uint_as_float(sv[2 * j + 1]) * f);
-                    pk[j] = *reinterpret_cast<uint32_t *>(&v2);
-                }
+                chunk_softmax_row<kPolyPairEvery>(sv, n_vis, w, sl2, pk);
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) pk[j] = 0u;
             }
-            if (t >= kSB &&
-                !warp_wait(BAR(BR::P_EMPTY + bsel), (uint32_t)((u - 1) & 1), limit_ns, abort_flag, status)) {
+            if (t >= NSV &&
+                !warp_wait(BAR(BR::PV_DONE + pb), (uint32_t)(((t / NSV) - 1) & 1), limit_ns, abort_flag, status)) {
                 ok = false;
                 break;
             }
-            tmem_st32(tmem + lane_off + kColP + (uint32_t)bsel * 32u, pk);
+            tmem_st32(tmem + lane_off + kColP + (uint32_t)pb * 32u, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(BR::P_FULL + bsel));
+            if (lane == 0) mbar_arrive(BAR(BR::PV_READY + pb));
         }
         if (ok && warp_wait(BAR(BR::O_FULL), 0, limit_ns, abort_flag, status)) {
             tc_fence_after();
@@ -543,12 +601,12 @@ __global__ void v_to_f16_kernel(const uint4 *__restrict__ in, uint4 *__restrict_
 
 constexpr int kSmemLimit = 227 * 1024;
 
-// Deepest key/value rings that fit: 0 = (6, 4), 1 = (4, 3), 2 = (2, 2), -1 = none.
+// Deepest value ring that fits (the key ring always has kSP pair slots): 0 = 4 value tiles,
+// 1 = 2, -1 = none.
 int ring_config(int k, int nwords, int BQ)
 {
-    if (make_layout(6, 4, k, nwords, BQ).total + 1024 <= kSmemLimit) return 0;
-    if (make_layout(4, 3, k, nwords, BQ).total + 1024 <= kSmemLimit) return 1;
-    if (make_layout(2, 2, k, nwords, BQ).total + 1024 <= kSmemLimit) return 2;
+    if (make_layout(kSP, 4, k, nwords, BQ).total + 1024 <= kSmemLimit) return 0;
+    if (make_layout(kSP, 2, k, nwords, BQ).total + 1024 <= kSmemLimit) return 1;
     return -1;
 }
 
@@ -573,19 +631,18 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V,
     dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
     const int cfg = ring_config(p.k, nwords, BQ);
     cudaError_t e = cudaErrorInvalidValue;
-#define HILS_LAUNCH_TC(NK, NV)                                                                              \
+#define HILS_LAUNCH_TC(NV)                                                                                  \
     {                                                                                                        \
-        const size_t smem = make_layout(NK, NV, p.k, nwords, BQ).total + 1024;                              \
-        auto kern = attend_tc_kernel<G, Tout, NK, NV>;                                                      \
+        const size_t smem = make_layout(kSP, NV, p.k, nwords, BQ).total + 1024;                             \
+        auto kern = attend_tc_kernel<G, Tout, NV>;                                                          \
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);              \
         if (e != cudaSuccess) return e;                                                                      \
         kern<<<grid, kThreads, smem, s>>>(tq, tk, tv, p, sel_idx, sel_score, static_cast<Tout *>(O),         \
                                           ctl.status, (unsigned long long)ctl.wait_limit, nwords,            \
                                           ctl.inject_stall);                                                 \
     }
-    if (cfg == 0) HILS_LAUNCH_TC(6, 4)
-    else if (cfg == 1) HILS_LAUNCH_TC(4, 3)
-    else HILS_LAUNCH_TC(2, 2)
+    if (cfg == 0) HILS_LAUNCH_TC(4)
+    else HILS_LAUNCH_TC(2)
 #undef HILS_LAUNCH_TC
     return cudaGetLastError();
 }

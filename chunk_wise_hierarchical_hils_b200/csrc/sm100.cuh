@@ -16,11 +16,15 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p)
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ unsigned long long global_timer_ns()
+// Time bounds run on the SM's cycle counter: reading it costs a few cycles, where the global
+// nanosecond timer costs hundreds, which a polling loop on the critical path cannot afford.  A bound
+// of limit_ns is taken as 2 cycles per ns; the SM clock stays below 2 GHz, so the bound lasts at
+// least limit_ns (longer when the clock is lower).
+__device__ __forceinline__ long long cycle_now() { return clock64(); }
+
+__device__ __forceinline__ bool past_limit(long long t0, unsigned long long limit_ns)
 {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
+    return (unsigned long long)(clock64() - t0) > 2ull * limit_ns;
 }
 
 // ---- mbarrier ---------------------------------------------------------------
@@ -96,15 +100,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
                                           volatile int *abort_flag, unsigned int *status)
 {
+    // a short spin first: most phases this wait is used for complete within a few hundred cycles
+    for (int i = 0; i < 32; ++i)
+        if (mbar_test(bar, parity)) return true;
     if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_timer_ns();
+    const long long t0 = cycle_now();
     for (;;) {
         if (*abort_flag) return false;
         if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
             *abort_flag = 1;
             return false;
         }
-        if (global_timer_ns() - t0 > limit_ns) {
+        if (past_limit(t0, limit_ns)) {
             *abort_flag = 1;
             atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
             return false;
@@ -116,9 +123,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 // Bounded wait used while draining at exit: no abort flag, its own limit.
 __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, unsigned long long limit_ns)
 {
-    const unsigned long long t0 = global_timer_ns();
+    const long long t0 = cycle_now();
     while (!mbar_try_wait(bar, parity))
-        if (global_timer_ns() - t0 > limit_ns) return false;
+        if (past_limit(t0, limit_ns)) return false;
     return true;
 }
 
@@ -254,6 +261,79 @@ __device__ __forceinline__ float exp2_poly(float x)
     const int n = __float_as_int(t) - __float_as_int(magic);
     const float p = fmaf(fmaf(fmaf(fmaf(0.0096003953f, f, 0.055916894f), f, 0.24023719f), f, 0.69312197f), f, 1.0f);
     return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// ---- packed float32 pairs (sm_100 f32x2 arithmetic, round to nearest, no flush) ----------
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_splat(float x) { return f2_pack(x, x); }
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// exp2_poly on a pair: the same float32 steps, rounding and coefficients, two lanes per
+// instruction where the f32x2 forms exist
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t xx)
+{
+    float x0, x1;
+    f2_unpack(xx, x0, x1);
+    const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t magic = f2_splat(12582912.0f);
+    const uint64_t t = f2_add(x, magic);
+    const uint64_t f = f2_sub(x, f2_sub(t, magic));
+    float t0, t1;
+    f2_unpack(t, t0, t1);
+    const int n0 = __float_as_int(t0) - __float_as_int(12582912.0f);
+    const int n1 = __float_as_int(t1) - __float_as_int(12582912.0f);
+    const uint64_t p = f2_fma(f2_fma(f2_fma(f2_fma(f2_splat(0.0096003953f), f, f2_splat(0.055916894f)), f,
+                                            f2_splat(0.24023719f)), f, f2_splat(0.69312197f)), f, f2_splat(1.0f));
+    float p0, p1;
+    f2_unpack(p, p0, p1);
+    return f2_pack(__int_as_float(__float_as_int(p0) + (n0 << 23)), __int_as_float(__float_as_int(p1) + (n1 << 23)));
 }
 
 // 2^x on the special-function unit (flushes subnormal results to zero)

@@ -23,6 +23,19 @@ def coeffs():
     return [np.float32(x) for x in nums]   # highest degree first
 
 
+def pair_coeffs():
+    """Coefficients of the two-lane form, in the order they appear (highest degree first)."""
+    src = open(HDR).read()
+    body = src[src.index("exp2_poly_x2("):]
+    body = body[body.index("const uint64_t p ="):]
+    body = body[:body.index(";")]
+    return [np.float32(float(x.rstrip("f"))) for x in re.findall(r"f2_splat\(([0-9.e-]+f)\)", body)]
+
+
+def test_pair_form_uses_the_same_coefficients():
+    assert pair_coeffs() == coeffs()
+
+
 def fma32(a, b, c):
     return (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(np.float32)
 
