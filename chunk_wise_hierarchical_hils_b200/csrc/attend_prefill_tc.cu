@@ -9,26 +9,28 @@
 //   Sec. 4 "Architecture": a GQA group's heads share the retrieved chunks.
 //
 // One CTA owns 128 rows = (128 / G) consecutive queries x the G heads of one
-// kv-group (row r = head * (128 / G) + query).  It walks the union of the
+// kv-group (row r = query * G + head, so that a warp's 32 rows cover 32 / G
+// whole queries and can skip a chunk none of them selected).  It walks the union of the
 // chunks its queries selected, in ascending chunk order, with warp-specialised
 // roles that meet on mbarriers:
 //   warp 0 (one thread)  TMA loads of Q once and of the union's K tiles, two
 //                        chunks per ring slot (128-byte swizzle, no multicast);
-//   warp 1 (one thread)  TMA loads of the V tiles, one chunk per ring slot;
+//   warp 1 (one thread)  TMA loads of the V tiles, two chunks per ring slot;
 //                        the warp also owns the TMEM allocation;
 //   warp 2 (one thread)  tcgen05.mma issue.  S = Q K^T (bf16, A and B from
 //                        shared memory) runs on two chunks at once (N = 128,
 //                        the tensor core's efficient width) into one of two
 //                        TMEM S buffers; O += P V (f16, P from TMEM, V from
-//                        shared memory) per chunk.  The issuer polls which of
-//                        the two is ready, key products first, so the softmax
-//                        warps never wait behind a value product;
+//                        shared memory) on the same pairs (K = 128 keys).  The
+//                        issuer polls which of the two is ready, key products
+//                        first, so the softmax warps never wait behind a value
+//                        product;
 //   warps 4..11          two groups of four warps, one thread per row; group
 //                        t % 2 handles chunk t: it reads S from TMEM (and frees
 //                        the S buffer at once), takes the softmax over the
 //                        chunk's visible keys, scales it by the row's fusion
 //                        weight (0 if the row's query did not select the chunk)
-//                        and writes P (f16) to one of four TMEM P buffers.  At
+//                        and writes P (f16) to its half of a TMEM P buffer.  At
 //                        the end both groups read O from TMEM and store it.
 // Because each chunk's softmax is normalised on its own and the fusion weights
 // are known before the loop, P already carries w_c / l_c and the accumulator
@@ -56,9 +58,9 @@ constexpr int kChunk = 64;        // C
 constexpr int kD = 128;           // d
 constexpr int kSP = 2;                // S buffers (a pair of chunks, 128 columns each) = key ring slots
 constexpr int kGroups = 2;            // softmax warp groups; group t % kGroups handles chunk t
-constexpr uint32_t kTmemCols = 512;   // S pair buffers (2 x 128 columns), O (128), up to 4 P buffers (32 each)
+constexpr uint32_t kTmemCols = 512;   // S pair buffers (2 x 128 columns), O (128), up to 2 P pair buffers (64 each)
 constexpr uint32_t kColO = 256, kColP = 384;
-constexpr uint32_t kPairBytes = 32768;   // K ring slot: [c0 d0-63 | c1 d0-63 | c0 d64-127 | c1 d64-127]
+constexpr uint32_t kPairBytes = 32768;   // K and V ring slots: [c0 d0-63 | c1 d0-63 | c0 d64-127 | c1 d64-127]
 constexpr unsigned long long kDrainNs = 2000000000ull;
 constexpr int kPolyPairEvery = 4; // exponential pairs computed by exp2_poly_x2: 1 in kPolyPairEvery
 
@@ -74,8 +76,8 @@ __host__ __device__ inline uint32_t al16(uint32_t x) { return (x + 15u) & ~15u; 
 
 constexpr int kMaxBars = 64;
 
-// Shared memory: Q (32 KB), kSP key slots (two chunks, 32 KB each) and a ring of NSV
-// value tiles (16 KB each), barriers, then the block's selection bookkeeping.
+// Shared memory: Q (32 KB), kSP key slots and NSV value slots (two chunks, 32 KB each), barriers,
+// then the block's selection bookkeeping.
 __host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nwords, int BQ)
 {
     Layout L;
@@ -83,7 +85,7 @@ __host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nword
     L.q = 0;
     L.k = 32768;
     L.v = L.k + (uint32_t)nsk * kPairBytes;
-    L.bar = L.v + (uint32_t)nsv * 16384u;
+    L.bar = L.v + (uint32_t)nsv * kPairBytes;
     L.misc = L.bar + kMaxBars * 8;
     L.bitmap = L.misc + 16;
     L.uni = al16(L.bitmap + 4u * (uint32_t)nwords);
@@ -97,13 +99,13 @@ __host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nword
     return L;
 }
 
-// Barrier slots.  Key slot / S buffer b (pair p uses b = p % 2) and value slot / P buffer s (chunk u
-// uses s = u % NSV):
+// Barrier slots.  Key slot / S buffer b (pair p uses b = p % 2) and value slot / P buffer s (pair p
+// uses s = p % NSV):
 //   K_LAND[b]    the pair's key tiles have landed (TMA transaction count)
 //   QK_READY[b]  S buffer b may take pair p: its key tiles are in (the key loader's arrival) and all
 //                eight softmax warps have read pair p - 2 out of it
 //   QK_DONE[b]   the key product of pair p is complete: S is ready and the key slot is free
-//   V_LAND[s], PV_READY[s] (the value loader + the four softmax warps that wrote P), PV_DONE[s] alike
+//   V_LAND[s], PV_READY[s] (the value loader + the eight softmax warps that wrote P), PV_DONE[s] alike
 // so the MMA issuer tests one barrier per product and commits to one.
 template <int NSV>
 struct Bars {
@@ -150,12 +152,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, unsigne
 
 // One loader thread streams n tiles through a ring of `slots` buffers: tile i goes to slot i % slots
 // once the consumer has finished tile i - slots (its `done` barrier), lands on `land`, and is then
-// announced on `ready` (which other arrivals may share).  Up to `slots` tiles are in flight.  On an
-// abort the thread waits, with its own bound, for the copies it started.  Returns the tiles announced.
+// announced on `ready` (which other arrivals may share; the last tile's announcement counts
+// 1 + tail_extra arrivals).  Up to `slots` tiles are in flight.  On an abort the thread waits, with its
+// own bound, for the copies it started.  Returns the tiles announced.
 template <typename Issue>
 __device__ __forceinline__ int stream_tiles(int n, int slots, uint32_t done0, uint32_t land0, uint32_t ready0,
-                                            Issue &&issue, unsigned long long limit_ns, volatile int *abort_flag,
-                                            unsigned int *status)
+                                            Issue &&issue, int tail_extra, unsigned long long limit_ns,
+                                            volatile int *abort_flag, unsigned int *status)
 {
     int issued = 0, landed = 0;
     long long t_prog = cycle_now();
@@ -172,7 +175,8 @@ __device__ __forceinline__ int stream_tiles(int n, int slots, uint32_t done0, ui
         const uint32_t lbar = land0 + 8u * (uint32_t)(landed % slots);
         const uint32_t lphase = (uint32_t)((landed / slots) & 1);
         if (landed < issued && mbar_test(lbar, lphase)) {
-            mbar_arrive(ready0 + 8u * (uint32_t)(landed % slots));
+            const int n_arrive = (landed == n - 1) ? 1 + tail_extra : 1;
+            for (int a = 0; a < n_arrive; ++a) mbar_arrive(ready0 + 8u * (uint32_t)(landed % slots));
             ++landed;
             t_prog = cycle_now();
             continue;
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < NSV; ++s) {
             mbar_init(BAR(BR::V_LAND + s), 1);
-            mbar_init(BAR(BR::PV_READY + s), 1 + 4);
+            mbar_init(BAR(BR::PV_READY + s), 1 + 4 * kGroups);
             mbar_init(BAR(BR::PV_DONE + s), 1);
         }
         mbar_init(BAR(BR::O_FULL), 1);
@@ -261,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
         mbar_arrive_expect_tx(BAR(BR::Q_FULL), 32768u);
-        tma_load_3d(sQ, &tmQ, BAR(BR::Q_FULL), 0, q0, b * p.H + g * G);
-        tma_load_3d(sQ + 16384u, &tmQ, BAR(BR::Q_FULL), 64, q0, b * p.H + g * G);
+        tma_load_3d(sQ, &tmQ, BAR(BR::Q_FULL), 0, b * p.H + g * G, q0);
+        tma_load_3d(sQ + 16384u, &tmQ, BAR(BR::Q_FULL), 64, b * p.H + g * G, q0);
     }
     if (warp == 1) {
         tmem_alloc(smem_addr(tmem_holder), kTmemCols);
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int e = tid; e < G * nq * ns; e += kThreads) {
         const int h = e / (nq * ns), rem = e % (nq * ns);
         const size_t row0 = (((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0;
-        scbuf[(h * BQ + rem / ns) * ns + rem % ns] = __ldg(sel_score + row0 * ns + rem);
+        scbuf[((rem / ns) * G + h) * ns + rem % ns] = __ldg(sel_score + row0 * ns + rem);
     }
     __syncthreads();
 
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid < kRows) {
         // fusion weights of each row, in the order of its query's chunk list
-        const int r = tid, qi = r % BQ;
+        const int r = tid, qi = r / G;
         if (qi < nq) {
             const float *sc = scbuf + r * ns;
             float M = -INFINITY;
@@ -383,24 +387,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             };
             const int landed = stream_tiles(n_pairs, kSP, BAR(BR::QK_DONE), BAR(BR::K_LAND), BAR(BR::QK_READY), issue,
-                                            limit_ns, abort_flag, status);
+                                            0, limit_ns, abort_flag, status);
             (void)landed;
             mbar_drain(BAR(BR::Q_FULL), 0, kDrainNs);
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- value tiles, one chunk per slot; a slot frees when its value product completes
+        // ---------------- value tiles, two chunks per slot; a slot frees when its value product completes
         if (lane == 0) {
-            auto issue = [&](int u) {
-                const int st = u % NSV;
-                const int row = kv_row0 + uni[u] * kChunk;
-                const uint32_t dst = sV + (uint32_t)st * 16384u;
-                mbar_arrive_expect_tx(BAR(BR::V_LAND + st), 16384u);
-                tma_load_2d(dst, &tmV, BAR(BR::V_LAND + st), 0, row);
-                tma_load_2d(dst + 8192u, &tmV, BAR(BR::V_LAND + st), 64, row);
+            const int n_pairs = (n_union + 1) >> 1;
+            auto issue = [&](int pr) {
+                const int st = pr % NSV;
+                const bool two = 2 * pr + 1 < n_union;
+                const uint32_t dst = sV + (uint32_t)st * kPairBytes;
+                mbar_arrive_expect_tx(BAR(BR::V_LAND + st), two ? 32768u : 16384u);
+                const int row0 = kv_row0 + uni[2 * pr] * kChunk;
+                tma_load_2d(dst, &tmV, BAR(BR::V_LAND + st), 0, row0);
+                tma_load_2d(dst + 16384u, &tmV, BAR(BR::V_LAND + st), 64, row0);
+                if (two) {
+                    const int row1 = kv_row0 + uni[2 * pr + 1] * kChunk;
+                    tma_load_2d(dst + 8192u, &tmV, BAR(BR::V_LAND + st), 0, row1);
+                    tma_load_2d(dst + 24576u, &tmV, BAR(BR::V_LAND + st), 64, row1);
+                }
             };
-            stream_tiles(n_union, NSV, BAR(BR::PV_DONE), BAR(BR::V_LAND), BAR(BR::PV_READY), issue, limit_ns,
-                         abort_flag, status);
+            // a lone last chunk has no second softmax group to announce its P: the loader stands in
+            stream_tiles(n_pairs, NSV, BAR(BR::PV_DONE), BAR(BR::V_LAND), BAR(BR::PV_READY), issue, (n_union & 1) ? 4 : 0,
+                         limit_ns, abort_flag, status);
         }
         __syncwarp();
     } else if (warp == 2) {
@@ -416,13 +428,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ok = ok && mbar_wait(BAR(BR::Q_FULL), 0, limit_ns, abort_flag, status);
             const int n_pairs = (n_union + 1) >> 1;
-            // descriptors: Q's eight K-steps, and the two key slots' and NSV value slots' bases
+            // descriptors of Q's eight K-steps
             uint64_t dq[8];
 #pragma unroll
             for (int s = 0; s < 8; ++s) dq[s] = smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024);
-            int qp = 0, pu = 0;
+            int qp = 0, vp = 0;
+            unsigned idle = 0;
             long long t_prog = cycle_now();
-            while (ok && pu < n_union) {
+            while (ok && vp < n_pairs) {
                 if (qp < n_pairs && mbar_test(BAR(BR::QK_READY + qp % kSP), (uint32_t)((qp / kSP) & 1))) {
                     tc_fence_after();
                     const uint32_t d_s = tmem + (uint32_t)(qp % kSP) * 128u;
@@ -437,27 +450,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                     t_prog = cycle_now();
                     continue;
                 }
-                const uint32_t pbar = BAR(BR::PV_READY + pu % NSV);
-                const uint32_t pphase = (uint32_t)((pu / NSV) & 1);
+                const uint32_t pbar = BAR(BR::PV_READY + vp % NSV);
+                const uint32_t pphase = (uint32_t)((vp / NSV) & 1);
                 if (mbar_test(pbar, pphase)) {
                     tc_fence_after();
-                    const uint32_t pa = tmem + kColP + (uint32_t)(pu % NSV) * 32u;
-                    const uint64_t dv = smem_desc_sw128(sV + (uint32_t)(pu % NSV) * 16384u, 8192, 1024);
+                    const uint32_t pa = tmem + kColP + (uint32_t)(vp % NSV) * 64u;
+                    const uint64_t dv = smem_desc_sw128(sV + (uint32_t)(vp % NSV) * kPairBytes, 16384, 1024);
+                    const int steps = (2 * vp + 1 < n_union) ? 8 : 4;
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_f16_ts(tmem + kColO, pa + 8u * s, dv + (uint64_t)((2048u * s) >> 4), IDESC_PV,
-                                   (pu > 0 || s > 0) ? 1u : 0u);
-                    mma_commit(BAR(BR::PV_DONE + pu % NSV));
-                    ++pu;
+                    for (int s = 0; s < 8; ++s)
+                        if (s < steps)
+                            mma_f16_ts(tmem + kColO, pa + 8u * s, dv + (uint64_t)((2048u * s) >> 4), IDESC_PV,
+                                       (vp > 0 || s > 0) ? 1u : 0u);
+                    mma_commit(BAR(BR::PV_DONE + vp % NSV));
+                    ++vp;
                     t_prog = cycle_now();
                     continue;
                 }
-                // nothing ready: bounded, sleeping wait for the next P (the usual next event)
+                // nothing ready: poll again (a test takes ~100 cycles, so the loop costs few issue
+                // slots and reacts at once); the grid's status word is read only now and then
                 if (*abort_flag) {
                     ok = false;
                     break;
                 }
-                if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
+                if ((++idle & 63) == 0 && *reinterpret_cast<volatile unsigned int *>(status) != 0u) {
                     *abort_flag = 1;
                     ok = false;
                     break;
@@ -468,7 +484,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                mbar_try_wait_sleep(pbar, pphase, 100u);
             }
             if (ok) mma_commit(BAR(BR::O_FULL));
             // drain: every issued MMA completes before TMEM is released
@@ -480,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- softmax (kGroups groups, alternate chunks) and epilogue ----
         const int grp = (warp - 4) >> 2;
         const int qq = warp & 3;
-        const int r = 32 * qq + lane, h = r / BQ, qi = r % BQ;
+        const int r = 32 * qq + lane, h = r % G, qi = r / G;
         const bool valid = qi < nq;
         const long long pos = (long long)p.q_offset + q0 + qi;
         const int own = (int)(pos / kChunk);
@@ -492,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int ptr = 0;
         bool ok = true;
         for (int t = grp; t < n_union; t += kGroups) {
-            const int pr = t >> 1, sb = pr % kSP, pb = t % NSV;
+            const int pr = t >> 1, sb = pr % kSP, pb = pr % NSV;
             if (!warp_wait(BAR(BR::QK_DONE + sb), (uint32_t)((pr / kSP) & 1), limit_ns, abort_flag, status)) {
                 ok = false;
                 break;
@@ -512,19 +527,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (ptr < cnt && lst[ptr] < c) ++ptr;
             const float w = (ptr < cnt && lst[ptr] == c) ? wr[ptr] : 0.f;
             uint32_t pk[32];
-            if (w > 0.f) {
+            if (__any_sync(0xFFFFFFFFu, w > 0.f)) {   // rows with w = 0 get P = 0 from the scaling
                 const int n_vis = (c == own) ? (int)(pos - (long long)c * kChunk + 1) : kChunk;
                 chunk_softmax_row<kPolyPairEvery>(sv, n_vis, w, sl2, pk);
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) pk[j] = 0u;
             }
-            if (t >= NSV &&
-                !warp_wait(BAR(BR::PV_DONE + pb), (uint32_t)(((t / NSV) - 1) & 1), limit_ns, abort_flag, status)) {
+            if (pr >= NSV &&
+                !warp_wait(BAR(BR::PV_DONE + pb), (uint32_t)(((pr / NSV) - 1) & 1), limit_ns, abort_flag, status)) {
                 ok = false;
                 break;
             }
-            tmem_st32(tmem + lane_off + kColP + (uint32_t)pb * 32u, pk);
+            tmem_st32(tmem + lane_off + kColP + (uint32_t)pb * 64u + (uint32_t)(t & 1) * 32u, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -601,12 +616,12 @@ __global__ void v_to_f16_kernel(const uint4 *__restrict__ in, uint4 *__restrict_
 
 constexpr int kSmemLimit = 227 * 1024;
 
-// Deepest value ring that fits (the key ring always has kSP pair slots): 0 = 4 value tiles,
-// 1 = 2, -1 = none.
+// Deepest value ring that fits (the key ring always has kSP pair slots): 0 = 2 value pair slots,
+// 1 = 1, -1 = none.
 int ring_config(int k, int nwords, int BQ)
 {
-    if (make_layout(kSP, 4, k, nwords, BQ).total + 1024 <= kSmemLimit) return 0;
-    if (make_layout(kSP, 2, k, nwords, BQ).total + 1024 <= kSmemLimit) return 1;
+    if (make_layout(kSP, 2, k, nwords, BQ).total + 1024 <= kSmemLimit) return 0;
+    if (make_layout(kSP, 1, k, nwords, BQ).total + 1024 <= kSmemLimit) return 1;
     return -1;
 }
 
@@ -616,9 +631,10 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V,
 {
     constexpr int BQ = kRows / G;
     CUtensorMap tq, tk, tv;
-    const cuuint64_t qd[3] = {(cuuint64_t)kD, (cuuint64_t)p.N, (cuuint64_t)p.B * p.H};
-    const cuuint64_t qs[2] = {(cuuint64_t)kD * 2, (cuuint64_t)p.N * kD * 2};
-    const cuuint32_t qb[3] = {64, (cuuint32_t)BQ, (cuuint32_t)G};
+    // Q viewed as (d, head, query): a box of G heads x BQ queries lands query-major, row = query * G + head
+    const cuuint64_t qd[3] = {(cuuint64_t)kD, (cuuint64_t)p.B * p.H, (cuuint64_t)p.N};
+    const cuuint64_t qs[2] = {(cuuint64_t)p.N * kD * 2, (cuuint64_t)kD * 2};
+    const cuuint32_t qb[3] = {64, (cuuint32_t)G, (cuuint32_t)BQ};
     const cuuint64_t kd[2] = {(cuuint64_t)kD, (cuuint64_t)p.B * p.Hkv * p.T};
     const cuuint64_t ks[1] = {(cuuint64_t)kD * 2};
     const cuuint32_t kb[2] = {64, (cuuint32_t)kChunk};
@@ -641,8 +657,8 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V,
                                           ctl.status, (unsigned long long)ctl.wait_limit, nwords,            \
                                           ctl.inject_stall);                                                 \
     }
-    if (cfg == 0) HILS_LAUNCH_TC(4)
-    else HILS_LAUNCH_TC(2)
+    if (cfg == 0) HILS_LAUNCH_TC(2)
+    else HILS_LAUNCH_TC(1)
 #undef HILS_LAUNCH_TC
     return cudaGetLastError();
 }

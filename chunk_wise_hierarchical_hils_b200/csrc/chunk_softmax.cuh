@@ -59,7 +59,7 @@ __device__ __forceinline__ void chunk_softmax_row(uint32_t (&sv)[64], int n_vis,
     }
     float l0, l1;
     f2_unpack(f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3])), l0, l1);
-    const uint64_t f = f2_splat(w / (l0 + l1));
+    const uint64_t f = f2_splat(__fdividef(w, l0 + l1));
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         float a0, a1;
