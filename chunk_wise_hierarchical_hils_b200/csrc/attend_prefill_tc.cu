@@ -17,21 +17,21 @@
 //                        chunks per ring slot (128-byte swizzle, no multicast);
 //   warp 1 (one thread)  TMA loads of the V tiles, two chunks per ring slot;
 //                        the warp also owns the TMEM allocation;
-//   warp 2 (one thread)  tcgen05.mma issue.  S = Q K^T (bf16, A and B from
-//                        shared memory) runs on two chunks at once (N = 128,
-//                        the tensor core's efficient width) into one of two
-//                        TMEM S buffers; O += P V (f16, P from TMEM, V from
-//                        shared memory) on the same pairs (K = 128 keys).  The
-//                        issuer polls which of the two is ready, key products
-//                        first, so the softmax warps never wait behind a value
-//                        product;
-//   warps 4..11          two groups of four warps, one thread per row; group
-//                        t % 2 handles chunk t: it reads S from TMEM (and frees
+//   warp 2 (one thread)  tcgen05.mma issue of S = Q K^T (bf16, A and B from
+//                        shared memory) on two chunks at once (N = 128, the
+//                        tensor core's efficient width) into one of two TMEM
+//                        S buffers;
+//   warp 3 (one thread)  tcgen05.mma issue of O += P V (f16, P from TMEM, V
+//                        from shared memory) on the same pairs (K = 128 keys);
+//                        two issuers keep the tensor core busy while either
+//                        one waits;
+//   warps 4..15          three groups of four warps, one thread per row; group
+//                        t % 3 handles chunk t: it reads S from TMEM (and frees
 //                        the S buffer at once), takes the softmax over the
 //                        chunk's visible keys, scales it by the row's fusion
 //                        weight (0 if the row's query did not select the chunk)
 //                        and writes P (f16) to its half of a TMEM P buffer.  At
-//                        the end both groups read O from TMEM and store it.
+//                        the end the groups read O from TMEM and store it.
 // Because each chunk's softmax is normalised on its own and the fusion weights
 // are known before the loop, P already carries w_c / l_c and the accumulator
 // needs no rescaling between chunks.  V is read as f16 (converted once per call
@@ -52,12 +52,12 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;     // 12 warps: K loads, V loads + TMEM, MMA issue, spare, 2 x 4 softmax
+constexpr int kGroups = 3;        // softmax warp groups (4 warps each); group t % kGroups handles chunk t
+constexpr int kThreads = 128 + 128 * kGroups;   // K loads, V loads + TMEM, QK issue, PV issue, softmax groups
 constexpr int kRows = 128;        // MMA M
 constexpr int kChunk = 64;        // C
 constexpr int kD = 128;           // d
 constexpr int kSP = 2;                // S buffers (a pair of chunks, 128 columns each) = key ring slots
-constexpr int kGroups = 2;            // softmax warp groups; group t % kGroups handles chunk t
 constexpr uint32_t kTmemCols = 512;   // S pair buffers (2 x 128 columns), O (128), up to 2 P pair buffers (64 each)
 constexpr uint32_t kColO = 256, kColP = 384;
 constexpr uint32_t kPairBytes = 32768;   // K and V ring slots: [c0 d0-63 | c1 d0-63 | c0 d64-127 | c1 d64-127]
@@ -103,7 +103,7 @@ __host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nword
 // uses s = p % NSV):
 //   K_LAND[b]    the pair's key tiles have landed (TMA transaction count)
 //   QK_READY[b]  S buffer b may take pair p: its key tiles are in (the key loader's arrival) and all
-//                eight softmax warps have read pair p - 2 out of it
+//                eight softmax warps of its two chunks have read pair p - 2 out of it
 //   QK_DONE[b]   the key product of pair p is complete: S is ready and the key slot is free
 //   V_LAND[s], PV_READY[s] (the value loader + the eight softmax warps that wrote P), PV_DONE[s] alike
 // so the MMA issuer tests one barrier per product and commits to one.
@@ -111,8 +111,8 @@ template <int NSV>
 struct Bars {
     static constexpr int Q_FULL = 0, K_LAND = 1, QK_READY = K_LAND + kSP, QK_DONE = QK_READY + kSP,
                          V_LAND = QK_DONE + kSP, PV_READY = V_LAND + NSV, PV_DONE = PV_READY + NSV,
-                         O_FULL = PV_DONE + NSV, MMA_DONE = O_FULL + 1;
-    static_assert(MMA_DONE < kMaxBars, "barrier slots");
+                         O_FULL = PV_DONE + NSV, MMA_DONE = O_FULL + 1;   // MMA_DONE + 0/1: the two issuers
+    static_assert(MMA_DONE + 1 < kMaxBars, "barrier slots");
 };
 
 __device__ __forceinline__ void store_row32(float *dst, const uint32_t *v)
@@ -248,17 +248,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(BAR(BR::Q_FULL), 1);
         for (int s = 0; s < kSP; ++s) {
             mbar_init(BAR(BR::K_LAND + s), 1);
-            mbar_init(BAR(BR::QK_READY + s), 1 + 4 * kGroups);
+            mbar_init(BAR(BR::QK_READY + s), 1 + 8);   // the key loader + 4 warps for each chunk of the pair
             mbar_init(BAR(BR::QK_DONE + s), 1);
-            for (int a = 0; a < 4 * kGroups; ++a) mbar_arrive(BAR(BR::QK_READY + s));   // pairs 0, 1: S free
+            for (int a = 0; a < 8; ++a) mbar_arrive(BAR(BR::QK_READY + s));   // pairs 0, 1: S free
         }
         for (int s = 0; s < NSV; ++s) {
             mbar_init(BAR(BR::V_LAND + s), 1);
-            mbar_init(BAR(BR::PV_READY + s), 1 + 4 * kGroups);
+            mbar_init(BAR(BR::PV_READY + s), 1 + 8);   // the value loader + 4 warps for each chunk
             mbar_init(BAR(BR::PV_DONE + s), 1);
         }
         mbar_init(BAR(BR::O_FULL), 1);
         mbar_init(BAR(BR::MMA_DONE), 1);
+        mbar_init(BAR(BR::MMA_DONE + 1), 1);
         fence_mbar_init();
         *abort_flag = 0;
         prefetch_tensormap(&tmQ);
@@ -415,84 +416,80 @@ __global__ void __launch_bounds__(kThreads, 1)
                          limit_ns, abort_flag, status);
         }
         __syncwarp();
-    } else if (warp == 2) {
-        // ---------------- MMA issue -------------------------------------------------------------
-        // The tensor core takes one MMA at a time from this thread (the issue returns about when the
-        // previous one is done), so the thread polls: the next key product whenever its keys are in and
-        // its S buffer has been read, else the next value product whenever its P and V are ready.
+    } else if (warp == 2 || warp == 3) {
+        // ---------------- MMA issue: warp 2 the key products, warp 3 the value products ---------
+        // The tensor core accepts one MMA at a time from a thread (the issue returns about when the
+        // previous one is done), so each issuer's waits and bookkeeping between products would
+        // leave it idle; with two issuers the other one's MMAs fill those gaps.
         if (lane == 0) {
+            const bool keys = (warp == 2);
+            const int n_pairs = (n_union + 1) >> 1;
             bool ok = true;
-            if (inject_stall) {
+            if (keys && inject_stall) {
                 // test control: wait once on a barrier nothing signals, so the bounded wait expires
                 ok = mbar_wait(BAR(BR::MMA_DONE), 0, limit_ns, abort_flag, status);
             }
-            ok = ok && mbar_wait(BAR(BR::Q_FULL), 0, limit_ns, abort_flag, status);
-            const int n_pairs = (n_union + 1) >> 1;
+            if (keys) ok = ok && mbar_wait(BAR(BR::Q_FULL), 0, limit_ns, abort_flag, status);
             // descriptors of Q's eight K-steps
             uint64_t dq[8];
 #pragma unroll
             for (int s = 0; s < 8; ++s) dq[s] = smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024);
-            int qp = 0, vp = 0;
-            unsigned idle = 0;
-            long long t_prog = cycle_now();
-            while (ok && vp < n_pairs) {
-                if (qp < n_pairs && mbar_test(BAR(BR::QK_READY + qp % kSP), (uint32_t)((qp / kSP) & 1))) {
-                    tc_fence_after();
-                    const uint32_t d_s = tmem + (uint32_t)(qp % kSP) * 128u;
-                    const uint64_t dk = smem_desc_sw128(sK + (uint32_t)(qp % kSP) * kPairBytes, 16, 1024);
-                    const uint32_t idesc = (2 * qp + 1 < n_union) ? IDESC_QK2 : IDESC_QK1;
+            for (int i = 0; ok && i < n_pairs; ++i) {
+                const uint32_t bar = keys ? BAR(BR::QK_READY + i % kSP) : BAR(BR::PV_READY + i % NSV);
+                const uint32_t phase = (uint32_t)((keys ? i / kSP : i / NSV) & 1);
+                // bounded poll (a test takes ~100 cycles, so the loop costs few issue slots); the grid's
+                // status word is read only now and then
+                const long long t0 = cycle_now();
+                unsigned idle = 0;
+                while (!mbar_test(bar, phase)) {
+                    if (*abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    if ((++idle & 63) == 0 && *reinterpret_cast<volatile unsigned int *>(status) != 0u) {
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                    if (past_limit(t0, limit_ns)) {
+                        *abort_flag = 1;
+                        atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!ok) break;
+                tc_fence_after();
+                if (keys) {
+                    const uint32_t d_s = tmem + (uint32_t)(i % kSP) * 128u;
+                    const uint64_t dk = smem_desc_sw128(sK + (uint32_t)(i % kSP) * kPairBytes, 16, 1024);
+                    const uint32_t idesc = (2 * i + 1 < n_union) ? IDESC_QK2 : IDESC_QK1;
 #pragma unroll
                     for (int s = 0; s < 8; ++s)
                         mma_bf16_ss(d_s, dq[s], dk + (uint64_t)(((s >> 2) * 16384u + (s & 3) * 32u) >> 4), idesc,
                                     s > 0 ? 1u : 0u);
-                    mma_commit(BAR(BR::QK_DONE + qp % kSP));
-                    ++qp;
-                    t_prog = cycle_now();
-                    continue;
-                }
-                const uint32_t pbar = BAR(BR::PV_READY + vp % NSV);
-                const uint32_t pphase = (uint32_t)((vp / NSV) & 1);
-                if (mbar_test(pbar, pphase)) {
-                    tc_fence_after();
-                    const uint32_t pa = tmem + kColP + (uint32_t)(vp % NSV) * 64u;
-                    const uint64_t dv = smem_desc_sw128(sV + (uint32_t)(vp % NSV) * kPairBytes, 16384, 1024);
-                    const int steps = (2 * vp + 1 < n_union) ? 8 : 4;
+                    mma_commit(BAR(BR::QK_DONE + i % kSP));
+                } else {
+                    const uint32_t pa = tmem + kColP + (uint32_t)(i % NSV) * 64u;
+                    const uint64_t dv = smem_desc_sw128(sV + (uint32_t)(i % NSV) * kPairBytes, 16384, 1024);
+                    const int steps = (2 * i + 1 < n_union) ? 8 : 4;
 #pragma unroll
                     for (int s = 0; s < 8; ++s)
                         if (s < steps)
                             mma_f16_ts(tmem + kColO, pa + 8u * s, dv + (uint64_t)((2048u * s) >> 4), IDESC_PV,
-                                       (vp > 0 || s > 0) ? 1u : 0u);
-                    mma_commit(BAR(BR::PV_DONE + vp % NSV));
-                    ++vp;
-                    t_prog = cycle_now();
-                    continue;
-                }
-                // nothing ready: poll again (a test takes ~100 cycles, so the loop costs few issue
-                // slots and reacts at once); the grid's status word is read only now and then
-                if (*abort_flag) {
-                    ok = false;
-                    break;
-                }
-                if ((++idle & 63) == 0 && *reinterpret_cast<volatile unsigned int *>(status) != 0u) {
-                    *abort_flag = 1;
-                    ok = false;
-                    break;
-                }
-                if (past_limit(t_prog, limit_ns)) {
-                    *abort_flag = 1;
-                    atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
-                    ok = false;
-                    break;
+                                       (i > 0 || s > 0) ? 1u : 0u);
+                    mma_commit(BAR(BR::PV_DONE + i % NSV));
                 }
             }
-            if (ok) mma_commit(BAR(BR::O_FULL));
-            // drain: every issued MMA completes before TMEM is released
-            mma_commit(BAR(BR::MMA_DONE));
-            mbar_drain(BAR(BR::MMA_DONE), 0, kDrainNs);
+            if (ok && !keys) mma_commit(BAR(BR::O_FULL));
+            // drain: every MMA this thread issued completes before TMEM is released
+            const uint32_t done = BAR(BR::MMA_DONE + (keys ? 0 : 1));
+            mma_commit(done);
+            mbar_drain(done, 0, kDrainNs);
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // ---------------- softmax (kGroups groups, alternate chunks) and epilogue ----
+        // ---------------- softmax (kGroups groups, chunks round-robin) and epilogue ----
         const int grp = (warp - 4) >> 2;
         const int qq = warp & 3;
         const int r = 32 * qq + lane, h = r % G, qi = r / G;
@@ -548,9 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && warp_wait(BAR(BR::O_FULL), 0, limit_ns, abort_flag, status)) {
             tc_fence_after();
             Tout *orow = O + ((((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi) * kD;
-#pragma unroll
-            for (int cg = 0; cg < 2; ++cg) {
-                const int col = grp * 64 + cg * 32;
+            for (int cb = grp; cb < kD / 32; cb += kGroups) {
+                const int col = cb * 32;
                 uint32_t v[32];
                 tmem_ld32(tmem + lane_off + kColO + (uint32_t)col, v);
                 tmem_wait_ld();
