@@ -14,8 +14,10 @@
 //   S[row, c] = q_{query, head} . L_c      (bf16 products, f32 accumulation)
 // into a double-buffered TMEM tile.  Four epilogue warps (one thread per row)
 // read S, form the group score mean_h(scale * S) with a butterfly over the G
-// lanes, and keep a per-row binary min-heap of the k best (group score, chunk)
-// keys; each row carries its own head's score as the heap payload, so the
+// lanes, and keep the k best (group score, chunk) keys of the row: for k <= 16
+// as a sorted list in registers, updated by a branch-free insertion network
+// (no memory latency on the insertion path), otherwise as a binary min-heap in
+// shared memory.  Each row carries its own head's score as the payload, so the
 // per-head slot scores come out of the same pass.  Ties go to the lower chunk
 // index through the key order.
 #include <cuda.h>
@@ -55,7 +57,7 @@ __host__ __device__ inline Layout make_layout(int k, int nsl)
     return L;
 }
 
-__device__ __noinline__ void sift_down_p(uint64_t *h, float *pl, int n, uint64_t x, float xp)
+__device__ __forceinline__ void sift_down_p(uint64_t *h, float *pl, int n, uint64_t x, float xp)
 {
     int e = 0;
     for (;;) {
@@ -73,16 +75,34 @@ __device__ __noinline__ void sift_down_p(uint64_t *h, float *pl, int n, uint64_t
     pl[e * kRows] = xp;
 }
 
-template <int G, int NSL>
+// Insert key x (payload xp) into the descending list a[0..RK) if it beats the last entry: every slot
+// takes its own, its upper neighbour's or the new entry's value from two comparisons, all at once.
+template <int RK>
+__device__ __forceinline__ void list_insert(uint64_t (&a)[RK], float (&ap)[RK], uint64_t x, float xp, bool on)
+{
+    bool gt[RK];
+#pragma unroll
+    for (int i = 0; i < RK; ++i) gt[i] = on && x > a[i];
+#pragma unroll
+    for (int i = RK - 1; i > 0; --i) {
+        a[i] = gt[i] ? (gt[i - 1] ? a[i - 1] : x) : a[i];
+        ap[i] = gt[i] ? (gt[i - 1] ? ap[i - 1] : xp) : ap[i];
+    }
+    a[0] = gt[0] ? x : a[0];
+    ap[0] = gt[0] ? xp : ap[0];
+}
+
+template <int G, int NSL, int RK>
 __global__ void __launch_bounds__(kThreads, 1)
     select_tc_kernel(const __grid_constant__ CUtensorMap tmL, Dims p, const __nv_bfloat16 *__restrict__ Q,
                      int32_t *__restrict__ sel_idx, float *__restrict__ sel_score, unsigned int *status,
                      unsigned long long limit_ns)
 {
     constexpr int BQ = kRows / G;
+    constexpr int RKN = RK > 0 ? RK : 1;   // register list length (unused when RK = 0)
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    const Layout Ly = make_layout(p.k, NSL);
+    const Layout Ly = make_layout(RK ? 0 : p.k, NSL);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q0 = blockIdx.x * BQ, g = blockIdx.y, b = blockIdx.z;
@@ -120,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(smem_addr(tmem_holder), kTmemCols);
         tmem_relinquish();
     }
-    for (int e = tid; e < p.k * kRows; e += kThreads) keys[e] = 0ull;
+    if (RK == 0)
+        for (int e = tid; e < p.k * kRows; e += kThreads) keys[e] = 0ull;
     // stage Q query-major in the 128-byte-swizzled K-major layout the MMA reads:
     // row r = query * G + head, two 64-column halves of 128 rows x 128 bytes
     for (int e = tid; e < kRows * 16; e += kThreads) {
@@ -190,6 +211,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t *hk = keys + r;
         float *hp = pay + r;
         float own = -INFINITY;
+        uint64_t top[RKN];
+        float topp[RKN];
+#pragma unroll
+        for (int i = 0; i < RKN; ++i) {
+            top[i] = 0ull;
+            topp[i] = 0.f;
+        }
         bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
             int w_ok = 1;
@@ -199,43 +227,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t sv[64];
-            tmem_ld32(trow + (uint32_t)(t & 1) * kTile, sv);
-            tmem_ld32(trow + (uint32_t)(t & 1) * kTile + 32u, sv + 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(S_FREE(t & 1));
             const int c0 = t * kTile;
 #pragma unroll
-            for (int j = 0; j < kTile; ++j) {
-                const float s = __uint_as_float(sv[j]);
-                float gs = s;
-#pragma unroll
-                for (int o = 1; o < G; o <<= 1) gs += __shfl_xor_sync(0xFFFFFFFFu, gs, o);
-                const int c = c0 + j;
-                if (valid && c < ci && p.k > 0) {
-                    const uint64_t key = make_key(gs * sc_g, c);
-                    if (key > hk[0]) sift_down_p(hk, hp, p.k, key, s * p.scale);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[32];
+                tmem_ld32(trow + (uint32_t)(t & 1) * kTile + 32u * half, sv);
+                tmem_wait_ld();
+                if (half == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(S_FREE(t & 1));
                 }
-                if (c == ci) own = s * p.scale;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float s = __uint_as_float(sv[j]);
+                    float gs = s;
+#pragma unroll
+                    for (int o = 1; o < G; o <<= 1) gs += __shfl_xor_sync(0xFFFFFFFFu, gs, o);
+                    const int c = c0 + 32 * half + j;
+                    const bool cand = valid && c < ci && p.k > 0;
+                    if (RK > 0) {
+                        const uint64_t key = make_key(gs * sc_g, c);
+                        const bool ins = cand && key > top[RKN - 1];
+                        if (__any_sync(0xFFFFFFFFu, ins)) list_insert<RKN>(top, topp, key, s * p.scale, ins);
+                    } else if (cand) {
+                        const uint64_t key = make_key(gs * sc_g, c);
+                        if (key > hk[0]) sift_down_p(hk, hp, p.k, key, s * p.scale);
+                    }
+                    if (c == ci) own = s * p.scale;
+                }
             }
         }
         if (ok && valid) {
-            // heap sort: slots 0..k-1 end in descending key order
-            for (int n = p.k; n > 1; --n) {
-                const uint64_t top = hk[0];
-                const float topp = hp[0];
-                sift_down_p(hk, hp, n - 1, hk[(n - 1) * kRows], hp[(n - 1) * kRows]);
-                hk[(n - 1) * kRows] = top;
-                hp[(n - 1) * kRows] = topp;
-            }
             const size_t row_g = (((size_t)b * p.Hkv + g) * p.N) + q0 + qi;
             const size_t row_h = (((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi;
             const int ns = p.k + 1;
-            if (h == 0)
-                for (int j = 0; j < p.k; ++j) sel_idx[row_g * p.k + j] = key_index(hk[j * kRows]);
-            for (int j = 0; j < p.k; ++j) sel_score[row_h * ns + j] = hk[j * kRows] ? hp[j * kRows] : -INFINITY;
+            if (RK > 0) {
+                // the list is already in descending key order
+#pragma unroll
+                for (int j = 0; j < RKN; ++j) {
+                    if (j < p.k) {
+                        if (h == 0) sel_idx[row_g * p.k + j] = key_index(top[j]);
+                        sel_score[row_h * ns + j] = top[j] ? topp[j] : -INFINITY;
+                    }
+                }
+            } else {
+                // heap sort: slots 0..k-1 end in descending key order
+                for (int n = p.k; n > 1; --n) {
+                    const uint64_t top0 = hk[0];
+                    const float topp0 = hp[0];
+                    sift_down_p(hk, hp, n - 1, hk[(n - 1) * kRows], hp[(n - 1) * kRows]);
+                    hk[(n - 1) * kRows] = top0;
+                    hp[(n - 1) * kRows] = topp0;
+                }
+                if (h == 0)
+                    for (int j = 0; j < p.k; ++j) sel_idx[row_g * p.k + j] = key_index(hk[j * kRows]);
+                for (int j = 0; j < p.k; ++j) sel_score[row_h * ns + j] = hk[j * kRows] ? hp[j * kRows] : -INFINITY;
+            }
             sel_score[row_h * ns + p.k] = own;
         }
         (void)own_s;
@@ -284,22 +332,22 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *L, int32_t *sel_i
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const int nsl = stages_for(p.k);
-    const size_t smem = make_layout(p.k, nsl).total + 1024;
+    const int rk = p.k <= 16 ? 16 : 0;   // register list for k <= 16, shared-memory heap above
+    const size_t smem = make_layout(rk ? 0 : p.k, nsl).total + 1024;
     dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
     cudaError_t e;
-    if (nsl == 2) {
-        auto kern = select_tc_kernel<G, 2>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kThreads, smem, s>>>(tl, p, static_cast<const __nv_bfloat16 *>(Q), sel_idx, sel_score,
-                                          ctl.status, (unsigned long long)ctl.wait_limit);
-    } else {
-        auto kern = select_tc_kernel<G, 4>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kThreads, smem, s>>>(tl, p, static_cast<const __nv_bfloat16 *>(Q), sel_idx, sel_score,
-                                          ctl.status, (unsigned long long)ctl.wait_limit);
+#define HILS_LAUNCH_SEL(NS, RKV)                                                                             \
+    {                                                                                                        \
+        auto kern = select_tc_kernel<G, NS, RKV>;                                                            \
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);              \
+        if (e != cudaSuccess) return e;                                                                      \
+        kern<<<grid, kThreads, smem, s>>>(tl, p, static_cast<const __nv_bfloat16 *>(Q), sel_idx, sel_score,  \
+                                          ctl.status, (unsigned long long)ctl.wait_limit);                   \
     }
+    if (rk) HILS_LAUNCH_SEL(2, 16)
+    else if (nsl == 2) HILS_LAUNCH_SEL(2, 0)
+    else HILS_LAUNCH_SEL(4, 0)
+#undef HILS_LAUNCH_SEL
     return cudaGetLastError();
 }
 
