@@ -17,7 +17,10 @@
 // lanes, and keep the k best (group score, chunk) keys of the row: for k <= 16
 // as a sorted list in registers, updated by a branch-free insertion network
 // (no memory latency on the insertion path), otherwise as a binary min-heap in
-// shared memory.  Each row carries its own head's score as the payload, so the
+// shared memory.  With the register list, a candidate that beats the row's
+// current k-th key is first queued in shared memory; the warp then inserts the
+// queued keys together, so it runs the network as often as its busiest row
+// needs rather than whenever any row has a candidate.  Each row carries its own head's score as the payload, so the
 // per-head slot scores come out of the same pass.  Ties go to the lower chunk
 // index through the key order.
 #include <cuda.h>
@@ -38,6 +41,7 @@ constexpr uint32_t kTileBytes = kTile * kD * 2;
 constexpr uint32_t kTmemCols = 128;       // two 64-column score buffers
 constexpr unsigned long long kDrainNs = 2000000000ull;
 constexpr uint32_t IDESC = idesc_bf16_f32(128, kTile, false, false);
+constexpr int kQueue = 16;                // register-list path: candidates queued per row between insertions
 
 struct Layout {
     uint32_t q, l, bar, misc, keys, pay, own, total;
@@ -102,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int RKN = RK > 0 ? RK : 1;   // register list length (unused when RK = 0)
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    const Layout Ly = make_layout(RK ? 0 : p.k, NSL);
+    const Layout Ly = make_layout(RK ? kQueue : p.k, NSL);   // register list: a kQueue-deep queue per row
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q0 = blockIdx.x * BQ, g = blockIdx.y, b = blockIdx.z;
@@ -238,8 +242,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(S_FREE(t & 1));
                 }
+                int qn = 0;   // queued candidates of this row (register-list path)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
+                    if (RK > 0 && j == kQueue) {
+                        // the queue is full after kQueue candidates: insert them before going on
+                        const int m = __reduce_max_sync(0xFFFFFFFFu, qn);
+                        for (int i = 0; i < m; ++i) {
+                            const bool on = i < qn;
+                            list_insert<RKN>(top, topp, on ? hk[i * kRows] : 0ull, on ? hp[i * kRows] : 0.f, on);
+                        }
+                        qn = 0;
+                    }
                     const float s = __uint_as_float(sv[j]);
                     float gs = s;
 #pragma unroll
@@ -248,13 +262,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool cand = valid && c < ci && p.k > 0;
                     if (RK > 0) {
                         const uint64_t key = make_key(gs * sc_g, c);
-                        const bool ins = cand && key > top[RKN - 1];
-                        if (__any_sync(0xFFFFFFFFu, ins)) list_insert<RKN>(top, topp, key, s * p.scale, ins);
+                        if (cand && key > top[RKN - 1]) {
+                            hk[qn * kRows] = key;
+                            hp[qn * kRows] = s * p.scale;
+                            ++qn;
+                        }
                     } else if (cand) {
                         const uint64_t key = make_key(gs * sc_g, c);
                         if (key > hk[0]) sift_down_p(hk, hp, p.k, key, s * p.scale);
                     }
                     if (c == ci) own = s * p.scale;
+                }
+                if (RK > 0) {
+                    // insert the queued keys: as many network passes as the warp's longest queue (the loop
+                    // above inserted and emptied the queue after its first kQueue candidates)
+                    const int m = __reduce_max_sync(0xFFFFFFFFu, qn);
+                    for (int i = 0; i < m; ++i) {
+                        const bool on = i < qn;
+                        list_insert<RKN>(top, topp, on ? hk[i * kRows] : 0ull, on ? hp[i * kRows] : 0.f, on);
+                    }
                 }
             }
         }
@@ -333,7 +359,7 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *L, int32_t *sel_i
         return cudaErrorInvalidValue;
     const int nsl = stages_for(p.k);
     const int rk = p.k <= 16 ? 16 : 0;   // register list for k <= 16, shared-memory heap above
-    const size_t smem = make_layout(rk ? 0 : p.k, nsl).total + 1024;
+    const size_t smem = make_layout(rk ? kQueue : p.k, nsl).total + 1024;
     dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
     cudaError_t e;
 #define HILS_LAUNCH_SEL(NS, RKV)                                                                             \
