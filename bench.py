@@ -79,19 +79,21 @@ def kernels_per_step(w):
     return 3 if (tc and w.C == 64) else 2   # selection; [V to f16 +] attention
 
 
-def kernel_traffic(kernel_file, workload):
+def kernel_traffic(kernel, workload):
     """DRAM bytes per launch from an ncu capture committed in profiles/traffic.json, or None.
 
-    The entry is used only while the kernel's source file is unchanged since the capture
-    (its SHA-256 is stored with the numbers) and for the same workload."""
+    The entry names the source files the kernel is built from with their SHA-256 at the time of the
+    capture; it is used only while every one of them is unchanged, and for the same workload."""
     import hashlib
     try:
-        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel_file]
-        src = os.path.join(ROOT, "chunk_wise_hierarchical_hils_b200", "csrc", kernel_file)
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
+        csrc = os.path.join(ROOT, "chunk_wise_hierarchical_hils_b200", "csrc")
+        for f, sha in rec["sources"].items():
+            if hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest() != sha:
+                return None
     except Exception:
         return None
-    if rec.get("source_sha256") != sha or rec.get("workload") != workload:
+    if rec.get("workload") != workload:
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -404,20 +406,28 @@ def run_hils(args, w):
         achieved = fl / (k2_avg * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": "chunk_attend_fuse (prefill)", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": kernel_traffic("attend_prefill_tc.cu", w.name),
+                "traffic": kernel_traffic("attend_prefill_tc", w.name),
                 "peak_kind": pk_kind + " bf16 sustained", "algorithmic_flops_per_launch": fl,
                 "launch_ms": k2_avg, "select_ms": k1_avg}
     else:
         unit = "GB/s"
         per_step_units = decode_bytes(w) / 1e9
         lb = landmark_bytes(w)
-        achieved = lb / (k1_avg * 1e-3) / 1e9
+        kvb = decode_bytes(w) - lb
         peak = pk["hbm_gbs"]
-        roof = {"bound": "hbm", "kernel": "score_select (decode landmark scan)", "achieved": achieved,
-                "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": kernel_traffic("select_decode.cu", w.name),
-                "peak_kind": pk_kind + " copy", "algorithmic_bytes_per_launch": lb, "launch_ms": k1_avg,
-                "attend_ms": k2_avg}
+        if k2_avg >= k1_avg:   # the dominant kernel: chunk attention (selected K/V) or the landmark scan
+            achieved = kvb / (k2_avg * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": "chunk_attend_fuse (decode)", "achieved": achieved, "peak": peak,
+                    "unit": "GB/s", "frac": achieved / peak, "traffic": kernel_traffic("attend_decode", w.name),
+                    "peak_kind": pk_kind + " copy", "algorithmic_bytes_per_launch": kvb, "launch_ms": k2_avg,
+                    "select_ms": k1_avg}
+        else:
+            achieved = lb / (k1_avg * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": "score_select (decode landmark scan)", "achieved": achieved,
+                    "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": kernel_traffic("select_decode", w.name),
+                    "peak_kind": pk_kind + " copy", "algorithmic_bytes_per_launch": lb, "launch_ms": k1_avg,
+                    "attend_ms": k2_avg}
     units_all = ws * per_step_units
     if args.scaling == "strong" and ws > 1:
         units_all = per_step_units * full_B / w.B   # ranks hold slices of one batch (equal slices assumed)
