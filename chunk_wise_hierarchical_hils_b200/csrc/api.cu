@@ -85,6 +85,13 @@ bool force_cuda_cores()
     return force && strcmp(force, "simt") == 0;
 }
 
+// Test control: HILS_DECODE_KERNEL=simt keeps decode attention on the CUDA-core kernel.
+bool force_decode_cuda_cores()
+{
+    const char *force = getenv("HILS_DECODE_KERNEL");
+    return force && strcmp(force, "simt") == 0;
+}
+
 hils_status check_ws(void *ws, size_t have, size_t need)
 {
     if (need == 0) return HILS_OK;
@@ -112,7 +119,11 @@ hils_status do_attend(const Dims &p, hils_dtype in, hils_dtype out, const void *
     DeviceCtl ctl;
     hils_status st = device_ctl(&ctl);
     if (st != HILS_OK) return st;
-    if (p.N == 1) return from_cuda(launch_attend_decode(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
+    if (p.N == 1) {
+        if (!force_decode_cuda_cores() && attend_decode_mma_supported(p, in))
+            return from_cuda(launch_attend_decode_mma(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
+        return from_cuda(launch_attend_decode(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
+    }
     return from_cuda(launch_attend_prefill(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
 }
 

@@ -146,10 +146,12 @@ cudaError_t launch_d(const Dims &p, const void *Q, const void *K, const void *V,
 
 }  // namespace
 
+// Partial sums (one entry per chunk slot: the tensor-core kernel keeps one per warp, the CUDA-core
+// kernel uses the first nsplit2 of them) and the (b, g) tickets.
 size_t decode_attend_ws_bytes(const Dims &p)
 {
     const DecodePlan plan = decode_plan(p);
-    return align_up((size_t)p.B * p.Hkv * plan.nsplit2 * p.G * p.d * sizeof(float), 256) +
+    return align_up((size_t)p.B * p.Hkv * plan.nsplit2 * plan.slots_per_cta * p.G * p.d * sizeof(float), 256) +
            align_up((size_t)p.B * p.Hkv * sizeof(unsigned int), 256);
 }
 

@@ -1,0 +1,333 @@
+// attend_decode_mma.cu -- split-K chunk attention and fusion for single-token decode on the tensor
+// cores (bf16 in, d = 128, C in {64, 128}, G <= 16).
+//
+// "Hierarchical Sparse Attention Done Right" (arXiv 2607.02980v1): Sec. 7 Analysis (per-token
+// decode touches a fixed budget of k+1 chunks); Abstract and Sec. 3 "Hierarchical softmax"
+// (softmax inside each chunk, chunks fused by a softmax over the retrieval scores); Sec. 4
+// "Architecture" (a GQA group's heads share the retrieved chunks).
+//
+// Decode moves k+1 chunks of keys and values per (b, g) and does little arithmetic on them, so the
+// kernel's job is to keep the copies streaming: the arithmetic must not hold a CTA's shared memory
+// longer than the copy of its next chunk takes.  The (b, g)'s k+1 chunks are split over CTAs of
+// SLOTS chunks each (the split plan of the decode selection); thread 0 of a CTA starts TMA tile
+// copies (128-byte swizzle, no multicast) of all its chunks at once, and one warp per chunk then
+// computes, with mma.sync m16n8k16 tiles whose 16 rows are the group's G query heads (zero
+// padded):
+//   S = Q K_c^T   (bf16 x bf16 -> f32),
+//   P = w_c * softmax(scale * S) over the visible keys, per row,
+//   O_part += P V_c   (P split into a bf16 high part and a bf16 remainder, so P keeps ~16 bits),
+// reading K and V with ldmatrix (transposed for V) from the swizzled tiles.  Each chunk's softmax
+// is normalised on its own and the fusion weights follow from the slot scores alone, so the
+// warps' partial outputs combine by plain addition: every warp writes its rows to the workspace
+// and the last CTA of the (b, g) (atomic ticket) adds them in slot order.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "attend_simt.cuh"
+#include "sm100.cuh"
+
+namespace hils {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kQPitch = 272;   // bytes per staged Q row (256 + 16: ldmatrix rows on distinct banks)
+constexpr unsigned long long kDrainNs = 2000000000ull;
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D (16x8 f32) += A (16x16 bf16, row-major fragment) * B (16x8 bf16, column-major fragment)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// A tile written by TMA with the 128-byte swizzle: rows of 128 bytes, the 16-byte piece j of row r
+// stored at piece j ^ (r % 8).
+__device__ __forceinline__ uint32_t sw128(uint32_t tile, int r, int j)
+{
+    return tile + (uint32_t)r * 128u + ((uint32_t)(j ^ (r & 7)) << 4);
+}
+
+template <typename Tout, int C, int SLOTS>
+__global__ void __launch_bounds__(32 * SLOTS, 1)
+    attend_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Dims p,
+                             DecodePlan plan, const __nv_bfloat16 *__restrict__ Q, const int32_t *__restrict__ sel_idx,
+                             const float *__restrict__ sel_score, float *__restrict__ partial,
+                             unsigned int *__restrict__ tickets, Tout *__restrict__ O, unsigned int *status,
+                             unsigned long long limit_ns)
+{
+    constexpr uint32_t HALF = C * 128;      // one 64-column half of a C-row tile
+    constexpr uint32_t SLOT = 4 * HALF;     // K halves, then V halves
+    constexpr int NT = C / 8;               // key tiles of 8
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    unsigned char *qs = base + SLOTS * SLOT;                                  // [16][kQPitch]
+    float *wsm = reinterpret_cast<float *>(qs + 16 * kQPitch);               // [16][SLOTS]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(wsm + 16 * SLOTS);          // [SLOTS]
+    __shared__ int s_chunk[SLOTS];
+    __shared__ int s_last;
+    __shared__ int s_abort;
+
+    const int split = blockIdx.x, bg = blockIdx.y, b = bg / p.Hkv, g = bg % p.Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.G;
+    const long long pos = p.q_offset;   // N == 1
+    const int ci = (int)(pos / C);
+    const int ns = p.k + 1;
+    const int j0 = split * SLOTS, j1 = min(j0 + SLOTS, ns);
+    const uint32_t slot0 = smem_addr(base);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int i = 0; i < SLOTS; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        fence_mbar_init();
+        for (int i = 0; i < SLOTS; ++i) {
+            const int j = j0 + i;
+            const int c = (j >= j1) ? -1 : (j < p.k) ? sel_idx[(size_t)bg * p.k + j] : ci;
+            s_chunk[i] = c;
+            if (c < 0) continue;
+            const int row = bg * p.T + c * C;
+            const uint32_t dst = slot0 + (uint32_t)i * SLOT, bar = smem_addr(&bars[i]);
+            mbar_arrive_expect_tx(bar, SLOT);
+            tma_load_2d(dst, &tmK, bar, 0, row);
+            tma_load_2d(dst + HALF, &tmK, bar, 64, row);
+            tma_load_2d(dst + 2 * HALF, &tmV, bar, 0, row);
+            tma_load_2d(dst + 3 * HALF, &tmV, bar, 64, row);
+        }
+    }
+    // the group's query rows, bf16, rows G..15 zero
+    for (int e = threadIdx.x; e < 16 * 16; e += 32 * SLOTS) {
+        const int r = e >> 4, seg = e & 15;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < G) v = __ldg(reinterpret_cast<const uint4 *>(Q + ((size_t)b * p.H + (size_t)g * G + r) * kD) + seg);
+        *reinterpret_cast<uint4 *>(qs + r * kQPitch + seg * 16) = v;
+    }
+    for (int h = warp; h < G; h += SLOTS)
+        warp_fusion_weights(sel_score + ((size_t)b * p.H + (size_t)g * G + h) * ns, ns, j0, j1, wsm + h * SLOTS);
+    __syncthreads();
+
+    const int gid = lane >> 2, tig = lane & 3;   // fragment row group and thread in group
+    float oacc[16][4];
+#pragma unroll
+    for (int nd = 0; nd < 16; ++nd)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[nd][e] = 0.f;
+
+    const int c = s_chunk[warp];
+    bool ok = true;
+    if (c >= 0) {
+        int w_ok = 1;
+        if (lane == 0) w_ok = mbar_wait(smem_addr(&bars[warp]), 0, limit_ns, &s_abort, status) ? 1 : 0;
+        ok = __shfl_sync(0xFFFFFFFFu, w_ok, 0) != 0;
+    }
+    if (c >= 0 && ok) {
+        const uint32_t kt = slot0 + (uint32_t)warp * SLOT, vt = kt + 2 * HALF;
+        const int n_vis = (int)min((long long)C, pos - (long long)c * C + 1);
+        const int mi = lane >> 3, rr = lane & 7;   // ldmatrix: the matrix and row this lane addresses
+
+        // S = Q K^T: 16 rows x C keys
+        float sacc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+        for (int ks2 = 0; ks2 < 4; ++ks2) {
+            // Q fragments of k-steps 2 ks2 and 2 ks2 + 1 (d = 32 ks2 .. 32 ks2 + 31)
+            uint32_t qa[2][4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int ks = 2 * ks2 + h2;
+                const uint32_t qaddr =
+                    smem_addr(qs) + (uint32_t)((rr + 8 * (mi & 1)) * kQPitch + (ks * 16 + 8 * (mi >> 1)) * 2);
+                ldsm_x4(qaddr, qa[h2][0], qa[h2][1], qa[h2][2], qa[h2][3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int key = nt * 8 + rr, dc = 4 * ks2 + mi;   // 16-byte piece of d
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(sw128(kt + (uint32_t)(dc >> 3) * HALF, key, dc & 7), b0, b1, b2, b3);
+                mma16816(sacc[nt], qa[0], b0, b1);
+                mma16816(sacc[nt], qa[1], b2, b3);
+            }
+        }
+
+        // softmax per row (rows gid and gid + 8), scaled by the row's fusion weight
+        const float sl2 = p.scale * 1.4426950408889634f;
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int key = nt * 8 + tig * 2 + e;
+                if (key >= n_vis) {
+                    sacc[nt][e] = -INFINITY;
+                    sacc[nt][2 + e] = -INFINITY;
+                }
+                m0 = fmaxf(m0, sacc[nt][e]);
+                m1 = fmaxf(m1, sacc[nt][2 + e]);
+            }
+        m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, 1));
+        m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, 2));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, 1));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, 2));
+        float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                sacc[nt][e] = exp2f((sacc[nt][e] - m0) * sl2);
+                sacc[nt][2 + e] = exp2f((sacc[nt][2 + e] - m1) * sl2);
+                l0 += sacc[nt][e];
+                l1 += sacc[nt][2 + e];
+            }
+        l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 1);
+        l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 2);
+        l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 1);
+        l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 2);
+        const float f0 = (gid < G) ? wsm[gid * SLOTS + warp] / l0 : 0.f;
+        const float f1 = (gid + 8 < G) ? wsm[(gid + 8) * SLOTS + warp] / l1 : 0.f;
+
+        // O += P V over the chunk's keys, 16 per k-step; P = high + remainder, both bf16
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+            float pv[8];
+            pv[0] = sacc[2 * kk][0] * f0;
+            pv[1] = sacc[2 * kk][1] * f0;
+            pv[2] = sacc[2 * kk][2] * f1;
+            pv[3] = sacc[2 * kk][3] * f1;
+            pv[4] = sacc[2 * kk + 1][0] * f0;
+            pv[5] = sacc[2 * kk + 1][1] * f0;
+            pv[6] = sacc[2 * kk + 1][2] * f1;
+            pv[7] = sacc[2 * kk + 1][3] * f1;
+            uint32_t ph[4], pl[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                ph[q] = pack_bf16(pv[2 * q], pv[2 * q + 1]);
+                const __nv_bfloat162 hv = *reinterpret_cast<const __nv_bfloat162 *>(&ph[q]);
+                pl[q] = pack_bf16(pv[2 * q] - __low2float(hv), pv[2 * q + 1] - __high2float(hv));
+            }
+#pragma unroll
+            for (int nd2 = 0; nd2 < 8; ++nd2) {
+                const int key = kk * 16 + rr + 8 * (mi & 1), dc = 2 * nd2 + (mi >> 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(sw128(vt + (uint32_t)(dc >> 3) * HALF, key, dc & 7), b0, b1, b2, b3);
+                mma16816(oacc[2 * nd2], ph, b0, b1);
+                mma16816(oacc[2 * nd2], pl, b0, b1);
+                mma16816(oacc[2 * nd2 + 1], ph, b2, b3);
+                mma16816(oacc[2 * nd2 + 1], pl, b2, b3);
+            }
+        }
+    }
+
+    // every warp writes its entry (zeros for an empty slot) so that the merge can add them all
+    const int n_entries = plan.nsplit2 * SLOTS;
+    float *mine = partial + ((size_t)bg * n_entries + (size_t)split * SLOTS + warp) * G * kD;
+#pragma unroll
+    for (int nd = 0; nd < 16; ++nd) {
+        const int col = nd * 8 + tig * 2;
+        if (gid < G) *reinterpret_cast<float2 *>(mine + gid * kD + col) = make_float2(oacc[nd][0], oacc[nd][1]);
+        if (gid + 8 < G)
+            *reinterpret_cast<float2 *>(mine + (gid + 8) * kD + col) = make_float2(oacc[nd][2], oacc[nd][3]);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && s_abort) {
+        // the copies must land before the CTA exits
+        for (int i = 0; i < SLOTS; ++i)
+            if (s_chunk[i] >= 0) mbar_drain(smem_addr(&bars[i]), 0, kDrainNs);
+    }
+
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(&tickets[bg], 1u) == (unsigned)(plan.nsplit2 - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const float *all = partial + (size_t)bg * n_entries * G * kD;
+    for (int e = threadIdx.x; e < G * kD; e += 32 * SLOTS) {
+        float a = 0.f;
+        for (int en = 0; en < n_entries; ++en) a += __ldcg(all + (size_t)en * G * kD + e);
+        const int h = e / kD, x = e % kD;
+        store_out(O + ((size_t)b * p.H + (size_t)g * G + h) * kD + x, a);
+    }
+}
+
+template <typename Tout, int C, int SLOTS>
+cudaError_t launch_cs(const Dims &p, const DecodePlan &plan, const CUtensorMap &tk, const CUtensorMap &tv,
+                      const void *Q, const int32_t *sel_idx, const float *sel_score, float *partial,
+                      unsigned int *tickets, void *O, const DeviceCtl &ctl, cudaStream_t s)
+{
+    const size_t smem = 1024 + (size_t)SLOTS * 4 * C * 128 + 16 * kQPitch + 16 * SLOTS * 4 + SLOTS * 8;
+    auto kern = attend_decode_mma_kernel<Tout, C, SLOTS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(plan.nsplit2, p.B * p.Hkv);
+    kern<<<grid, 32 * SLOTS, smem, s>>>(tk, tv, p, plan, static_cast<const __nv_bfloat16 *>(Q), sel_idx, sel_score,
+                                        partial, tickets, static_cast<Tout *>(O), ctl.status,
+                                        (unsigned long long)ctl.wait_limit);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attend_decode_mma_supported(const Dims &p, hils_dtype in)
+{
+    if (in != HILS_BF16 || p.d != kD || p.N != 1 || p.G > 16) return false;
+    const DecodePlan plan = decode_plan(p);
+    return (p.C == 64 && plan.slots_per_cta == 2) || (p.C == 128 && plan.slots_per_cta == 1);
+}
+
+cudaError_t launch_attend_decode_mma(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
+                                     const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
+                                     const DeviceCtl &ctl, cudaStream_t s)
+{
+    const DecodePlan plan = decode_plan(p);
+    float *partial = static_cast<float *>(ws);
+    unsigned int *tickets = reinterpret_cast<unsigned int *>(
+        static_cast<char *>(ws) +
+        align_up((size_t)p.B * p.Hkv * plan.nsplit2 * plan.slots_per_cta * p.G * kD * sizeof(float), 256));
+    cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)p.B * p.Hkv * sizeof(unsigned int), s);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tk, tv;
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)p.B * p.Hkv * p.T};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)p.C};
+    if (!encode_tensor_map_sw128(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, 2, dims, strides, box) ||
+        !encode_tensor_map_sw128(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, 2, dims, strides, box))
+        return cudaErrorInvalidValue;
+    if (p.C == 64)
+        return out == HILS_F32
+                   ? launch_cs<float, 64, 2>(p, plan, tk, tv, Q, sel_idx, sel_score, partial, tickets, O, ctl, s)
+                   : launch_cs<__nv_bfloat16, 64, 2>(p, plan, tk, tv, Q, sel_idx, sel_score, partial, tickets, O,
+                                                     ctl, s);
+    return out == HILS_F32
+               ? launch_cs<float, 128, 1>(p, plan, tk, tv, Q, sel_idx, sel_score, partial, tickets, O, ctl, s)
+               : launch_cs<__nv_bfloat16, 128, 1>(p, plan, tk, tv, Q, sel_idx, sel_score, partial, tickets, O, ctl,
+                                                  s);
+}
+
+}  // namespace hils

@@ -1,6 +1,7 @@
 // internal.h -- resolved problem description and kernel launchers (not part of the ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -64,6 +65,17 @@ cudaError_t launch_attend_decode(const Dims &p, hils_dtype in, hils_dtype out, c
                                  const void *K, const void *V, const int32_t *sel_idx,
                                  const float *sel_score, void *O, void *ws, const DeviceCtl &ctl,
                                  cudaStream_t s);
+
+// Single-token decode attention on the tensor cores (mma.sync tiles): bf16, d = 128, C in {64, 128}.
+bool attend_decode_mma_supported(const Dims &p, hils_dtype in);
+cudaError_t launch_attend_decode_mma(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
+                                     const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
+                                     const DeviceCtl &ctl, cudaStream_t s);
+
+// TMA tile map (no interleave, 128-byte swizzle, 256-byte L2 promotion, zero fill out of bounds); rank 1..3,
+// strides in bytes for dimensions 1..rank-1.  False when the driver's encoder is missing or rejects the map.
+bool encode_tensor_map_sw128(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, int rank,
+                             const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box);
 
 // Device status word and wait limit of the current device (looked up once per device).
 hils_status device_ctl(DeviceCtl *ctl);

@@ -46,6 +46,8 @@ DECODE = [
        l_mode="iid"),
     wl("decode_k64_c128", B=1, H=16, Hkv=4, N=1, T=128 * 700, q_offset=128 * 700 - 1, C=128, k=64, seed=125,
        l_mode="iid"),
+    wl("decode_g16_partial_chunk", B=2, H=16, Hkv=1, N=1, T=3000, q_offset=2999, k=8, seed=126),
+    wl("decode_g1_c128", B=3, H=4, Hkv=4, N=1, T=128 * 40 + 77, q_offset=128 * 40 + 76, C=128, k=5, seed=127),
 ]
 
 
@@ -68,7 +70,15 @@ def test_cuda_core_kernel_too(w, monkeypatch):
     _check(st)
 
 
-@pytest.mark.parametrize("w", [CASES[1], DECODE[0]], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [DECODE[0], DECODE[2], DECODE[4], DECODE[5]], ids=lambda w: w.name)
+def test_cuda_core_decode_too(w, monkeypatch):
+    """The CUDA-core decode attention kernel, forced, on shapes the tensor-core tile kernel normally takes."""
+    monkeypatch.setenv("HILS_DECODE_KERNEL", "simt")
+    st, _ = parity.run_small(w)
+    _check(st)
+
+
+@pytest.mark.parametrize("w", [CASES[1], DECODE[0], DECODE[5]], ids=lambda w: w.name)
 def test_bf16_output(w):
     st, _ = parity.run_small(w, out_dtype="bf16")
     _check(st)
