@@ -342,26 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j == p.k) qcnt[qi] = rank + 1;   // the own chunk is the largest
         }
     }
-    __syncthreads();
-
-    if (tid < kRows) {
-        // fusion weights of each row, in the order of its query's chunk list
-        const int r = tid, qi = r / G;
-        if (qi < nq) {
-            const float *sc = scbuf + r * ns;
-            float M = -INFINITY;
-            for (int j = 0; j < ns; ++j) M = fmaxf(M, sc[j]);
-            float Z = 0.f;
-            for (int j = 0; j < ns; ++j) Z += (sc[j] == -INFINITY) ? 0.f : __expf(sc[j] - M);
-            const float iz = 1.0f / Z;
-            const int *slt = qslot + qi * ns;
-            const int cnt = qcnt[qi];
-            for (int pos = 0; pos < cnt; ++pos) {
-                const float sj = sc[slt[pos]];
-                wts[r * ns + pos] = (sj == -INFINITY) ? 0.f : __expf(sj - M) * iz;
-            }
-        }
-    }
+    // the union and the chunk lists are complete: the loaders start now, while the first softmax
+    // warps compute the fusion weights
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -490,6 +472,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp >= 4) {
         // ---------------- softmax (kGroups groups, chunks round-robin) and epilogue ----
+        if (warp < 8) {
+            // fusion weights of each row, in the order of its query's chunk list (warps 4..7)
+            const int r = tid - 128, qi = r / G;
+            if (qi < nq) {
+                const float *sc = scbuf + r * ns;
+                float M = -INFINITY;
+                for (int j = 0; j < ns; ++j) M = fmaxf(M, sc[j]);
+                float Z = 0.f;
+                for (int j = 0; j < ns; ++j) Z += (sc[j] == -INFINITY) ? 0.f : __expf(sc[j] - M);
+                const float iz = 1.0f / Z;
+                const int *slt = qslot + qi * ns;
+                const int cnt = qcnt[qi];
+                for (int pos = 0; pos < cnt; ++pos) {
+                    const float sj = sc[slt[pos]];
+                    wts[r * ns + pos] = (sj == -INFINITY) ? 0.f : __expf(sj - M) * iz;
+                }
+            }
+        }
+        // the softmax warps wait for the weights (named barrier 1: warps 4..15 only)
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * 4 * kGroups) : "memory");
         const int grp = (warp - 4) >> 2;
         const int qq = warp & 3;
         const int r = 32 * qq + lane, h = r % G, qi = r / G;
