@@ -48,6 +48,11 @@
  * failures of bounded waits are reported by hils_sync_status().
  * Thread safety: calls may come from several host threads; kernels that share
  * one workspace must not overlap on the GPU.
+ * Kernel choice: the tensor-core kernels run whenever they cover the problem
+ * (bf16 inputs, d = 128; prefill C = 64; decode C in {64, 128}), the CUDA-core
+ * kernels otherwise.  As a test control, the environment variables
+ * HILS_PREFILL_KERNEL=simt and HILS_DECODE_KERNEL=simt force the CUDA-core
+ * prefill and decode-attention kernels; results agree within the parity bounds.
  */
 #ifndef HILS_H
 #define HILS_H
