@@ -108,8 +108,16 @@ __global__ void attend_decode_kernel(Dims p, DecodePlan plan, const Tin *__restr
     const float *base = partial + ((size_t)bg * plan.nsplit2 * p.G + warp) * D;
 #pragma unroll
     for (int x = 0; x < D / 32; ++x) {
+        // splits added in order, eight loads in flight at a time
         float a = 0.f;
-        for (int sp = 0; sp < plan.nsplit2; ++sp) a += __ldcg(base + (size_t)sp * p.G * D + lane + 32 * x);
+        for (int sp0 = 0; sp0 < plan.nsplit2; sp0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = (sp0 + u < plan.nsplit2) ? __ldcg(base + (size_t)(sp0 + u) * p.G * D + lane + 32 * x) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) a += v[u];
+        }
         store_out(O + row_h * D + lane + 32 * x, a);
     }
 }

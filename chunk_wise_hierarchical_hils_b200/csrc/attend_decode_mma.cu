@@ -267,12 +267,31 @@ __global__ void __launch_bounds__(32 * SLOTS, 1)
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const float *all = partial + (size_t)bg * n_entries * G * kD;
-    for (int e = threadIdx.x; e < G * kD; e += 32 * SLOTS) {
-        float a = 0.f;
-        for (int en = 0; en < n_entries; ++en) a += __ldcg(all + (size_t)en * G * kD + e);
-        const int h = e / kD, x = e % kD;
-        store_out(O + ((size_t)b * p.H + (size_t)g * G + h) * kD + x, a);
+    // each thread adds four columns over the entries in slot order, with eight entries' loads in
+    // flight at a time (the entries come from L2; one at a time, the merge would be latency-bound)
+    const float4 *all = reinterpret_cast<const float4 *>(partial + (size_t)bg * n_entries * G * kD);
+    const int n4 = G * kD / 4;
+    for (int e4 = threadIdx.x; e4 < n4; e4 += 32 * SLOTS) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int en0 = 0; en0 < n_entries; en0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = (en0 + u < n_entries) ? __ldcg(all + (size_t)(en0 + u) * n4 + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                a.x += v[u].x;
+                a.y += v[u].y;
+                a.z += v[u].z;
+                a.w += v[u].w;
+            }
+        }
+        const int h = (4 * e4) / kD, x = (4 * e4) % kD;
+        Tout *dst = O + ((size_t)b * p.H + (size_t)g * G + h) * kD + x;
+        store_out(dst, a.x);
+        store_out(dst + 1, a.y);
+        store_out(dst + 2, a.z);
+        store_out(dst + 3, a.w);
     }
 }
 
