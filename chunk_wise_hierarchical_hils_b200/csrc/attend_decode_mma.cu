@@ -119,12 +119,21 @@ __global__ void __launch_bounds__(32 * SLOTS, 1)
             tma_load_2d(dst + 3 * HALF, &tmV, bar, 64, row);
         }
     }
-    // the group's query rows, bf16, rows G..15 zero
-    for (int e = threadIdx.x; e < 16 * 16; e += 32 * SLOTS) {
-        const int r = e >> 4, seg = e & 15;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < G) v = __ldg(reinterpret_cast<const uint4 *>(Q + ((size_t)b * p.H + (size_t)g * G + r) * kD) + seg);
-        *reinterpret_cast<uint4 *>(qs + r * kQPitch + seg * 16) = v;
+    // the group's query rows, bf16, rows G..15 zero (all of a thread's loads issued before its stores)
+    {
+        constexpr int PER = 256 / (32 * SLOTS);
+        uint4 v[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = threadIdx.x + u * 32 * SLOTS, r = e >> 4, seg = e & 15;
+            v[u] = (r < G) ? __ldg(reinterpret_cast<const uint4 *>(Q + ((size_t)b * p.H + (size_t)g * G + r) * kD) + seg)
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = threadIdx.x + u * 32 * SLOTS, r = e >> 4, seg = e & 15;
+            *reinterpret_cast<uint4 *>(qs + r * kQPitch + seg * 16) = v[u];
+        }
     }
     for (int h = warp; h < G; h += SLOTS)
         warp_fusion_weights(sel_score + ((size_t)b * p.H + (size_t)g * G + h) * ns, ns, j0, j1, wsm + h * SLOTS);

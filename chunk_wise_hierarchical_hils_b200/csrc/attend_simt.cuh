@@ -120,21 +120,25 @@ __device__ __forceinline__ void warp_attend_chunk(const float *qsm, const Tin *K
 
 // Fusion weights of the slots [j0, j1) for one head: softmax over all ns slot
 // scores (-inf = empty slot).  Warp-cooperative; lane 0.. writes w[j - j0].
+// The row's scores (ns <= HILS_MAX_K + 1 <= 96) are read once, all at the same time.
 __device__ __forceinline__ void warp_fusion_weights(const float *score_row, int ns, int j0, int j1, float *w)
 {
     const int lane = threadIdx.x & 31;
-    float mx = -INFINITY;
-    for (int j = lane; j < ns; j += 32) mx = fmaxf(mx, score_row[j]);
-    mx = warp_max(mx);
-    float z = 0.f;
-    for (int j = lane; j < ns; j += 32) {
-        const float s = score_row[j];
-        z += (s == -INFINITY) ? 0.f : expf(s - mx);
+    float s[3];
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+        const int j = lane + 32 * u;
+        s[u] = (j < ns) ? score_row[j] : -INFINITY;
     }
+    float mx = warp_max(fmaxf(fmaxf(s[0], s[1]), s[2]));
+    float z = 0.f;
+#pragma unroll
+    for (int u = 0; u < 3; ++u) z += (s[u] == -INFINITY) ? 0.f : expf(s[u] - mx);
     z = warp_sum(z);
-    for (int j = j0 + lane; j < j1; j += 32) {
-        const float s = score_row[j];
-        w[j - j0] = (s == -INFINITY) ? 0.f : expf(s - mx) / z;
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+        const int j = lane + 32 * u;
+        if (j >= j0 && j < j1) w[j - j0] = (s[u] == -INFINITY) ? 0.f : expf(s[u] - mx) / z;
     }
 }
 

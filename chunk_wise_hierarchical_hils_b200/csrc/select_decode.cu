@@ -77,8 +77,15 @@ __global__ void __launch_bounds__(NT) select_decode_kernel(Dims p, DecodePlan pl
         for (int s = 0; s < min(RING, n_stages); ++s) issue(s);
     }
     if (tid < D) {
+        // the G heads' values (G <= 16) loaded together, then added in head order
+        float v[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h)
+            v[h] = (h < p.G) ? to_float(Q[((size_t)b * p.H + (size_t)g * p.G + h) * D + tid]) : 0.f;
         float a = 0.f;
-        for (int h = 0; h < p.G; ++h) a += to_float(Q[((size_t)b * p.H + (size_t)g * p.G + h) * D + tid]);
+#pragma unroll
+        for (int h = 0; h < 16; ++h)
+            if (h < p.G) a += v[h];
         qs[tid] = a * (p.scale / (float)p.G);
     }
     __syncthreads();

@@ -148,14 +148,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = tid; e < p.k * kRows; e += kThreads) keys[e] = 0ull;
     // stage Q query-major in the 128-byte-swizzled K-major layout the MMA reads:
     // row r = query * G + head, two 64-column halves of 128 rows x 128 bytes
-    for (int e = tid; e < kRows * 16; e += kThreads) {
-        const int r = e >> 4, half = (e >> 3) & 1, j = e & 7;
-        const int qi = r / G, h = r % G;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (qi < nq)
-            v = __ldg(reinterpret_cast<const uint4 *>(
-                Q + ((((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi) * kD + half * 64 + j * 8));
-        *reinterpret_cast<uint4 *>(base + Ly.q + half * 16384u + (uint32_t)r * 128u + ((j ^ (r & 7)) << 4)) = v;
+    // (loads issued in batches of 8 per thread before the stores: one memory latency per batch)
+    for (int e0 = tid; e0 < kRows * 16; e0 += 8 * kThreads) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * kThreads;
+            const int r = e >> 4, half = (e >> 3) & 1, j = e & 7;
+            const int qi = r / G, h = r % G;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (e < kRows * 16 && qi < nq)
+                v[u] = __ldg(reinterpret_cast<const uint4 *>(
+                    Q + ((((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi) * kD + half * 64 + j * 8));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * kThreads;
+            const int r = e >> 4, half = (e >> 3) & 1, j = e & 7;
+            if (e < kRows * 16)
+                *reinterpret_cast<uint4 *>(base + Ly.q + half * 16384u + (uint32_t)r * 128u + ((j ^ (r & 7)) << 4)) =
+                    v[u];
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
