@@ -1,0 +1,57 @@
+"""Host-side pieces of the benchmark (CPU): the algorithmic work and bytes it reports, and the rule
+that an ncu traffic figure is used only for the kernel sources it was captured on."""
+import hashlib
+import importlib.util
+import json
+import os
+
+import pytest
+
+from synth.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def load_bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_algorithmic_figures_of_the_workloads():
+    b = load_bench()
+    w = WORKLOADS["prefill_8k"]
+    # 4 N (k+1) C d per head: 4 * 8192 * 17 * 64 * 128 * (4 * 32 heads)
+    assert b.attention_flops(w) == 4.0 * 8192 * 17 * 64 * 128 * 128
+    assert abs(b.attention_flops(w) - 5.841e11) / 5.841e11 < 1e-3
+    d = WORKLOADS["decode_128k"]
+    # landmarks of 2047 past chunks + K and V of 33 chunks of 64 rows, bf16, per (b, g), 128 of them
+    lm = 2 * 128 * 128 * 2047
+    kv = 2 * 128 * 128 * 33 * 2 * 64
+    assert b.landmark_bytes(d) == lm
+    assert b.decode_bytes(d) == lm + kv
+    assert abs(b.decode_bytes(d) - 205.5e6) / 205.5e6 < 1e-3   # about 205 MB a decode step
+
+
+def _fake_tree(tmp_path, text):
+    csrc = tmp_path / "chunk_wise_hierarchical_hils_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text(text)
+    (tmp_path / "profiles").mkdir()
+    rec = {"kern": {"workload": "prefill_8k", "dram_bytes_per_launch": 1234,
+                    "sources": {"k.cu": hashlib.sha256(b"kernel v1").hexdigest()}}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    return tmp_path
+
+
+@pytest.mark.parametrize("text,workload,expect", [
+    ("kernel v1", "prefill_8k", 1234),     # same source, same workload
+    ("kernel v2", "prefill_8k", None),     # source changed since the capture
+    ("kernel v1", "decode_128k", None),    # another workload
+])
+def test_traffic_only_for_the_captured_sources(tmp_path, text, workload, expect):
+    b = load_bench()
+    b.ROOT = str(_fake_tree(tmp_path, text))
+    assert b.kernel_traffic("kern", workload) == expect
+    assert b.kernel_traffic("missing", workload) is None
