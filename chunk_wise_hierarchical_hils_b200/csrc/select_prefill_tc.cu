@@ -96,6 +96,37 @@ __device__ __forceinline__ void list_insert(uint64_t (&a)[RK], float (&ap)[RK], 
     ap[0] = gt[0] ? xp : ap[0];
 }
 
+// Sort a[0..RK) (RK a power of two) into descending order, payloads alongside: a bitonic
+// network with every index known at compile time, so the list stays in registers.
+template <int RK>
+__device__ __forceinline__ void list_sort_desc(uint64_t (&a)[RK], float (&ap)[RK])
+{
+    static_assert(RK == 16, "the network below is written out for 16 entries");
+#pragma unroll
+    for (int ls = 1; ls <= 4; ++ls) {
+#pragma unroll
+        for (int lt = ls - 1; lt >= 0; --lt) {
+            const int size = 1 << ls, stride = 1 << lt;
+#pragma unroll
+            for (int i = 0; i < RK; ++i) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    // blocks with (i & size) == 0 go descending, the others ascending; the last
+                    // merge (size == RK) leaves everything descending
+                    const bool desc = (i & size) == 0;
+                    const bool swap = desc ? (a[i] < a[j]) : (a[i] > a[j]);
+                    const uint64_t ki = a[i], kj = a[j];
+                    const float pi = ap[i], pj = ap[j];
+                    a[i] = swap ? kj : ki;
+                    a[j] = swap ? ki : kj;
+                    ap[i] = swap ? pj : pi;
+                    ap[j] = swap ? pi : pj;
+                }
+            }
+        }
+    }
+}
+
 template <int G, int NSL, int RK>
 __global__ void __launch_bounds__(kThreads, 1)
     select_tc_kernel(const __grid_constant__ CUtensorMap tmL, Dims p, const __nv_bfloat16 *__restrict__ Q,
@@ -259,11 +290,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     if (RK > 0 && j == kQueue) {
-                        // the queue is full after kQueue candidates: insert them before going on
-                        const int m = __reduce_max_sync(0xFFFFFFFFu, qn);
-                        for (int i = 0; i < m; ++i) {
-                            const bool on = i < qn;
-                            list_insert<RKN>(top, topp, on ? hk[i * kRows] : 0ull, on ? hp[i * kRows] : 0.f, on);
+                        // the queue is full after kQueue candidates: insert them before going on.  The
+                        // first time the list is still empty and the queue holds at most RK keys: they
+                        // are copied in and sorted by a network instead of inserted one by one.
+                        bool filled = false;
+                        if constexpr (RKN == kQueue) {
+                            if (t == 0 && half == 0) {
+#pragma unroll
+                                for (int i = 0; i < RKN; ++i) {
+                                    const bool on = i < qn;
+                                    top[i] = on ? hk[i * kRows] : 0ull;
+                                    topp[i] = on ? hp[i * kRows] : 0.f;
+                                }
+                                list_sort_desc<RKN>(top, topp);
+                                filled = true;
+                            }
+                        }
+                        if (!filled) {
+                            const int m = __reduce_max_sync(0xFFFFFFFFu, qn);
+                            for (int i = 0; i < m; ++i) {
+                                const bool on = i < qn;
+                                list_insert<RKN>(top, topp, on ? hk[i * kRows] : 0ull, on ? hp[i * kRows] : 0.f, on);
+                            }
                         }
                         qn = 0;
                     }
