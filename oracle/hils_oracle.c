@@ -23,8 +23,8 @@
  * definition); the query's own chunk is always fused in addition to the K
  * retrieved past chunks, causally masked.
  *
- * Readings where the page is silent (each is listed with its reason in the
- * design notes):
+ * Readings where the page is silent (the plainest ones the rest of the page
+ * supports):
  *   - one scale (1/sqrt(d) by default) for retrieval scores and token logits;
  *   - the own chunk c_i = floor(p_i / C) is scored with its own landmark;
  *   - a query with fewer than K past chunks takes all of them;
