@@ -345,6 +345,170 @@ int hils_oracle_forward(int B, int H, int Hkv, int N, int T, int d, int C, int k
     return 0;
 }
 
+/* ---------------------------------------------------------------------------
+ * Extension for the next rows of the method (the local window and the bias of
+ * the surrogate mass).  The functions above are unchanged; these reduce to them
+ * with wc = 1 and no bias.
+ *
+ * Local window (Sec. 2 Preliminary: block-sparse attention combines a local
+ * sliding window with K retrieved chunks, the window aligned to chunk
+ * boundaries so that it never overlaps a retrieved chunk; Sec. 5, Experimental
+ * setup: a 512-token window with 64-token chunks): the window is the query's own
+ * chunk and the wc - 1 chunks before it; every one is attended like a retrieved
+ * chunk and fused by the same softmax over retrieval scores, and retrieval
+ * ranks only the chunks before the window.  (Reading: the pages do not say how
+ * the window enters the fusion; treating its chunks as always-retrieved chunks
+ * is the one that keeps a single hierarchical softmax, and with wc = 1 it is the
+ * method above.)
+ *
+ * Bias (Sec. 3, Linear surrogate for chunk mass: an affine surrogate of the
+ * chunk mass, query-summary relevance plus an entropy-based bias per chunk):
+ * bias[c] is added to every head's retrieval score of chunk c, so to the group
+ * score as well; the fusion weights use the biased scores.
+ * ------------------------------------------------------------------------- */
+
+/* Selection with a window of wc >= 1 chunks for one query group.
+ *   q    [G][d], L [c_i+1][d], bias [c_i+1] or NULL
+ *   sel  [k+wc]   out: top-min(k, #candidates) of chunks 0..c_i-wc in rank order
+ *                 (-1 padded), then the window chunks c_i-wc+1 .. c_i ascending
+ *                 (-1 for the ones before chunk 0)
+ *   shat [c_i+1]  out (may be NULL): biased group scores of chunks 0..c_i      */
+void hils_oracle_select_window(int G, int d, int C, int k, int wc, long pos, double scale,
+                               const double *q, const double *L, const double *bias, int *sel,
+                               double *shat_out)
+{
+    int ci = (int)(pos / C);
+    double *shat = (double *)malloc(sizeof(double) * (size_t)(ci + 1));
+    hils_oracle_group_scores(G, d, ci + 1, scale, q, L, shat);
+    if (bias)
+        for (int c = 0; c <= ci; ++c) shat[c] += bias[c];
+    int n_cand = PLANTED(14) ? ci : ci - wc + 1;  /* planted mistake 14: window chunks also candidates */
+    if (n_cand < 0) n_cand = 0;
+    hils_oracle_topk(n_cand, k, shat, sel);
+    for (int j = 0; j < wc; ++j) {
+        int c = ci - wc + 1 + j - (PLANTED(12) ? 1 : 0);   /* planted mistake 12: window one chunk early */
+        sel[k + j] = c >= 0 ? c : -1;
+    }
+    if (shat_out) memcpy(shat_out, shat, sizeof(double) * (size_t)(ci + 1));
+    free(shat);
+}
+
+/* Attention inside ns slots and their fusion, for one query group.
+ *   sel [ns] chunk per slot (-1 = empty); Lsel [ns][d]; bsel [ns] or NULL: the
+ *   slots' biases; Ksel, Vsel [ns][C][d]; s, w [G][ns]; o [G][d] (as
+ *   hils_oracle_attend, with s_{h,c} = scale q_h . L_c + bias_c).             */
+void hils_oracle_attend_slots(int G, int d, int C, int ns, long pos, double scale,
+                              const double *q, const int *sel, const double *Lsel, const double *bsel,
+                              const double *Ksel, const double *Vsel, double *s, double *w, double *o)
+{
+    double *ochunk = (double *)calloc((size_t)ns * d, sizeof(double));
+    double *logit = (double *)malloc(sizeof(double) * (size_t)C);
+    for (int h = 0; h < G; ++h) {
+        const double *qh = q + (size_t)h * d;
+        double *sh = s + (size_t)h * ns, *wh = w + (size_t)h * ns, *oh = o + (size_t)h * d;
+        memset(ochunk, 0, sizeof(double) * (size_t)ns * d);
+        for (int j = 0; j < ns; ++j) {
+            int c = sel[j];
+            if (c < 0) { sh[j] = -INFINITY; continue; }
+            sh[j] = retrieval_score(qh, Lsel + (size_t)j * d, d, scale) + ((bsel && !PLANTED(13)) ? bsel[j] : 0.0);
+                                                  /* planted mistake 13: bias left out of the fusion */
+            long first = (long)c * C;
+            int n_vis = 0;
+            for (int t = 0; t < C && first + t <= pos; ++t) {
+                logit[t] = scale * dot(qh, Ksel + ((size_t)j * C + t) * d, d);
+                n_vis = t + 1;
+            }
+            if (n_vis == 0) { sh[j] = -INFINITY; continue; }
+            double m = logit[0];
+            for (int t = 1; t < n_vis; ++t) if (logit[t] > m) m = logit[t];
+            double den = 0.0;
+            for (int t = 0; t < n_vis; ++t) den += exp(logit[t] - m);
+            double *ocj = ochunk + (size_t)j * d;
+            for (int t = 0; t < n_vis; ++t) {
+                double p = exp(logit[t] - m) / den;
+                const double *vt = Vsel + ((size_t)j * C + t) * d;
+                for (int x = 0; x < d; ++x) ocj[x] += p * vt[x];
+            }
+        }
+        double M = -INFINITY;
+        for (int j = 0; j < ns; ++j) if (sh[j] > M) M = sh[j];
+        double Z = 0.0;
+        for (int j = 0; j < ns; ++j) wh[j] = (sh[j] == -INFINITY) ? 0.0 : exp(sh[j] - M);
+        for (int j = 0; j < ns; ++j) Z += wh[j];
+        for (int j = 0; j < ns; ++j) wh[j] /= Z;
+        for (int x = 0; x < d; ++x) oh[x] = 0.0;
+        for (int j = 0; j < ns; ++j)
+            for (int x = 0; x < d; ++x) oh[x] += wh[j] * ochunk[(size_t)j * d + x];
+    }
+    free(logit);
+    free(ochunk);
+}
+
+/* Whole forward pass with a window of wc chunks and an optional bias
+ * [B][Hkv][nL]; layouts as hils_oracle_forward with k+wc slots per query. */
+int hils_oracle_forward_window(int B, int H, int Hkv, int N, int T, int d, int C, int k, int wc,
+                               long q_offset, double scale,
+                               const double *Q, const double *K, const double *V, const double *L,
+                               const double *bias, double *O, int *sel_out, double *s_out, double *w_out,
+                               int nthreads)
+{
+    if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N < 0 || T <= 0 || d <= 0 || C <= 0 || k < 0 || wc < 1)
+        return -1;
+    if (q_offset < 0 || q_offset + N > T) return -1;
+    int G = H / Hkv, nL = (T + C - 1) / C, ns = k + wc;
+    long n_items = (long)B * Hkv * N;
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double *q = (double *)malloc(sizeof(double) * (size_t)G * d);
+        double *Ls = (double *)malloc(sizeof(double) * (size_t)ns * d);
+        double *bs = (double *)malloc(sizeof(double) * (size_t)ns);
+        double *Ks = (double *)calloc((size_t)ns * C * d, sizeof(double));
+        double *Vs = (double *)calloc((size_t)ns * C * d, sizeof(double));
+        double *s = (double *)malloc(sizeof(double) * (size_t)G * ns);
+        double *w = (double *)malloc(sizeof(double) * (size_t)G * ns);
+        double *o = (double *)malloc(sizeof(double) * (size_t)G * d);
+        int *sel = (int *)malloc(sizeof(int) * (size_t)ns);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 16)
+#endif
+        for (long it = 0; it < n_items; ++it) {
+            int i = (int)(it % N), g = (int)((it / N) % Hkv), b = (int)(it / ((long)N * Hkv));
+            long pos = q_offset + i;
+            for (int h = 0; h < G; ++h)
+                memcpy(q + (size_t)h * d, Q + ((((size_t)b * H + (size_t)g * G + h) * N) + i) * d,
+                       sizeof(double) * (size_t)d);
+            const double *Lbg = L + ((size_t)b * Hkv + g) * nL * d;
+            const double *Kbg = K + ((size_t)b * Hkv + g) * T * d;
+            const double *Vbg = V + ((size_t)b * Hkv + g) * T * d;
+            const double *bbg = bias ? bias + ((size_t)b * Hkv + g) * nL : NULL;
+            hils_oracle_select_window(G, d, C, k, wc, pos, scale, q, Lbg, bbg, sel, NULL);
+            for (int j = 0; j < ns; ++j) {
+                int c = sel[j];
+                bs[j] = 0.0;
+                if (c < 0) continue;
+                bs[j] = bbg ? bbg[c] : 0.0;
+                memcpy(Ls + (size_t)j * d, Lbg + (size_t)c * d, sizeof(double) * (size_t)d);
+                int rows = (c + 1) * C <= T ? C : T - c * C;
+                memcpy(Ks + (size_t)j * C * d, Kbg + (size_t)c * C * d, sizeof(double) * (size_t)rows * d);
+                memcpy(Vs + (size_t)j * C * d, Vbg + (size_t)c * C * d, sizeof(double) * (size_t)rows * d);
+            }
+            hils_oracle_attend_slots(G, d, C, ns, pos, scale, q, sel, Ls, bbg ? bs : NULL, Ks, Vs, s, w, o);
+            for (int h = 0; h < G; ++h) {
+                size_t row = (((size_t)b * H + (size_t)g * G + h) * N) + i;
+                if (O) memcpy(O + row * d, o + (size_t)h * d, sizeof(double) * (size_t)d);
+                if (s_out) memcpy(s_out + row * ns, s + (size_t)h * ns, sizeof(double) * (size_t)ns);
+                if (w_out) memcpy(w_out + row * ns, w + (size_t)h * ns, sizeof(double) * (size_t)ns);
+            }
+            if (sel_out) memcpy(sel_out + ((((size_t)b * Hkv + g) * N) + i) * ns, sel, sizeof(int) * (size_t)ns);
+        }
+        free(q); free(Ls); free(bs); free(Ks); free(Vs); free(s); free(w); free(o); free(sel);
+    }
+    return 0;
+}
+
 /* Threads the OpenMP runtime would use (1 without OpenMP). */
 int hils_oracle_max_threads(void)
 {

@@ -48,6 +48,9 @@ def lib():
         L.hils_oracle_forward.argtypes = [ctypes.c_int] * 8 + [ctypes.c_long, ctypes.c_double, _D, _D, _D, _D,
                                                                _D, _I, _D, _D, ctypes.c_int]
         L.hils_oracle_forward.restype = ctypes.c_int
+        L.hils_oracle_forward_window.argtypes = [ctypes.c_int] * 9 + [ctypes.c_long, ctypes.c_double, _D, _D, _D,
+                                                                      _D, _D, _D, _I, _D, _D, ctypes.c_int]
+        L.hils_oracle_forward_window.restype = ctypes.c_int
         L.hils_oracle_max_threads.restype = ctypes.c_int
     return _lib
 
@@ -93,6 +96,37 @@ def forward(Q, K, V, L, C, k, q_offset=0, scale=None, nthreads=None):
     nthreads = max_threads() if nthreads is None else nthreads
     rc = lib().hils_oracle_forward(B, H, Hkv, N, T, d, C, k, q_offset, scale, _dp(Q), _dp(K), _dp(V), _dp(L),
                                    _dp(O), _ip(sel), _dp(s), _dp(w), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the shapes")
+    return {"O": O, "sel": sel, "s": s, "w": w}
+
+
+def forward_window(Q, K, V, L, C, k, wc, q_offset=0, scale=None, bias=None, nthreads=None):
+    """Forward pass with a local window of wc chunks (the own chunk and the wc-1 before it, always
+    attended; retrieval ranks only the chunks before the window) and an optional per-chunk bias
+    [B,Hkv,ceil(T/C)] added to the retrieval scores.  wc = 1 and bias None give forward().
+
+    Returns dict with O [B,H,N,d], sel [B,Hkv,N,k+wc] (top-k in rank order, then the window
+    chunks ascending), s and w [B,H,N,k+wc].
+    """
+    Q, K, V, L = _f64(Q), _f64(K), _f64(V), _f64(L)
+    B, H, N, d = Q.shape
+    _, Hkv, T, _ = K.shape
+    nL = -(-T // C)
+    assert L.shape == (B, Hkv, nL, d), L.shape
+    if bias is not None:
+        bias = _f64(bias)
+        assert bias.shape == (B, Hkv, nL), bias.shape
+    scale = default_scale(d) if scale is None else scale
+    ns = k + wc
+    O = np.zeros((B, H, N, d))
+    sel = np.zeros((B, Hkv, N, ns), dtype=np.int32)
+    s = np.zeros((B, H, N, ns))
+    w = np.zeros((B, H, N, ns))
+    nthreads = max_threads() if nthreads is None else nthreads
+    rc = lib().hils_oracle_forward_window(B, H, Hkv, N, T, d, C, k, wc, q_offset, scale, _dp(Q), _dp(K), _dp(V),
+                                          _dp(L), _dp(bias) if bias is not None else None, _dp(O), _ip(sel),
+                                          _dp(s), _dp(w), int(nthreads))
     if rc != 0:
         raise ValueError("oracle rejected the shapes")
     return {"O": O, "sel": sel, "s": s, "w": w}
