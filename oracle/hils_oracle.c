@@ -509,6 +509,49 @@ int hils_oracle_forward_window(int B, int H, int Hkv, int N, int T, int d, int C
     return 0;
 }
 
+/* Landmarks and their biases from the chunks' keys (Sec. 3, Linear surrogate for
+ * chunk mass: a landmark token appended to each chunk supplies a learned query;
+ * that query's distribution over the chunk's keys weights the key sum that forms
+ * the summary, and the entropy-based bias tends to log S for uniform scores and
+ * to 0 when one score dominates).  For chunk c with landmark query u_c:
+ *     p_t  = softmax_t(scale * u_c . k_t) over the chunk's keys (a partial last chunk
+ *            uses the keys it has),
+ *     L_c  = sum_t p_t k_t,
+ *     beta_c = -sum_t p_t log p_t   (the entropy of p).
+ * (Reading: the summary page names the ingredients, not the formula; this is the
+ * plain one, and with it scale * q . L_c + beta_c never exceeds the chunk's
+ * log-sum-exp mass log sum_t exp(scale * q . k_t), with equality for q = u_c.)
+ *   K [T][d] of one (b, g); U [nL][d] landmark queries; L [nL][d], beta [nL] out. */
+void hils_oracle_landmarks(int T, int d, int C, double scale, const double *K, const double *U,
+                           double *L, double *beta)
+{
+    int nL = (T + C - 1) / C;
+    double *sc = (double *)malloc(sizeof(double) * (size_t)C);
+    for (int c = 0; c < nL; ++c) {
+        int rows = (c + 1) * C <= T ? C : T - c * C;
+        const double *u = U + (size_t)c * d;
+        double m = -INFINITY;
+        for (int t = 0; t < rows; ++t) {
+            sc[t] = (PLANTED(15) ? 1.0 : scale) * dot(u, K + ((size_t)c * C + t) * d, d);
+                                                  /* planted mistake 15: scale dropped from the landmark scores */
+            if (sc[t] > m) m = sc[t];
+        }
+        double z = 0.0;
+        for (int t = 0; t < rows; ++t) z += exp(sc[t] - m);
+        double *Lc = L + (size_t)c * d, h = 0.0;
+        for (int x = 0; x < d; ++x) Lc[x] = 0.0;
+        for (int t = 0; t < rows; ++t) {
+            double pt = exp(sc[t] - m) / z;
+            const double *kt = K + ((size_t)c * C + t) * d;
+            for (int x = 0; x < d; ++x) Lc[x] += pt * kt[x];
+            if (pt > 0.0) h -= pt * log(pt);
+        }
+        beta[c] = PLANTED(16) ? -h : PLANTED(17) ? log((double)rows) : h;
+                                                  /* planted mistakes 16, 17: entropy negated; log C always */
+    }
+    free(sc);
+}
+
 /* Threads the OpenMP runtime would use (1 without OpenMP). */
 int hils_oracle_max_threads(void)
 {

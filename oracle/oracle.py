@@ -51,6 +51,7 @@ def lib():
         L.hils_oracle_forward_window.argtypes = [ctypes.c_int] * 9 + [ctypes.c_long, ctypes.c_double, _D, _D, _D,
                                                                       _D, _D, _D, _I, _D, _D, ctypes.c_int]
         L.hils_oracle_forward_window.restype = ctypes.c_int
+        L.hils_oracle_landmarks.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, _D, _D, _D]
         L.hils_oracle_max_threads.restype = ctypes.c_int
     return _lib
 
@@ -130,6 +131,27 @@ def forward_window(Q, K, V, L, C, k, wc, q_offset=0, scale=None, bias=None, nthr
     if rc != 0:
         raise ValueError("oracle rejected the shapes")
     return {"O": O, "sel": sel, "s": s, "w": w}
+
+
+def landmarks(K, U, C, scale=None):
+    """Landmarks L [B,Hkv,nL,d] and entropy biases beta [B,Hkv,nL] from keys K [B,Hkv,T,d] and
+    per-chunk landmark queries U [B,Hkv,nL,d]: L_c = sum_t p_t k_t, beta_c = -sum_t p_t log p_t,
+    p = softmax over the chunk's keys of scale * u_c . k_t."""
+    K, U = _f64(K), _f64(U)
+    B, Hkv, T, d = K.shape
+    nL = -(-T // C)
+    assert U.shape == (B, Hkv, nL, d), U.shape
+    scale = default_scale(d) if scale is None else scale
+    L = np.zeros((B, Hkv, nL, d))
+    beta = np.zeros((B, Hkv, nL))
+    for b in range(B):
+        for g in range(Hkv):
+            Lbg = np.zeros((nL, d))
+            bbg = np.zeros(nL)
+            lib().hils_oracle_landmarks(T, d, C, scale, _dp(np.ascontiguousarray(K[b, g])),
+                                        _dp(np.ascontiguousarray(U[b, g])), _dp(Lbg), _dp(bbg))
+            L[b, g], beta[b, g] = Lbg, bbg
+    return L, beta
 
 
 def group_scores(q, Lrows, scale):
