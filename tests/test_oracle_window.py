@@ -137,11 +137,23 @@ def test_weights_are_a_distribution_over_filled_slots():
     assert np.all((w == 0) == np.isneginf(s))
 
 
+def test_decode_equals_the_last_prefill_query():
+    # one query at the last position of the cache gives the same result as the last query of the
+    # full prefill (the window and the bias depend on the position only)
+    B, H, Hkv, T, d, C = 1, 4, 2, 203, 8, 16
+    Q, K, V, L = _problem(23, B, H, Hkv, T, d, C)
+    bias = np.random.default_rng(24).standard_normal((B, Hkv, -(-T // C)))
+    full = orc.forward_window(Q, K, V, L, C=C, k=3, wc=2, bias=bias, nthreads=2)
+    one = orc.forward_window(Q[:, :, T - 1:T], K, V, L, C=C, k=3, wc=2, q_offset=T - 1, bias=bias, nthreads=1)
+    assert np.array_equal(full["sel"][:, :, T - 1:T], one["sel"])
+    assert np.max(np.abs(full["O"][:, :, T - 1:T] - one["O"])) <= 1e-15
+
+
 PINS = [test_one_chunk_window_without_bias_is_the_method, test_window_covering_every_chunk_is_dense_causal_attention,
         test_window_only_is_sliding_window_attention, test_window_plus_full_retrieval_is_dense,
         test_window_and_retrieved_chunks_are_disjoint_and_ordered, test_selection_is_the_best_biased_subset,
         test_common_bias_changes_nothing_and_a_large_bias_is_retrieved_first,
-        test_weights_are_a_distribution_over_filled_slots]
+        test_weights_are_a_distribution_over_filled_slots, test_decode_equals_the_last_prefill_query]
 
 PLANTED = {
     12: "window taken one chunk early (own chunk left out)",
