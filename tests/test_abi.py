@@ -94,3 +94,26 @@ def test_status_strings():
     for s in range(6):
         assert hils.hils_status_string(s).startswith("HILS_")
     assert "unknown" in hils.hils_status_string(99)
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """A C99 program that includes only the header compiles, links against the library and calls it
+    (no GPU work: the version and a status string)."""
+    import subprocess
+    src = tmp_path / "use_hils.c"
+    src.write_text(
+        '#include "hils.h"\n'
+        "#include <stdio.h>\n"
+        "int main(void) {\n"
+        "    hils_problem p = {0};\n"
+        "    size_t bytes = 0;\n"
+        "    (void)p; (void)bytes;\n"
+        '    printf("%d %s\\n", hils_version(), hils_status_string(HILS_OK));\n'
+        "    return 0;\n"
+        "}\n")
+    exe = tmp_path / "use_hils"
+    libdir = os.path.dirname(hils.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-L", libdir, "-lhils", "-Wl,-rpath," + libdir, "-o", str(exe)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out[0] == "100"
