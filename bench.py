@@ -40,6 +40,9 @@ def parse():
     ap.add_argument("--cpu-blocks", type=int, default=16, help="64-query blocks in the oracle sample")
     ap.add_argument("--override", nargs="*", default=[], metavar="KEY=VALUE",
                     help="change workload fields, e.g. B=4 T=524288 q_offset=524287 (smaller profiling cases)")
+    ap.add_argument("--part", default="forward", choices=["forward", "landmarks"],
+                    help="forward: the hot path (default); landmarks: landmark generation over the "
+                         "workload's whole key cache")
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
                     help="weak: every rank runs the whole workload; strong: the batch is split over ranks")
     return ap.parse_args()
@@ -69,6 +72,13 @@ def decode_bytes(w):
 def landmark_bytes(w):
     es = 2 if w.dtype == "bf16" else 4
     return es * w.B * w.Hkv * w.d * (w.q_offset // w.C)
+
+
+def landmark_gen_bytes(w):
+    """Landmark generation over every chunk: the key cache and the landmark queries read once, the
+    landmarks and the float biases written once."""
+    es = 2 if w.dtype == "bf16" else 4
+    return w.B * w.Hkv * (es * w.T * w.d + 2 * es * w.nL * w.d + 4 * w.nL)
 
 
 def kernels_per_step(w):
@@ -451,6 +461,108 @@ def run_hils(args, w):
         dist.destroy_process_group()
 
 
+def run_landmarks(args, w):
+    """Landmark generation (hils_landmarks) over the workload's whole key cache, one call per step.
+
+    The landmark queries are the workload's landmark tensor (seeded synthetic values of the same shape);
+    the metric is algorithmic bytes per second against the measured copy bandwidth."""
+    import torch
+    import chunk_wise_hierarchical_hils_b200 as hils
+    from synth import gpu as synth_gpu
+
+    ws, rank, local = dist_setup(args)
+    dev = synth_gpu.alloc_inputs(w)
+    del dev["Q"], dev["V"]
+    dt = {"f32": hils.HILS_F32, "bf16": hils.HILS_BF16}[w.dtype]
+    p = hils.problem(w.B, 1, w.Hkv, 1, w.T, w.d, w.C, 0, 0, dt, dt)
+    K, U = dev["K"], dev["L"]
+    Lout = torch.empty_like(U)
+    beta = torch.empty((w.B, w.Hkv, w.nL), dtype=torch.float32, device="cuda")
+    nbytes = landmark_gen_bytes(w)
+
+    def call():
+        hils.hils_landmarks(p, K, U, Lout, beta)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    g_ = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_):
+        call()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    barrier(ws)
+    torch.cuda.synchronize()
+    sampler.start()
+    a_, z_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_.record(stream)
+    for _ in range(args.steps):
+        g_.replay()
+    z_.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop()
+    ms = allmax(ws, [a_.elapsed_time(z_) / args.steps])[0]
+    del g_
+    if hils.hils_sync_status() != hils.HILS_OK:
+        raise RuntimeError("device-side failure")
+
+    # end to end: keys and landmark queries from pinned host memory, landmarks and biases back
+    Kh, Uh = K.cpu().pin_memory(), U.cpu().pin_memory()
+    Lh, bh = torch.empty(Lout.shape, dtype=Lout.dtype).pin_memory(), torch.empty(beta.shape).pin_memory()
+
+    def e2e_step():
+        K.copy_(Kh, non_blocking=True)
+        U.copy_(Uh, non_blocking=True)
+        call()
+        Lh.copy_(Lout, non_blocking=True)
+        bh.copy_(beta, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allmax(ws, [e0.elapsed_time(e1) / args.e2e_steps])[0]
+
+    pk, pk_kind = peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    value = ws * achieved
+    line = {"metric": "HiLS landmark generation GB/s at 1 B200; % of HBM roofline", "value": value,
+            "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded Philox4x32-10 inputs)", "config": dict(config_of(w, ws), part="landmarks"),
+            "roofline": {"bound": "hbm", "kernel": "landmarks", "achieved": achieved, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                         "peak_kind": pk_kind + " copy", "algorithmic_bytes_per_launch": nbytes,
+                         "launch_ms": ms},
+            "e2e": {"value": ws * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": Kh.numel() * Kh.element_size() + Uh.numel() * Uh.element_size(),
+                    "d2h_bytes_per_step": Lh.numel() * Lh.element_size() + bh.numel() * 4, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps, "clocks": clocks,
+            "timing": "CUDA-graph replays of one hils_landmarks call, CUDA events on the replay stream"}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        from oracle import oracle as orc
+        n = min(w.nL, 4096)                      # a bounded slice: the first n chunks of (b, g) = (0, 0)
+        K64 = K[0:1, 0:1, :min(w.T, n * w.C)].double().cpu().numpy()
+        U64 = U[0:1, 0:1, :n].double().cpu().numpy()
+        t0 = time.perf_counter()
+        orc.landmarks(K64, U64, w.C)
+        t = time.perf_counter() - t0
+        es = 2 if w.dtype == "bf16" else 4
+        line["cpu_baseline"] = {"value": (K64.size + 2 * U64.size) * es / t / 1e9, "unit": "GB/s", "cores": 1,
+                                "kind": "oracle", "sample": "%d chunks of one (b, kv-head), one thread" % n}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     from synth.workloads import WORKLOADS
@@ -459,8 +571,12 @@ def main():
         kv = dict(x.split("=", 1) for x in args.override)
         w = w.with_(**{k: type(getattr(w, k))(v) for k, v in kv.items()})
         w = w.with_(name=w.name + "[" + ",".join(args.override) + "]")
+    if args.impl == "reference" and args.part == "landmarks":
+        raise SystemExit("--part landmarks times the library; its line carries the oracle as cpu_baseline")
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.part == "landmarks":
+        run_landmarks(args, w)
     else:
         run_hils(args, w)
 

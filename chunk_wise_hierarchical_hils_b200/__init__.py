@@ -27,7 +27,7 @@ HILS_MAX_GROUP = 16
 EXPORTS = ("hils_status_string", "hils_version", "hils_validate", "hils_score_select_workspace_size",
            "hils_chunk_attend_fuse_workspace_size", "hils_forward_workspace_size", "hils_score_select",
            "hils_chunk_attend_fuse", "hils_forward", "hils_sync_status", "hils_set_wait_limit",
-           "hils_decode_score_select_noalloc", "hils_debug_inject_stall")
+           "hils_decode_score_select_noalloc", "hils_debug_inject_stall", "hils_landmarks")
 HILS_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -68,6 +68,7 @@ def _load():
     lib.hils_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.hils_decode_score_select_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
     lib.hils_debug_inject_stall.argtypes = [ctypes.c_int]
+    lib.hils_landmarks.argtypes = [P, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp]
     for n in EXPORTS[2:]:
         if n not in ("hils_status_string", "hils_version"):
             getattr(lib, n).restype = ctypes.c_int
@@ -183,6 +184,16 @@ def hils_decode_score_select_noalloc(p, Q, L, sel_idx, sel_score, stream=None):
     _check(_lib.hils_decode_score_select_noalloc(ctypes.byref(p), _ptr(Q), _ptr(L), _ptr(sel_idx),
                                                  _ptr(sel_score), _stream(stream)),
            "hils_decode_score_select_noalloc")
+
+
+def hils_landmarks(p, K, U, L, beta=None, c_begin=0, c_end=None, stream=None):
+    """Landmarks L and entropy biases beta of chunks [c_begin, c_end) from keys K and landmark queries U.
+
+    c_end defaults to the number of chunks, ceil(T / C); see include/hils.h."""
+    if c_end is None:
+        c_end = (p.T + p.C - 1) // p.C
+    _check(_lib.hils_landmarks(ctypes.byref(p), _ptr(K), _ptr(U), _ptr(L), _ptr(beta), int(c_begin), int(c_end),
+                               _stream(stream)), "hils_landmarks")
 
 
 def problem(B, H, Hkv, N, T, d, C, k, q_offset=0, in_dtype=HILS_BF16, out_dtype=None, scale=0.0):

@@ -251,6 +251,25 @@ hils_status hils_forward(const hils_problem *p, const void *Q, const void *K, co
     return do_attend(d, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, scratch, s);
 }
 
+hils_status hils_landmarks(const hils_problem *p, const void *K, const void *U, void *L, float *beta, int c_begin,
+                           int c_end, void *stream)
+{
+    if (!p) return HILS_ERR_INVALID_ARG;
+    if (p->B < 1 || p->Hkv < 1 || p->T < 1 || p->C < 1) return HILS_ERR_INVALID_ARG;
+    if (p->in_dtype != HILS_F32 && p->in_dtype != HILS_BF16) return HILS_ERR_INVALID_ARG;
+    if (!(p->scale >= 0.f) || isinf(p->scale)) return HILS_ERR_INVALID_ARG;
+    if (p->d != 64 && p->d != 128) return HILS_ERR_UNSUPPORTED;
+    const long long nL = ((long long)p->T + p->C - 1) / p->C;
+    if (c_begin < 0 || c_end < c_begin || c_end > nL) return HILS_ERR_INVALID_ARG;
+    if (!K || !U || !L) return HILS_ERR_INVALID_ARG;
+    if (!aligned16(K) || !aligned16(U) || !aligned16(L) || (reinterpret_cast<uintptr_t>(beta) & 3u))
+        return HILS_ERR_INVALID_ARG;
+    if (!landmarks_launchable(p->B, p->Hkv, c_end - c_begin)) return HILS_ERR_UNSUPPORTED;
+    const float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+    return from_cuda(launch_landmarks(p->B, p->Hkv, p->T, p->d, p->C, scale, p->in_dtype, K, U, L, beta, c_begin,
+                                      c_end, static_cast<cudaStream_t>(stream)));
+}
+
 hils_status hils_sync_status(void *stream)
 {
     DeviceCtl ctl;

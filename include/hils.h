@@ -143,6 +143,31 @@ HILS_API hils_status hils_forward(const hils_problem *p, const void *Q, const vo
                          void *stream);
 
 /*
+ * Landmark generation (Sec. 3 Methodology, "Linear surrogate for chunk mass":
+ * a landmark token appended to each chunk supplies a learned query whose
+ * attention over the chunk's keys yields the chunk's compressed key).  For
+ * every (b, g) and every chunk c in [c_begin, c_end), with key rows
+ * t = c*C .. min(c*C + C, T) - 1 and landmark query u_c:
+ *   p_t    = softmax over the chunk's rows of scale * <u_c, k_t>
+ *   L_c    = sum_t p_t k_t        (in_dtype; bf16 rounded to nearest even)
+ *   beta_c = -sum_t p_t ln p_t    (float, the entropy: 0 <= beta_c <= ln rows)
+ * Layouts: K [B][Hkv][T][d], U [B][Hkv][nL][d] and L [B][Hkv][nL][d] in
+ * in_dtype, beta [B][Hkv][nL] float, nL = ceil(T / C); rows of L and beta
+ * outside [c_begin, c_end) are not written.  beta may be NULL (not written).
+ * L must not overlap K or U.
+ * Uses p->B, Hkv, T, d, C, in_dtype and scale (0 selects 1/sqrt(d)); the
+ * other fields are ignored.  Here C may be any chunk size >= 1 (the last
+ * chunk may be partial); d is 64 or 128 (else HILS_ERR_UNSUPPORTED).
+ * K, U and L 16-byte aligned, beta 4-byte aligned; 0 <= c_begin <= c_end <= nL
+ * (else HILS_ERR_INVALID_ARG, nothing launched; c_begin == c_end launches
+ * nothing).  A decode step that completes chunk c calls it with
+ * c_begin = c, c_end = c + 1.  Reads every key row of the range once; needs
+ * no workspace; asynchronous on `stream`.
+ */
+HILS_API hils_status hils_landmarks(const hils_problem *p, const void *K, const void *U, void *L, float *beta,
+                                    int c_begin, int c_end, void *stream);
+
+/*
  * Synchronise `stream` and report device-side status since the last call:
  * HILS_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the kernel then
  * skipped its remaining work and released its resources), HILS_ERR_CUDA if

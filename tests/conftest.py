@@ -9,3 +9,16 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+# Suites that run after all others, in this order, so that a run stopping at its first failure has
+# already run the forward-path suites: the allocation-free entry point (its first call sets up a
+# per-device array) and landmark generation (a step before the forward path).
+RUN_LAST = ("test_zz_no_alloc.py", "test_parity_landmarks.py")
+
+
+def pytest_collection_modifyitems(config, items):
+    def order(item):
+        name = os.path.basename(str(item.fspath))
+        return RUN_LAST.index(name) + 1 if name in RUN_LAST else 0
+    items.sort(key=order)

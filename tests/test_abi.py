@@ -78,6 +78,32 @@ def test_errors_before_launch():
     assert e.value.status == hils.HILS_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("kw,args,status", [
+    ({"d": 96}, (16, 16, 16, 16, 0, 4), hils.HILS_ERR_UNSUPPORTED),
+    ({"C": 0}, (16, 16, 16, 16, 0, 4), hils.HILS_ERR_INVALID_ARG),
+    ({}, (16, 16, 16, 16, 0, 5), hils.HILS_ERR_INVALID_ARG),         # c_end past the last chunk (T/C = 4)
+    ({}, (16, 16, 16, 16, 3, 2), hils.HILS_ERR_INVALID_ARG),         # c_end < c_begin
+    ({}, (16, 16, 16, 16, -1, 2), hils.HILS_ERR_INVALID_ARG),
+    ({}, (0, 16, 16, 16, 0, 4), hils.HILS_ERR_INVALID_ARG),          # K null
+    ({}, (16, 16, 24, 16, 0, 4), hils.HILS_ERR_INVALID_ARG),         # L misaligned
+    ({}, (16, 16, 32, 18, 0, 4), hils.HILS_ERR_INVALID_ARG),         # beta misaligned
+    ({"scale": float("inf")}, (16, 16, 16, 16, 0, 4), hils.HILS_ERR_INVALID_ARG),
+])
+def test_landmarks_errors_before_launch(kw, args, status):
+    """hils_landmarks checks its shape, range and pointers on the host; only B, Hkv, T, d, C, dtype, scale count."""
+    p = prob(**kw)
+    K, U, L, beta, c0, c1 = args
+    with pytest.raises(hils.HilsError) as e:
+        hils.hils_landmarks(p, K, U, L, beta, c0, c1, stream=0)
+    assert e.value.status == status
+
+
+def test_landmarks_empty_range_launches_nothing():
+    # fields the call does not use may hold anything; an empty chunk range returns at once
+    p = prob(H=3, N=0, k=-5, C=7)
+    hils.hils_landmarks(p, 16, 16, 32, None, 2, 2, stream=0)
+
+
 def test_workspace_sizes():
     p = prob()
     assert hils.hils_score_select_workspace_size(p) == 0

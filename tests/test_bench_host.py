@@ -34,6 +34,16 @@ def test_algorithmic_figures_of_the_workloads():
     assert abs(b.decode_bytes(d) - 205.5e6) / 205.5e6 < 1e-3   # about 205 MB a decode step
 
 
+def test_landmark_generation_bytes():
+    b = load_bench()
+    w = WORKLOADS["decode_4m_needles"]
+    # per kv-head: 4,194,304 key rows of 128 bf16, then 65,536 landmark queries in and landmarks out
+    # (128 bf16 each) and 65,536 float biases out; 8 kv-heads
+    per_head = 4194304 * 128 * 2 + 2 * 65536 * 128 * 2 + 65536 * 4
+    assert b.landmark_gen_bytes(w) == 8 * per_head
+    assert abs(b.landmark_gen_bytes(w) - 8.86e9) / 8.86e9 < 1e-3
+
+
 def _fake_tree(tmp_path, text):
     csrc = tmp_path / "chunk_wise_hierarchical_hils_b200" / "csrc"
     csrc.mkdir(parents=True)
