@@ -58,6 +58,7 @@ constexpr int kRows = 128;        // MMA M
 constexpr int kChunk = 64;        // C
 constexpr int kD = 128;           // d
 constexpr int kSP = 2;                // S buffers (a pair of chunks, 128 columns each) = key ring slots
+constexpr int kPB = 2;                // P buffers (a pair of chunks, 64 columns each)
 constexpr uint32_t kTmemCols = 512;   // S pair buffers (2 x 128 columns), O (128), up to 2 P pair buffers (64 each)
 constexpr uint32_t kColO = 256, kColP = 384;
 constexpr uint32_t kPairBytes = 32768;   // K and V ring slots: [c0 d0-63 | c1 d0-63 | c0 d64-127 | c1 d64-127]
@@ -99,19 +100,27 @@ __host__ __device__ inline Layout make_layout(int nsk, int nsv, int k, int nword
     return L;
 }
 
-// Barrier slots.  Key slot / S buffer b (pair p uses b = p % 2) and value slot / P buffer s (pair p
-// uses s = p % NSV):
+// Barrier slots.  Key slot / S buffer b (pair p uses b = p % 2), P buffer b (p % 2 as well: TMEM
+// always holds two) and value slot v (p % NSV):
 //   K_LAND[b]    the pair's key tiles have landed (TMA transaction count)
 //   QK_READY[b]  S buffer b may take pair p: its key tiles are in (the key loader's arrival) and all
 //                eight softmax warps of its two chunks have read pair p - 2 out of it
 //   QK_DONE[b]   the key product of pair p is complete: S is ready and the key slot is free
-//   V_LAND[s], PV_READY[s] (the value loader + the eight softmax warps that wrote P), PV_DONE[s] alike
-// so the MMA issuer tests one barrier per product and commits to one.
+//   V_LAND[v]    the pair's value tiles have landed
+//   PV_READY[b]  the value product of pair p may start: its values are in (the value loader's
+//                arrival) and the eight softmax warps of its two chunks wrote P buffer b
+//   PV_DONE[b]   the value product of pair p is complete: P buffer b is free, and so is the value
+//                slot of pair p
+// so the MMA issuer tests one barrier per product and commits to one.  P buffers and their barriers
+// go by p % 2 even with a single value slot: a softmax warp skips pairs (chunk t goes to group
+// t % 3), and a parity wait is only sound while the waiter is at most one phase behind, which two
+// P buffers guarantee (a warp that writes pair p has already seen the value product of p - 4 done)
+// and one would not.
 template <int NSV>
 struct Bars {
     static constexpr int Q_FULL = 0, K_LAND = 1, QK_READY = K_LAND + kSP, QK_DONE = QK_READY + kSP,
-                         V_LAND = QK_DONE + kSP, PV_READY = V_LAND + NSV, PV_DONE = PV_READY + NSV,
-                         O_FULL = PV_DONE + NSV, MMA_DONE = O_FULL + 1;   // MMA_DONE + 0/1: the two issuers
+                         V_LAND = QK_DONE + kSP, PV_READY = V_LAND + NSV, PV_DONE = PV_READY + kPB,
+                         O_FULL = PV_DONE + kPB, MMA_DONE = O_FULL + 1;   // MMA_DONE + 0/1: the two issuers
     static_assert(MMA_DONE + 1 < kMaxBars, "barrier slots");
 };
 
@@ -151,10 +160,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, unsigne
 }
 
 // One loader thread streams n tiles through a ring of `slots` buffers: tile i goes to slot i % slots
-// once the consumer has finished tile i - slots (its `done` barrier), lands on `land`, and is then
-// announced on `ready` (which other arrivals may share; the last tile's announcement counts
-// 1 + tail_extra arrivals).  Up to `slots` tiles are in flight.  On an abort the thread waits, with its
-// own bound, for the copies it started.  Returns the tiles announced.
+// once the consumer has finished tile i - slots (completion barriers `done` go by tile % 2), lands on
+// `land` (by slot), and is then announced on `ready` (by tile % 2; other arrivals may share it; the
+// last tile's announcement counts 1 + tail_extra arrivals).  Up to `slots` tiles are in flight.  On
+// an abort the thread waits, with its own bound, for the copies it started.  Returns the tiles
+// announced.
 template <typename Issue>
 __device__ __forceinline__ int stream_tiles(int n, int slots, uint32_t done0, uint32_t land0, uint32_t ready0,
                                             Issue &&issue, int tail_extra, unsigned long long limit_ns,
@@ -164,9 +174,9 @@ __device__ __forceinline__ int stream_tiles(int n, int slots, uint32_t done0, ui
     long long t_prog = cycle_now();
     bool ok = true;
     while (landed < n) {
+        const int freed = issued - slots;   // the tile that last used the next slot
         if (issued < n && issued < landed + slots &&
-            (issued < slots ||
-             mbar_test(done0 + 8u * (uint32_t)(issued % slots), (uint32_t)(((issued / slots) - 1) & 1)))) {
+            (freed < 0 || mbar_test(done0 + 8u * (uint32_t)(freed & 1), (uint32_t)((freed >> 1) & 1)))) {
             issue(issued);
             ++issued;
             t_prog = cycle_now();
@@ -176,7 +186,7 @@ __device__ __forceinline__ int stream_tiles(int n, int slots, uint32_t done0, ui
         const uint32_t lphase = (uint32_t)((landed / slots) & 1);
         if (landed < issued && mbar_test(lbar, lphase)) {
             const int n_arrive = (landed == n - 1) ? 1 + tail_extra : 1;
-            for (int a = 0; a < n_arrive; ++a) mbar_arrive(ready0 + 8u * (uint32_t)(landed % slots));
+            for (int a = 0; a < n_arrive; ++a) mbar_arrive(ready0 + 8u * (uint32_t)(landed & 1));
             ++landed;
             t_prog = cycle_now();
             continue;
@@ -197,7 +207,7 @@ __device__ __forceinline__ int stream_tiles(int n, int slots, uint32_t done0, ui
             break;
         }
         if (landed < issued) mbar_try_wait_sleep(lbar, lphase, 200u);
-        else mbar_try_wait_sleep(done0 + 8u * (uint32_t)(issued % slots), (uint32_t)(((issued / slots) - 1) & 1), 200u);
+        else mbar_try_wait_sleep(done0 + 8u * (uint32_t)(freed & 1), (uint32_t)((freed >> 1) & 1), 200u);
     }
     if (!ok)   // the copies must land before the CTA exits
         for (int v = landed; v < issued; ++v)
@@ -252,8 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(BAR(BR::QK_DONE + s), 1);
             for (int a = 0; a < 8; ++a) mbar_arrive(BAR(BR::QK_READY + s));   // pairs 0, 1: S free
         }
-        for (int s = 0; s < NSV; ++s) {
-            mbar_init(BAR(BR::V_LAND + s), 1);
+        for (int s = 0; s < NSV; ++s) mbar_init(BAR(BR::V_LAND + s), 1);
+        for (int s = 0; s < kPB; ++s) {
             mbar_init(BAR(BR::PV_READY + s), 1 + 8);   // the value loader + 4 warps for each chunk
             mbar_init(BAR(BR::PV_DONE + s), 1);
         }
@@ -417,8 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int s = 0; s < 8; ++s) dq[s] = smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024);
             for (int i = 0; ok && i < n_pairs; ++i) {
-                const uint32_t bar = keys ? BAR(BR::QK_READY + i % kSP) : BAR(BR::PV_READY + i % NSV);
-                const uint32_t phase = (uint32_t)((keys ? i / kSP : i / NSV) & 1);
+                const uint32_t bar = keys ? BAR(BR::QK_READY + i % kSP) : BAR(BR::PV_READY + i % kPB);
+                const uint32_t phase = (uint32_t)((keys ? i / kSP : i / kPB) & 1);
                 // bounded poll (a test takes ~100 cycles, so the loop costs few issue slots); the grid's
                 // status word is read only now and then
                 const long long t0 = cycle_now();
@@ -452,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     s > 0 ? 1u : 0u);
                     mma_commit(BAR(BR::QK_DONE + i % kSP));
                 } else {
-                    const uint32_t pa = tmem + kColP + (uint32_t)(i % NSV) * 64u;
+                    const uint32_t pa = tmem + kColP + (uint32_t)(i % kPB) * 64u;
                     const uint64_t dv = smem_desc_sw128(sV + (uint32_t)(i % NSV) * kPairBytes, 16384, 1024);
                     const int steps = (2 * i + 1 < n_union) ? 8 : 4;
 #pragma unroll
@@ -460,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (s < steps)
                             mma_f16_ts(tmem + kColO, pa + 8u * s, dv + (uint64_t)((2048u * s) >> 4), IDESC_PV,
                                        (i > 0 || s > 0) ? 1u : 0u);
-                    mma_commit(BAR(BR::PV_DONE + i % NSV));
+                    mma_commit(BAR(BR::PV_DONE + i % kPB));
                 }
             }
             if (ok && !keys) mma_commit(BAR(BR::O_FULL));
@@ -506,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int ptr = 0;
         bool ok = true;
         for (int t = grp; t < n_union; t += kGroups) {
-            const int pr = t >> 1, sb = pr % kSP, pb = pr % NSV;
+            const int pr = t >> 1, sb = pr % kSP, pb = pr % kPB;
             if (!warp_wait(BAR(BR::QK_DONE + sb), (uint32_t)((pr / kSP) & 1), limit_ns, abort_flag, status)) {
                 ok = false;
                 break;
@@ -533,8 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) pk[j] = 0u;
             }
-            if (pr >= NSV &&
-                !warp_wait(BAR(BR::PV_DONE + pb), (uint32_t)(((pr / NSV) - 1) & 1), limit_ns, abort_flag, status)) {
+            if (pr >= kPB &&
+                !warp_wait(BAR(BR::PV_DONE + pb), (uint32_t)(((pr / kPB) - 1) & 1), limit_ns, abort_flag, status)) {
                 ok = false;
                 break;
             }
