@@ -27,7 +27,8 @@ HILS_MAX_GROUP = 16
 EXPORTS = ("hils_status_string", "hils_version", "hils_validate", "hils_score_select_workspace_size",
            "hils_chunk_attend_fuse_workspace_size", "hils_forward_workspace_size", "hils_score_select",
            "hils_chunk_attend_fuse", "hils_forward", "hils_sync_status", "hils_set_wait_limit",
-           "hils_decode_score_select_noalloc", "hils_debug_inject_stall", "hils_landmarks")
+           "hils_decode_score_select_noalloc", "hils_debug_inject_stall", "hils_landmarks",
+           "hils_score_select_window", "hils_forward_window_workspace_size", "hils_forward_window")
 HILS_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -69,6 +70,10 @@ def _load():
     lib.hils_decode_score_select_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
     lib.hils_debug_inject_stall.argtypes = [ctypes.c_int]
     lib.hils_landmarks.argtypes = [P, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp]
+    ci = ctypes.c_int
+    lib.hils_score_select_window.argtypes = [P, ci, vp, vp, vp, vp, vp, vp]
+    lib.hils_forward_window_workspace_size.argtypes = [P, ci, ctypes.POINTER(sz)]
+    lib.hils_forward_window.argtypes = [P, ci, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for n in EXPORTS[2:]:
         if n not in ("hils_status_string", "hils_version"):
             getattr(lib, n).restype = ctypes.c_int
@@ -194,6 +199,29 @@ def hils_landmarks(p, K, U, L, beta=None, c_begin=0, c_end=None, stream=None):
         c_end = (p.T + p.C - 1) // p.C
     _check(_lib.hils_landmarks(ctypes.byref(p), _ptr(K), _ptr(U), _ptr(L), _ptr(beta), int(c_begin), int(c_end),
                                _stream(stream)), "hils_landmarks")
+
+
+def hils_score_select_window(p, window_chunks, bias, Q, L, sel_idx, sel_score, stream=None):
+    """Selection with a window of window_chunks chunks and an optional per-chunk bias [B,Hkv,nL] (float32).
+
+    sel_idx holds k + window_chunks - 1 slots per query, sel_score k + window_chunks; see include/hils.h."""
+    _check(_lib.hils_score_select_window(ctypes.byref(p), int(window_chunks), _ptr(bias), _ptr(Q), _ptr(L),
+                                         _ptr(sel_idx), _ptr(sel_score), _stream(stream)),
+           "hils_score_select_window")
+
+
+def hils_forward_window_workspace_size(p, window_chunks):
+    n = ctypes.c_size_t(0)
+    _check(_lib.hils_forward_window_workspace_size(ctypes.byref(p), int(window_chunks), ctypes.byref(n)),
+           "hils_forward_window_workspace_size")
+    return n.value
+
+
+def hils_forward_window(p, window_chunks, bias, Q, K, V, L, O, workspace=None, stream=None):
+    """The forward pass with a local window and a per-chunk bias (bias may be None)."""
+    wp, wn = _ws(workspace)
+    _check(_lib.hils_forward_window(ctypes.byref(p), int(window_chunks), _ptr(bias), _ptr(Q), _ptr(K), _ptr(V),
+                                    _ptr(L), _ptr(O), wp, wn, _stream(stream)), "hils_forward_window")
 
 
 def problem(B, H, Hkv, N, T, d, C, k, q_offset=0, in_dtype=HILS_BF16, out_dtype=None, scale=0.0):

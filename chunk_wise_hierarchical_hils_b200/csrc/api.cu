@@ -127,6 +127,20 @@ hils_status do_attend(const Dims &p, hils_dtype in, hils_dtype out, const void *
     return from_cuda(launch_attend_prefill(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
 }
 
+// The problem the chunk attention sees under a window of wc chunks: k + wc - 1 past slots per query.
+hils_status resolve_window(const hils_problem *p, int wc, Dims *base, Dims *att)
+{
+    hils_status st = resolve(p, base);
+    if (st != HILS_OK) return st;
+    if (wc < 1) return HILS_ERR_INVALID_ARG;
+    if ((long long)p->k + wc - 1 > HILS_MAX_K) return HILS_ERR_UNSUPPORTED;
+    hils_problem q = *p;
+    q.k = p->k + wc - 1;
+    return resolve(&q, att);
+}
+
+bool aligned4(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
+
 }  // namespace
 
 // Prefill dispatch: the tensor-core kernel when it covers the shape, else CUDA cores.
@@ -249,6 +263,53 @@ hils_status hils_forward(const hils_problem *p, const void *Q, const void *K, co
     st = do_select(d, p->in_dtype, Q, L, sel_idx, sel_score, scratch, s);
     if (st != HILS_OK) return st;
     return do_attend(d, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, scratch, s);
+}
+
+hils_status hils_score_select_window(const hils_problem *p, int window_chunks, const float *bias, const void *Q,
+                                     const void *L, int32_t *sel_idx, float *sel_score, void *stream)
+{
+    Dims d, da;
+    hils_status st = resolve_window(p, window_chunks, &d, &da);
+    if (st != HILS_OK) return st;
+    if (!Q || !L || !sel_score || (da.k > 0 && !sel_idx)) return HILS_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(L) || (sel_idx && !aligned16(sel_idx)) || !aligned16(sel_score) ||
+        !aligned4(bias))
+        return HILS_ERR_INVALID_ARG;
+    return from_cuda(launch_select_window(d, p->in_dtype, window_chunks, bias, Q, L, sel_idx, sel_score,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+hils_status hils_forward_window_workspace_size(const hils_problem *p, int window_chunks, size_t *bytes)
+{
+    Dims d, da;
+    if (!bytes) return HILS_ERR_INVALID_ARG;
+    hils_status st = resolve_window(p, window_chunks, &d, &da);
+    if (st != HILS_OK) return st;
+    *bytes = sel_idx_bytes(da) + sel_score_bytes(da) + attend_ws(da, p->in_dtype);
+    return HILS_OK;
+}
+
+hils_status hils_forward_window(const hils_problem *p, int window_chunks, const float *bias, const void *Q,
+                                const void *K, const void *V, const void *L, void *O, void *workspace,
+                                size_t workspace_bytes, void *stream)
+{
+    Dims d, da;
+    hils_status st = resolve_window(p, window_chunks, &d, &da);
+    if (st != HILS_OK) return st;
+    if (!Q || !K || !V || !L || !O) return HILS_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(L) || !aligned16(O) || !aligned4(bias))
+        return HILS_ERR_INVALID_ARG;
+    const size_t need = sel_idx_bytes(da) + sel_score_bytes(da) + attend_ws(da, p->in_dtype);
+    st = check_ws(workspace, workspace_bytes, need);
+    if (st != HILS_OK) return st;
+    char *ws = static_cast<char *>(workspace);
+    int32_t *sel_idx = reinterpret_cast<int32_t *>(ws);
+    float *sel_score = reinterpret_cast<float *>(ws + sel_idx_bytes(da));
+    void *scratch = ws + sel_idx_bytes(da) + sel_score_bytes(da);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = from_cuda(launch_select_window(d, p->in_dtype, window_chunks, bias, Q, L, sel_idx, sel_score, s));
+    if (st != HILS_OK) return st;
+    return do_attend(da, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, scratch, s);
 }
 
 hils_status hils_landmarks(const hils_problem *p, const void *K, const void *U, void *L, float *beta, int c_begin,

@@ -72,6 +72,11 @@ cudaError_t launch_attend_decode_mma(const Dims &p, hils_dtype out, const void *
                                      const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
                                      const DeviceCtl &ctl, cudaStream_t s);
 
+// Selection with a local window of wc chunks and an optional per-chunk bias (float [B][Hkv][nL]):
+// sel_idx rows of k + wc - 1 past slots, sel_score rows of k + wc (see select_window.cu).
+cudaError_t launch_select_window(const Dims &p, hils_dtype in, int wc, const float *bias, const void *Q,
+                                 const void *L, int32_t *sel_idx, float *sel_score, cudaStream_t s);
+
 // Landmark generation for chunks [c_begin, c_end) of every (b, g): one warp per chunk, key rows read once.
 bool landmarks_launchable(long long B, long long Hkv, int span);
 cudaError_t launch_landmarks(int B, int Hkv, int T, int d, int C, float scale, hils_dtype in, const void *K,

@@ -143,6 +143,45 @@ HILS_API hils_status hils_forward(const hils_problem *p, const void *Q, const vo
                          void *stream);
 
 /*
+ * Selection with a local window and a per-chunk bias (Sec. 2 Preliminary and
+ * Sec. 5 Small-scale Studies, "Experimental setup": a sliding-window branch
+ * keeps the recent context in every query's attention; Sec. 3 Methodology,
+ * "Linear surrogate for chunk mass": the surrogate mass adds a per-chunk bias
+ * to the query-landmark score).  Chunk-aligned reading: the window is the own
+ * chunk c_i and the window_chunks - 1 chunks before it (window_chunks >= 1,
+ * else HILS_ERR_INVALID_ARG); those are always attended and never retrieval
+ * candidates, so retrieval ranks only c <= c_i - window_chunks.  bias
+ * [B][Hkv][nL] float, device memory, 4-byte aligned, or NULL (no bias): added
+ * to every head's score of chunk c, hence to the group score and to the fusion
+ * scores.  Writes the selection in the form hils_chunk_attend_fuse reads for a
+ * problem with k' = k + window_chunks - 1 past slots (k' <= HILS_MAX_K, else
+ * HILS_ERR_UNSUPPORTED):
+ *   sel_idx   [B][Hkv][N][k']   the top-min(k, candidates) chunks in rank order
+ *                               (-1 padded to k), then the window's past chunks
+ *                               c_i - window_chunks + 1 .. c_i - 1 ascending
+ *                               (-1 below chunk 0);
+ *   sel_score [B][H][N][k' + 1] each slot's scale * <q_h, L_c> + bias_c, the own
+ *                               chunk last, -INFINITY for empty slots.
+ * window_chunks = 1 with bias NULL selects what hils_score_select selects.
+ * No workspace; Q, L, sel_idx and sel_score as for hils_score_select.
+ */
+HILS_API hils_status hils_score_select_window(const hils_problem *p, int window_chunks, const float *bias,
+                                              const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
+                                              void *stream);
+
+/*
+ * The windowed, biased forward pass: hils_score_select_window, then
+ * hils_chunk_attend_fuse on the problem with k' = k + window_chunks - 1 (the
+ * window's chunks are attended and fused like retrieved ones; the own chunk is
+ * causal).  The selection is kept in the workspace, whose size
+ * hils_forward_window_workspace_size reports.
+ */
+HILS_API hils_status hils_forward_window_workspace_size(const hils_problem *p, int window_chunks, size_t *bytes);
+HILS_API hils_status hils_forward_window(const hils_problem *p, int window_chunks, const float *bias,
+                                         const void *Q, const void *K, const void *V, const void *L, void *O,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Landmark generation (Sec. 3 Methodology, "Linear surrogate for chunk mass":
  * a landmark token appended to each chunk supplies a learned query whose
  * attention over the chunk's keys yields the chunk's compressed key).  For

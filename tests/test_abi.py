@@ -104,6 +104,43 @@ def test_landmarks_empty_range_launches_nothing():
     hils.hils_landmarks(p, 16, 16, 32, None, 2, 2, stream=0)
 
 
+@pytest.mark.parametrize("kw,wc,status", [
+    ({}, 0, hils.HILS_ERR_INVALID_ARG),                  # a window holds at least the own chunk
+    ({"k": 60}, 6, hils.HILS_ERR_UNSUPPORTED),           # k + wc - 1 = 65 past slots
+    ({"d": 96}, 2, hils.HILS_ERR_UNSUPPORTED),
+    ({"C": 48}, 2, hils.HILS_ERR_UNSUPPORTED),
+])
+def test_window_validation(kw, wc, status):
+    with pytest.raises(hils.HilsError) as e:
+        hils.hils_forward_window_workspace_size(prob(**kw), wc)
+    assert e.value.status == status
+    with pytest.raises(hils.HilsError) as e:
+        hils.hils_score_select_window(prob(**kw), wc, None, 16, 16, 16, 16, stream=0)
+    assert e.value.status == status
+
+
+def test_window_errors_before_launch():
+    p = prob()
+    with pytest.raises(hils.HilsError) as e:       # bias misaligned
+        hils.hils_score_select_window(p, 2, 18, 16, 16, 16, 16, stream=0)
+    assert e.value.status == hils.HILS_ERR_INVALID_ARG
+    with pytest.raises(hils.HilsError) as e:       # sel_idx missing while k + wc - 1 > 0
+        hils.hils_score_select_window(p, 2, None, 16, 16, None, 16, stream=0)
+    assert e.value.status == hils.HILS_ERR_INVALID_ARG
+    need = hils.hils_forward_window_workspace_size(p, 3)
+    with pytest.raises(hils.HilsError) as e:
+        hils.hils_forward_window(p, 3, None, 16, 16, 16, 16, 16, (16, need - 1), stream=0)
+    assert e.value.status == hils.HILS_ERR_WORKSPACE
+
+
+def test_window_workspace_covers_the_wider_selection():
+    # the window adds wc - 1 past slots per query: the workspace holds their indices and scores
+    p = prob()
+    one, three = hils.hils_forward_window_workspace_size(p, 1), hils.hils_forward_window_workspace_size(p, 3)
+    assert one == hils.hils_forward_workspace_size(p)
+    assert three >= one + 2 * 2 * 256 * 4 + 2 * 8 * 256 * 4 * 2
+
+
 def test_workspace_sizes():
     p = prob()
     assert hils.hils_score_select_workspace_size(p) == 0
