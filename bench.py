@@ -40,9 +40,12 @@ def parse():
     ap.add_argument("--cpu-blocks", type=int, default=16, help="64-query blocks in the oracle sample")
     ap.add_argument("--override", nargs="*", default=[], metavar="KEY=VALUE",
                     help="change workload fields, e.g. B=4 T=524288 q_offset=524287 (smaller profiling cases)")
-    ap.add_argument("--part", default="forward", choices=["forward", "landmarks"],
+    ap.add_argument("--part", default="forward", choices=["forward", "landmarks", "window"],
                     help="forward: the hot path (default); landmarks: landmark generation over the "
-                         "workload's whole key cache")
+                         "workload's whole key cache; window: the forward pass with a local window of "
+                         "--window-chunks chunks and a per-chunk bias")
+    ap.add_argument("--window-chunks", type=int, default=8,
+                    help="window of --part window in chunks (8 x 64 = a 512-token window)")
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
                     help="weak: every rank runs the whole workload; strong: the batch is split over ranks")
     return ap.parse_args()
@@ -563,6 +566,74 @@ def run_landmarks(args, w):
         dist.destroy_process_group()
 
 
+def run_window(args, w):
+    """The forward pass with a local window and a per-chunk bias (hils_forward_window), one call per step.
+
+    Algorithmic work: the attention FLOPs over k + wc slots per query (nominal, as for the plain path)."""
+    import numpy as np
+    import torch
+    import chunk_wise_hierarchical_hils_b200 as hils
+    from synth import gpu as synth_gpu
+
+    ws, rank, local = dist_setup(args)
+    wc = args.window_chunks
+    dev = synth_gpu.alloc_inputs(w)
+    dt = {"f32": hils.HILS_F32, "bf16": hils.HILS_BF16}[w.dtype]
+    p = hils.problem(w.B, w.H, w.Hkv, w.N, w.T, w.d, w.C, w.k, w.q_offset, dt, dt)
+    bias = torch.from_numpy(np.random.default_rng(w.seed + 7).standard_normal((w.B, w.Hkv, w.nL))
+                            .astype(np.float32)).cuda()
+    O = torch.empty((w.B, w.H, w.N, w.d), dtype=dev["Q"].dtype, device="cuda")
+    wsp = torch.empty(hils.hils_forward_window_workspace_size(p, wc), dtype=torch.uint8, device="cuda")
+
+    def call():
+        hils.hils_forward_window(p, wc, bias, dev["Q"], dev["K"], dev["V"], dev["L"], O, wsp)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    g_ = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_):
+        call()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    barrier(ws)
+    torch.cuda.synchronize()
+    sampler.start()
+    a_, z_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_.record(stream)
+    for _ in range(args.steps):
+        g_.replay()
+    z_.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop()
+    ms = allmax(ws, [a_.elapsed_time(z_) / args.steps])[0]
+    del g_
+    if hils.hils_sync_status() != hils.HILS_OK:
+        raise RuntimeError("device-side failure")
+    pk, pk_kind = peaks()
+    wk = w.with_(k=w.k + wc - 1)
+    fl = attention_flops(wk)
+    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    achieved = fl / (ms * 1e-3) / 1e12
+    units = w.B * w.N if w.N > 1 else w.B
+    line = {"metric": "HiLS fwd with a %d-chunk local window and chunk bias, tokens/s at 1 B200" % wc,
+            "value": ws * units / (ms * 1e-3), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded Philox4x32-10 inputs)",
+            "config": dict(config_of(w, ws), part="window", window_chunks=wc),
+            "roofline": {"bound": "tensor", "kernel": "whole step (selection + attention)", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_kind": pk_kind + " bf16 sustained", "algorithmic_flops_per_launch": fl},
+            "gpu_launches": kernels_per_step(w) * args.steps, "clocks": clocks,
+            "timing": "CUDA-graph replays of one hils_forward_window call, CUDA events on the replay stream"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     from synth.workloads import WORKLOADS
@@ -571,12 +642,14 @@ def main():
         kv = dict(x.split("=", 1) for x in args.override)
         w = w.with_(**{k: type(getattr(w, k))(v) for k, v in kv.items()})
         w = w.with_(name=w.name + "[" + ",".join(args.override) + "]")
-    if args.impl == "reference" and args.part == "landmarks":
-        raise SystemExit("--part landmarks times the library; its line carries the oracle as cpu_baseline")
+    if args.impl == "reference" and args.part != "forward":
+        raise SystemExit("--part %s times the library only; the reference arm covers the forward path" % args.part)
     if args.impl == "reference":
         run_reference(args, w)
     elif args.part == "landmarks":
         run_landmarks(args, w)
+    elif args.part == "window":
+        run_window(args, w)
     else:
         run_hils(args, w)
 
