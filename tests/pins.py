@@ -16,6 +16,10 @@ What pins what:
     causality (future rows do not matter), decode == last prefill query,
     identical heads == one head.
   * fusion weights are a distribution over the filled slots.
+  * matrix form: given only the selected chunk indices, a dense attention row
+    A_ij = w_{c(j)} * softmax over chunk c(j)'s visible keys, with the weights recomputed
+    here from the landmark scores, reproduces the output (o = A V); its rows sum to 1 and
+    it is zero outside the selected chunks' visible ranges.
 """
 import itertools
 import json
@@ -236,8 +240,50 @@ def pin_invariances():
     return fails
 
 
+def pin_matrix_form():
+    """The second, independent formulation of steps 3-6: one dense row of attention weights per
+    (b, h, i) over all T keys, built with numpy from the selection alone."""
+    fails = []
+    for (B, H, Hkv, T, d, C, k, q_offset) in [(2, 4, 2, 70, 8, 8, 3, 0), (1, 2, 1, 100, 6, 16, 2, 60)]:
+        N = T - q_offset
+        Q, K, V, L = _problem(31 + T, B, H, Hkv, T, d, C)
+        Q = Q[:, :, q_offset:]
+        scale = 1.0 / math.sqrt(d)
+        res = orc.forward(Q, K, V, L, C=C, k=k, q_offset=q_offset, scale=scale, nthreads=2)
+        G = H // Hkv
+        A = np.zeros((B, H, N, T))
+        for b in range(B):
+            for h in range(H):
+                g = h // G
+                for i in range(N):
+                    pos = q_offset + i
+                    chunks = [int(c) for c in res["sel"][b, g, i] if c >= 0]
+                    if pos // C not in chunks or len(set(chunks)) != len(chunks):
+                        fails.append("matrix form: slot list of (%d, %d, %d) is not past chunks + own" % (b, g, i))
+                        continue
+                    q = Q[b, h, i]
+                    s = np.array([scale * q @ L[b, g, c] for c in chunks])
+                    w = np.exp(s - s.max())
+                    w /= w.sum()
+                    for wc, c in zip(w, chunks):
+                        j0, j1 = c * C, min(c * C + C, pos + 1)
+                        logit = scale * K[b, g, j0:j1] @ q
+                        p = np.exp(logit - logit.max())
+                        A[b, h, i, j0:j1] = wc * p / p.sum()
+        O = np.einsum("bhit,bhtd->bhid", A, np.repeat(V, G, axis=1))
+        e = _maxerr(res["O"], O)
+        if not e <= 1e-12:
+            fails.append("matrix form B%d T%d q_offset %d: max err %.3g" % (B, T, q_offset, e))
+        if _maxerr(A.sum(axis=-1), np.ones(A.shape[:-1])) > 1e-12:
+            fails.append("matrix form: rows do not sum to 1")
+        future = np.arange(T)[None, None, None, :] > (q_offset + np.arange(N))[None, None, :, None]
+        if (A[np.broadcast_to(future, A.shape)] != 0).any():
+            fails.append("matrix form: weight on a future key")
+    return fails
+
+
 ALL_PINS = [pin_dense_reduction, pin_one_chunk, pin_hand_worked, pin_brute_force_selection,
-            pin_tie_lowest_index, pin_needle_retrieved, pin_invariances]
+            pin_tie_lowest_index, pin_needle_retrieved, pin_invariances, pin_matrix_form]
 
 
 def run_all():
