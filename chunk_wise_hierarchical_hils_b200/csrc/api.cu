@@ -85,6 +85,13 @@ bool force_cuda_cores()
     return force && strcmp(force, "simt") == 0;
 }
 
+// Debug control: HILS_CHECK_SELECTION=1 checks a caller's selection before chunk attention.
+bool check_caller_selection()
+{
+    const char *v = getenv("HILS_CHECK_SELECTION");
+    return v && strcmp(v, "1") == 0;
+}
+
 // Test control: HILS_DECODE_KERNEL=simt keeps decode attention on the CUDA-core kernel.
 bool force_decode_cuda_cores()
 {
@@ -238,6 +245,10 @@ hils_status hils_chunk_attend_fuse(const hils_problem *p, const void *Q, const v
         return HILS_ERR_INVALID_ARG;
     st = check_ws(workspace, workspace_bytes, attend_ws(d, p->in_dtype));
     if (st != HILS_OK) return st;
+    if (check_caller_selection()) {
+        st = check_selection(d, sel_idx, static_cast<cudaStream_t>(stream));
+        if (st != HILS_OK) return st;
+    }
     return do_attend(d, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, workspace,
                      static_cast<cudaStream_t>(stream));
 }

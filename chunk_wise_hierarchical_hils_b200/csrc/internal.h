@@ -77,6 +77,10 @@ cudaError_t launch_attend_decode_mma(const Dims &p, hils_dtype out, const void *
 cudaError_t launch_select_window(const Dims &p, hils_dtype in, int wc, const float *bias, const void *Q,
                                  const void *L, int32_t *sel_idx, float *sel_score, cudaStream_t s);
 
+// Debug check of a caller-supplied selection (entries -1 or past chunks of their query, no repeats in a
+// row): runs a kernel on s, waits for it and returns HILS_ERR_INVALID_ARG when a row breaks the rule.
+hils_status check_selection(const Dims &p, const int32_t *sel_idx, cudaStream_t s);
+
 // Landmark generation for chunks [c_begin, c_end) of every (b, g): one warp per chunk, key rows read once.
 bool landmarks_launchable(long long B, long long Hkv, int span);
 cudaError_t launch_landmarks(int B, int Hkv, int T, int d, int C, float scale, hils_dtype in, const void *K,

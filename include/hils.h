@@ -125,8 +125,12 @@ HILS_API hils_status hils_score_select(const hils_problem *p, const void *Q, con
  * Steps 3-4 (Abstract; Sec. 3 "Hierarchical softmax") for a given selection:
  * gathers the selected chunks' keys and values once per kv-group, attends
  * inside each, and fuses with softmax(sel_score) per head.  Writes O.
- * sel_idx entries must be -1 or a past chunk of the query (0 <= c < c_i);
- * anything else is undefined behaviour checked only by the debug build.
+ * sel_idx entries must be -1 or a past chunk of the query (0 <= c < c_i), and
+ * a row must not name a chunk twice; the kernels trust this.  With the
+ * environment variable HILS_CHECK_SELECTION=1 (a debug aid) the call first
+ * checks every row on the GPU, waits for the verdict (synchronising `stream`)
+ * and returns HILS_ERR_INVALID_ARG, launching nothing else, when a row breaks
+ * the rule.
  */
 HILS_API hils_status hils_chunk_attend_fuse(const hils_problem *p, const void *Q, const void *K,
                                    const void *V, const int32_t *sel_idx,
