@@ -214,7 +214,7 @@ def shard_batch(B, world, rank):
 def cpu_baseline(w, n_blocks, block=64, seed=5):
     """The float64 oracle on a bounded sample: n_blocks blocks of `block` consecutive queries of batch 0.
 
-    Returns (value in the workload's unit, cores, description)."""
+    Returns (value in the workload's unit, cores, description, seconds of oracle time)."""
     import numpy as np
     from oracle import oracle as orc
     from synth import workloads as W
@@ -250,7 +250,7 @@ def cpu_baseline(w, n_blocks, block=64, seed=5):
         per_group_bytes = decode_bytes(w) / (w.B * w.Hkv)
         return (per_group_bytes * len(items) / t / 1e9, 1,
                 "%d of %d decode query groups (b, kv-head), one thread each, host input generation untimed"
-                % (len(items), w.B * w.Hkv))
+                % (len(items), w.B * w.Hkv), t)
     b = 0
     K = np.stack([W.k_rows(w, b, g, 0, w.T)[0] for g in range(w.Hkv)])[None]
     V = np.stack([W.v_rows(w, b, g, 0, w.T)[0] for g in range(w.Hkv)])[None]
@@ -265,7 +265,7 @@ def cpu_baseline(w, n_blocks, block=64, seed=5):
         t += time.perf_counter() - t0
         ntok += block
     return (ntok / t, cores, "%d blocks of %d consecutive queries (all %d heads) of batch 0 at random offsets; "
-            "OpenMP over query groups; host input generation untimed" % (len(starts), block, w.H))
+            "OpenMP over query groups; host input generation untimed" % (len(starts), block, w.H), t)
 
 
 def run_reference(args, w):
@@ -273,14 +273,16 @@ def run_reference(args, w):
     if rank != 0:
         return
     unit = "tokens/s" if w.N > 1 else "GB/s"
-    vals = []
+    vals, secs = [], []
     for s in range(args.warmup + args.steps):
-        v, cores, desc = cpu_baseline(w, n_blocks=2, seed=100 + s)
+        v, cores, desc, t = cpu_baseline(w, n_blocks=2, seed=100 + s)
         if s >= args.warmup:
             vals.append(v)
+            secs.append(t)
     value = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc},
@@ -455,7 +457,7 @@ def run_hils(args, w):
             "gpu_launches": kernels_per_step(w) * args.steps, "clocks": clocks,
             "timing": "CUDA-graph replays of the library calls, CUDA events on the replay stream"}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        v, cores, desc = cpu_baseline(w, args.cpu_blocks)
+        v, cores, desc, _ = cpu_baseline(w, args.cpu_blocks)
         line["cpu_baseline"] = {"value": v, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -65,3 +65,28 @@ def test_traffic_only_for_the_captured_sources(tmp_path, text, workload, expect)
     b.ROOT = str(_fake_tree(tmp_path, text))
     assert b.kernel_traffic("kern", workload) == expect
     assert b.kernel_traffic("missing", workload) is None
+
+
+@pytest.mark.parametrize("workload", ["tiny_f32", "decode_128k"])
+def test_reference_arm_prints_one_contract_line(workload):
+    """bench.py --impl reference times the oracle on the host (no GPU) and prints one JSON line with the
+    contract's keys; for the small case the whole run takes seconds."""
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", "--workload", workload], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    line = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["config"]["workload"] == workload
+    assert line["value"] > 0 and line["ms_per_step"] > 0 and line["steps"] == 1
+    assert line["unit"] == ("GB/s" if workload.startswith("decode") else "tokens/s")
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
