@@ -70,7 +70,7 @@
 extern "C" {
 #endif
 
-#define HILS_VERSION 100    /* 1.0.0 */
+#define HILS_VERSION 110    /* 1.1.0: adds the window/bias selection and forward, and landmark generation */
 #define HILS_MAX_K 64       /* largest supported top-k */
 #define HILS_MAX_GROUP 16   /* largest supported H / Hkv */
 

@@ -22,7 +22,7 @@ def test_header_symbols_exported():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) <= set(hils.EXPORTS) | set(names)
-    assert hils.hils_version() == 100
+    assert hils.hils_version() == 110
 
 
 def test_struct_layout_matches_header():
