@@ -179,4 +179,4 @@ def test_header_is_plain_c_and_links(tmp_path):
     subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
                            "-L", libdir, "-lhils", "-Wl,-rpath," + libdir, "-o", str(exe)])
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
-    assert out[0] == "100"
+    assert out[0] == "110"
