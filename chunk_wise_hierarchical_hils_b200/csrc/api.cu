@@ -5,6 +5,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "next_rows.h"
 
 namespace hils {
 

@@ -6,6 +6,7 @@
 // with the check switched on the library first runs this kernel, reads its verdict and refuses the
 // call (nothing else launched) when any row breaks the rule.
 #include "common.cuh"
+#include "next_rows.h"
 
 namespace hils {
 namespace {

@@ -21,6 +21,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "next_rows.h"
 
 namespace hils {
 

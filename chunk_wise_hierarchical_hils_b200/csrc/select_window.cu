@@ -21,6 +21,7 @@
 // block per (b, g); each thread keeps a heap over a strided share of the candidates, and the block's
 // radix top-k merges the heaps.
 #include "common.cuh"
+#include "next_rows.h"
 
 namespace hils {
 namespace {
