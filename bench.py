@@ -513,8 +513,13 @@ def run_landmarks(args, w):
         raise RuntimeError("device-side failure")
 
     # end to end: keys and landmark queries from pinned host memory, landmarks and biases back
-    Kh, Uh = K.cpu().pin_memory(), U.cpu().pin_memory()
-    Lh, bh = torch.empty(Lout.shape, dtype=Lout.dtype).pin_memory(), torch.empty(beta.shape).pin_memory()
+    # pinned buffers allocated directly (a 4M-token key cache is 8.6 GB: no pageable intermediate copy)
+    Kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
+    Uh = torch.empty(U.shape, dtype=U.dtype, pin_memory=True)
+    Kh.copy_(K)
+    Uh.copy_(U)
+    Lh = torch.empty(Lout.shape, dtype=Lout.dtype, pin_memory=True)
+    bh = torch.empty(beta.shape, dtype=beta.dtype, pin_memory=True)
 
     def e2e_step():
         K.copy_(Kh, non_blocking=True)
