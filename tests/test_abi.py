@@ -141,6 +141,19 @@ def test_window_workspace_covers_the_wider_selection():
     assert three >= one + 2 * 2 * 256 * 4 + 2 * 8 * 256 * 4 * 2
 
 
+@pytest.mark.parametrize("kw", [dict(), dict(N=1, T=131072, q_offset=131071, B=4, H=32, Hkv=8, k=32)])
+def test_window_workspace_is_the_attention_of_the_wider_selection(kw):
+    # hils_forward_window = window selection (no scratch) + hils_chunk_attend_fuse on k' = k + wc - 1 slots:
+    # its workspace holds sel_idx [.., k'] and sel_score [.., k' + 1] (256-byte aligned) and the attention's
+    p = prob(**kw)
+    wc = 4
+    pk = prob(**dict(kw, k=p.k + wc - 1))
+    B, H, Hkv, N, kp = p.B, p.H, p.Hkv, p.N, p.k + wc - 1
+    up = lambda x: (x + 255) // 256 * 256
+    want = up(B * Hkv * N * kp * 4) + up(B * H * N * (kp + 1) * 4) + hils.hils_chunk_attend_fuse_workspace_size(pk)
+    assert hils.hils_forward_window_workspace_size(p, wc) == want
+
+
 def test_workspace_sizes():
     p = prob()
     assert hils.hils_score_select_workspace_size(p) == 0
