@@ -466,6 +466,35 @@ def run_hils(args, w):
         dist.destroy_process_group()
 
 
+def timed_graph_replays(call, args, ws, local):
+    """Warm up `call`, capture it in a CUDA graph and time args.steps replays with CUDA events on the
+    replay stream, barriers and clock sampling around them.  Returns (ms per replay, max over ranks;
+    clock record)."""
+    import torch
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    barrier(ws)
+    torch.cuda.synchronize()
+    sampler.start()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop()
+    ms = allmax(ws, [start.elapsed_time(end) / args.steps])[0]
+    del graph
+    return ms, clocks
+
+
 def run_landmarks(args, w):
     """Landmark generation (hils_landmarks) over the workload's whole key cache, one call per step.
 
@@ -488,29 +517,10 @@ def run_landmarks(args, w):
     def call():
         hils.hils_landmarks(p, K, U, Lout, beta)
 
-    for _ in range(args.warmup):
-        call()
-    torch.cuda.synchronize()
-    g_ = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_):
-        call()
-    stream = torch.cuda.current_stream()
-    sampler = ClockSampler(local)
-    barrier(ws)
-    torch.cuda.synchronize()
-    sampler.start()
-    a_, z_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a_.record(stream)
-    for _ in range(args.steps):
-        g_.replay()
-    z_.record(stream)
-    torch.cuda.synchronize()
-    barrier(ws)
-    clocks = sampler.stop()
-    ms = allmax(ws, [a_.elapsed_time(z_) / args.steps])[0]
-    del g_
+    ms, clocks = timed_graph_replays(call, args, ws, local)
     if hils.hils_sync_status() != hils.HILS_OK:
         raise RuntimeError("device-side failure")
+    stream = torch.cuda.current_stream()
 
     # end to end: keys and landmark queries from pinned host memory, landmarks and biases back
     # pinned buffers allocated directly (a 4M-token key cache is 8.6 GB: no pageable intermediate copy)
@@ -595,27 +605,7 @@ def run_window(args, w):
     def call():
         hils.hils_forward_window(p, wc, bias, dev["Q"], dev["K"], dev["V"], dev["L"], O, wsp)
 
-    for _ in range(args.warmup):
-        call()
-    torch.cuda.synchronize()
-    g_ = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_):
-        call()
-    stream = torch.cuda.current_stream()
-    sampler = ClockSampler(local)
-    barrier(ws)
-    torch.cuda.synchronize()
-    sampler.start()
-    a_, z_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a_.record(stream)
-    for _ in range(args.steps):
-        g_.replay()
-    z_.record(stream)
-    torch.cuda.synchronize()
-    barrier(ws)
-    clocks = sampler.stop()
-    ms = allmax(ws, [a_.elapsed_time(z_) / args.steps])[0]
-    del g_
+    ms, clocks = timed_graph_replays(call, args, ws, local)
     if hils.hils_sync_status() != hils.HILS_OK:
         raise RuntimeError("device-side failure")
     pk, pk_kind = peaks()
