@@ -42,6 +42,8 @@ namespace {
 
 bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
+}  // namespace
+
 hils_status resolve(const hils_problem *p, Dims *o)
 {
     if (!p) return HILS_ERR_INVALID_ARG;
@@ -67,6 +69,8 @@ hils_status resolve(const hils_problem *p, Dims *o)
     if (o->N == 1 && decode_select_smem_bytes(*o, p->in_dtype) > 200 * 1024) return HILS_ERR_UNSUPPORTED;
     return HILS_OK;
 }
+
+namespace {
 
 size_t sel_idx_bytes(const Dims &p) { return align_up((size_t)p.B * p.Hkv * p.N * p.k * sizeof(int32_t), 256); }
 size_t sel_score_bytes(const Dims &p) { return align_up((size_t)p.B * p.H * p.N * (p.k + 1) * sizeof(float), 256); }

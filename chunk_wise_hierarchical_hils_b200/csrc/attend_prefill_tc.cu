@@ -21,8 +21,8 @@
 //                        shared memory) on two chunks at once (N = 128, the
 //                        tensor core's efficient width) into one of two TMEM
 //                        S buffers;
-//   warp 3 (one thread)  tcgen05.mma issue of O += P V (f16, P from TMEM, V
-//                        from shared memory) on the same pairs (K = 128 keys);
+//   warp 3 (one thread)  tcgen05.mma issue of O += P V (f16 or bf16, P from
+//                        TMEM, V from shared memory) on the same pairs (K = 128 keys);
 //                        two issuers keep the tensor core busy while either
 //                        one waits;
 //   warps 4..15          three groups of four warps, one thread per row; group
@@ -30,12 +30,21 @@
 //                        the S buffer at once), takes the softmax over the
 //                        chunk's visible keys, scales it by the row's fusion
 //                        weight (0 if the row's query did not select the chunk)
-//                        and writes P (f16) to its half of a TMEM P buffer.  At
+//                        and writes P (16-bit) to its half of a TMEM P buffer.  At
 //                        the end the groups read O from TMEM and store it.
 // Because each chunk's softmax is normalised on its own and the fusion weights
 // are known before the loop, P already carries w_c / l_c and the accumulator
-// needs no rescaling between chunks.  V is read as f16 (converted once per call
-// by a streaming pass), so P can be kept in f16 with a 2^-11 rounding.
+// needs no rescaling between chunks.
+//
+// Value product precision.  The definition holds for any finite input, and V
+// enters the product exactly in both of two forms.  A streaming pass converts V
+// to f16 once per call and flags every (b, kv-head) slice holding a value of
+// magnitude >= 65536, where f16 overflows (every bf16 value below that is
+// exact in f16; the few below 2^-14 become f16 subnormals, within 2^-25).  A
+// block of an unflagged slice reads the f16 copy and rounds P to f16 (relative
+// 2^-11); a block of a flagged slice reads V as given and rounds P to bf16
+// (relative 2^-8).  The output error from rounding P is at most that relative
+// error times the largest |v| the row attends to (the row's P sums to one).
 //
 // Every barrier wait is bounded: on expiry the CTA records HILS_ERR_TIMEOUT,
 // stops issuing work, waits (with its own bound) for the copies and MMAs it has
@@ -68,6 +77,7 @@ constexpr int kPolyPairEvery = 4; // exponential pairs computed by exp2_poly_x2:
 constexpr uint32_t IDESC_QK2 = idesc_bf16_f32(128, 128, false, false);  // S = Q K^T over two chunks, K-major
 constexpr uint32_t IDESC_QK1 = idesc_bf16_f32(128, 64, false, false);   // the same for a lone last chunk
 constexpr uint32_t IDESC_PV = idesc_f16_f32(128, 128, false, true);    // O += P V, f16, V MN-major
+constexpr uint32_t IDESC_PV_BF16 = idesc_bf16_f32(128, 128, false, true);   // the same in bf16 (wide slices)
 
 struct Layout {
     uint32_t q, k, v, bar, misc, bitmap, uni, selbuf, scbuf, qlist, qslot, qcnt, wts, total;
@@ -218,8 +228,9 @@ __device__ __forceinline__ int stream_tiles(int n, int slots, uint32_t done0, ui
 template <int G, typename Tout, int NSV>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, Dims p, const int32_t *__restrict__ sel_idx,
-                     const float *__restrict__ sel_score, Tout *__restrict__ O, unsigned int *status,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmVb, Dims p,
+                     const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_score,
+                     const unsigned int *__restrict__ wide_flags, Tout *__restrict__ O, unsigned int *status,
                      unsigned long long limit_ns, int nwords, int inject_stall)
 {
     constexpr int BQ = kRows / G;
@@ -234,6 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q0 = (int)(gridDim.x - 1 - blockIdx.x) * BQ, g = blockIdx.y, b = blockIdx.z;
     const int nq = min(BQ, p.N - q0);
     const int ns = p.k + 1;
+    // a slice whose values overflow f16 takes the bf16 value product (V as given, P in bf16)
+    const bool wide = __ldg(wide_flags + b * p.Hkv + g) != 0u;
+    const CUtensorMap *tmVsel = wide ? &tmVb : &tmV;
 
     const uint32_t sQ = smem_addr(base + Ly.q), sK = smem_addr(base + Ly.k), sV = smem_addr(base + Ly.v);
     const uint32_t bar0 = smem_addr(base + Ly.bar);
@@ -274,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
+        prefetch_tensormap(tmVsel);
         mbar_arrive_expect_tx(BAR(BR::Q_FULL), 32768u);
         tma_load_3d(sQ, &tmQ, BAR(BR::Q_FULL), 0, b * p.H + g * G, q0);
         tma_load_3d(sQ + 16384u, &tmQ, BAR(BR::Q_FULL), 64, b * p.H + g * G, q0);
@@ -395,12 +409,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dst = sV + (uint32_t)st * kPairBytes;
                 mbar_arrive_expect_tx(BAR(BR::V_LAND + st), two ? 32768u : 16384u);
                 const int row0 = kv_row0 + uni[2 * pr] * kChunk;
-                tma_load_2d(dst, &tmV, BAR(BR::V_LAND + st), 0, row0);
-                tma_load_2d(dst + 16384u, &tmV, BAR(BR::V_LAND + st), 64, row0);
+                tma_load_2d(dst, tmVsel, BAR(BR::V_LAND + st), 0, row0);
+                tma_load_2d(dst + 16384u, tmVsel, BAR(BR::V_LAND + st), 64, row0);
                 if (two) {
                     const int row1 = kv_row0 + uni[2 * pr + 1] * kChunk;
-                    tma_load_2d(dst + 8192u, &tmV, BAR(BR::V_LAND + st), 0, row1);
-                    tma_load_2d(dst + 24576u, &tmV, BAR(BR::V_LAND + st), 64, row1);
+                    tma_load_2d(dst + 8192u, tmVsel, BAR(BR::V_LAND + st), 0, row1);
+                    tma_load_2d(dst + 24576u, tmVsel, BAR(BR::V_LAND + st), 64, row1);
                 }
             };
             // a lone last chunk has no second softmax group to announce its P: the loader stands in
@@ -416,6 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const bool keys = (warp == 2);
             const int n_pairs = (n_union + 1) >> 1;
+            const uint32_t idesc_pv = wide ? IDESC_PV_BF16 : IDESC_PV;
             bool ok = true;
             if (keys && inject_stall) {
                 // test control: wait once on a barrier nothing signals, so the bounded wait expires
@@ -468,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int s = 0; s < 8; ++s)
                         if (s < steps)
-                            mma_f16_ts(tmem + kColO, pa + 8u * s, dv + (uint64_t)((2048u * s) >> 4), IDESC_PV,
+                            mma_f16_ts(tmem + kColO, pa + 8u * s, dv + (uint64_t)((2048u * s) >> 4), idesc_pv,
                                        (i > 0 || s > 0) ? 1u : 0u);
                     mma_commit(BAR(BR::PV_DONE + i % kPB));
                 }
@@ -538,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[32];
             if (__any_sync(0xFFFFFFFFu, w > 0.f)) {   // rows with w = 0 get P = 0 from the scaling
                 const int n_vis = (c == own) ? (int)(pos - (long long)c * kChunk + 1) : kChunk;
-                chunk_softmax_row<kPolyPairEvery>(sv, n_vis, w, sl2, pk);
+                chunk_softmax_row<kPolyPairEvery>(sv, n_vis, w, sl2, pk, wide);
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) pk[j] = 0u;
@@ -607,18 +622,26 @@ bool encode(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, int rank, c
     return r == CUDA_SUCCESS;
 }
 
-// V (bf16) -> f16, 8 elements per 16-byte vector; exact for |v| < 65504.
-__global__ void v_to_f16_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, size_t n)
+// V (bf16) -> f16, 8 elements per 16-byte vector.  Every bf16 value of magnitude below 65536 is
+// exact in f16 (below 2^-14 as an f16 subnormal, within 2^-25); a vector holding a larger one
+// raises the flag of its (b, kv-head) slice (vec_per_slice vectors each), and the attention blocks
+// of a flagged slice read V as given instead of this copy.  The flags start at zero.
+__global__ void v_to_f16_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, size_t n,
+                                size_t vec_per_slice, unsigned int *__restrict__ wide_flags)
 {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
         const uint4 u = __ldg(in + i);
         uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        bool big = false;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+            // bf16 magnitude bits >= 0x4780 means |v| >= 2^16 (or not finite)
+            big |= (w[e] & 0x7FFFu) >= 0x4780u || ((w[e] >> 16) & 0x7FFFu) >= 0x4780u;
             __half2 h2 = __floats2half2_rn(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
             w[e] = *reinterpret_cast<uint32_t *>(&h2);
         }
         out[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        if (big) atomicOr(wide_flags + i / vec_per_slice, 1u);
     }
 }
 
@@ -634,11 +657,12 @@ int ring_config(int k, int nwords, int BQ)
 }
 
 template <int G, typename Tout>
-cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V, const int32_t *sel_idx,
-                     const float *sel_score, void *O, const DeviceCtl &ctl, cudaStream_t s)
+cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V16, const void *V,
+                     const unsigned int *wide_flags, const int32_t *sel_idx, const float *sel_score, void *O,
+                     const DeviceCtl &ctl, cudaStream_t s)
 {
     constexpr int BQ = kRows / G;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tvb;
     // Q viewed as (d, head, query): a box of G heads x BQ queries lands query-major, row = query * G + head
     const cuuint64_t qd[3] = {(cuuint64_t)kD, (cuuint64_t)p.B * p.H, (cuuint64_t)p.N};
     const cuuint64_t qs[2] = {(cuuint64_t)p.N * kD * 2, (cuuint64_t)kD * 2};
@@ -648,7 +672,8 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V,
     const cuuint32_t kb[2] = {64, (cuuint32_t)kChunk};
     if (!encode(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, 3, qd, qs, qb) ||
         !encode(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, 2, kd, ks, kb) ||
-        !encode(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, V, 2, kd, ks, kb))
+        !encode(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, V16, 2, kd, ks, kb) ||
+        !encode(&tvb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, 2, kd, ks, kb))
         return cudaErrorInvalidValue;
     const int c_max = (int)(((long long)p.q_offset + p.N - 1) / kChunk);
     const int nwords = c_max / 32 + 1;
@@ -661,7 +686,8 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V,
         auto kern = attend_tc_kernel<G, Tout, NV>;                                                          \
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);              \
         if (e != cudaSuccess) return e;                                                                      \
-        kern<<<grid, kThreads, smem, s>>>(tq, tk, tv, p, sel_idx, sel_score, static_cast<Tout *>(O),         \
+        kern<<<grid, kThreads, smem, s>>>(tq, tk, tv, tvb, p, sel_idx, sel_score, wide_flags,                 \
+                                          static_cast<Tout *>(O),                                            \
                                           ctl.status, (unsigned long long)ctl.wait_limit, nwords,            \
                                           ctl.inject_stall);                                                 \
     }
@@ -672,17 +698,20 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *K, const void *V,
 }
 
 template <typename Tout>
-cudaError_t launch_o(const Dims &p, const void *Q, const void *K, const void *V, const int32_t *sel_idx,
-                     const float *sel_score, void *O, const DeviceCtl &ctl, cudaStream_t s)
+cudaError_t launch_o(const Dims &p, const void *Q, const void *K, const void *V16, const void *V,
+                     const unsigned int *wf, const int32_t *sel_idx, const float *sel_score, void *O,
+                     const DeviceCtl &ctl, cudaStream_t s)
 {
     switch (p.G) {
-    case 1: return launch_g<1, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
-    case 2: return launch_g<2, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
-    case 4: return launch_g<4, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
-    case 8: return launch_g<8, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
-    default: return launch_g<16, Tout>(p, Q, K, V, sel_idx, sel_score, O, ctl, s);
+    case 1: return launch_g<1, Tout>(p, Q, K, V16, V, wf, sel_idx, sel_score, O, ctl, s);
+    case 2: return launch_g<2, Tout>(p, Q, K, V16, V, wf, sel_idx, sel_score, O, ctl, s);
+    case 4: return launch_g<4, Tout>(p, Q, K, V16, V, wf, sel_idx, sel_score, O, ctl, s);
+    case 8: return launch_g<8, Tout>(p, Q, K, V16, V, wf, sel_idx, sel_score, O, ctl, s);
+    default: return launch_g<16, Tout>(p, Q, K, V16, V, wf, sel_idx, sel_score, O, ctl, s);
     }
 }
+
+size_t v16_bytes(const Dims &p) { return align_up((size_t)p.B * p.Hkv * p.T * kD * 2, 256); }
 
 }  // namespace
 
@@ -695,9 +724,10 @@ bool attend_tc_supported(const Dims &p, hils_dtype in)
     return ring_config(p.k, c_max / 32 + 1, kRows / p.G) >= 0;
 }
 
+// V as f16, then one flag word per (b, kv-head) slice
 size_t attend_tc_ws_bytes(const Dims &p)
 {
-    return align_up((size_t)p.B * p.Hkv * p.T * kD * 2, 256);   // V as f16
+    return v16_bytes(p) + align_up((size_t)p.B * p.Hkv * sizeof(unsigned int), 256);
 }
 
 cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
@@ -705,11 +735,15 @@ cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *
                                      const DeviceCtl &ctl, cudaStream_t s)
 {
     const size_t n16 = (size_t)p.B * p.Hkv * p.T * kD / 8;
-    v_to_f16_kernel<<<148 * 8, 256, 0, s>>>(static_cast<const uint4 *>(V), static_cast<uint4 *>(ws), n16);
-    cudaError_t e = cudaGetLastError();
+    unsigned int *wide = reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + v16_bytes(p));
+    cudaError_t e = cudaMemsetAsync(wide, 0, (size_t)p.B * p.Hkv * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
-    if (out == HILS_F32) return launch_o<float>(p, Q, K, ws, sel_idx, sel_score, O, ctl, s);
-    return launch_o<__nv_bfloat16>(p, Q, K, ws, sel_idx, sel_score, O, ctl, s);
+    v_to_f16_kernel<<<148 * 8, 256, 0, s>>>(static_cast<const uint4 *>(V), static_cast<uint4 *>(ws), n16,
+                                            (size_t)p.T * kD / 8, wide);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (out == HILS_F32) return launch_o<float>(p, Q, K, ws, V, wide, sel_idx, sel_score, O, ctl, s);
+    return launch_o<__nv_bfloat16>(p, Q, K, ws, V, wide, sel_idx, sel_score, O, ctl, s);
 }
 
 }  // namespace hils

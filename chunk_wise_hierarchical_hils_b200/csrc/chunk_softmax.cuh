@@ -5,10 +5,12 @@
 // see; the chunk's result enters the output with the row's fusion weight w.  Both factors are
 // applied here, so P = w * softmax(s[0 .. n_vis)) with P = 0 for masked keys.
 //
-// sv holds the row's 64 raw scores q.k (float bits) and is overwritten; pk receives P as 32 f16
-// pairs (key 2j in the low half).  sl2 = scale * log2(e), so exp(scale (s - m)) = 2^(sl2 s - sl2 m).
+// sv holds the row's 64 raw scores q.k (float bits) and is overwritten; pk receives P as 32 pairs of
+// 16-bit values (key 2j in the low half): f16, or bf16 when p_bf16 is set (the caller's value tiles
+// are then bf16 too).  sl2 = scale * log2(e), so exp(scale (s - m)) = 2^(sl2 s - sl2 m).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -20,7 +22,7 @@ namespace hils {
 // (exp2_poly_x2), the rest on the special-function unit.  POLY_PAIR_EVERY = 0: all on the latter.
 template <int POLY_PAIR_EVERY>
 __device__ __forceinline__ void chunk_softmax_row(uint32_t (&sv)[64], int n_vis, float w, float sl2,
-                                                  uint32_t (&pk)[32])
+                                                  uint32_t (&pk)[32], bool p_bf16 = false)
 {
     using namespace sm100;
     if (n_vis < 64) {
@@ -60,12 +62,22 @@ __device__ __forceinline__ void chunk_softmax_row(uint32_t (&sv)[64], int n_vis,
     float l0, l1;
     f2_unpack(f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3])), l0, l1);
     const uint64_t f = f2_splat(__fdividef(w, l0 + l1));
+    if (p_bf16) {   // uniform over the block: one branch around the packing loop
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        float a0, a1;
-        f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), f), a0, a1);
-        __half2 v2 = __floats2half2_rn(a0, a1);
-        pk[j] = *reinterpret_cast<uint32_t *>(&v2);
+        for (int j = 0; j < 32; ++j) {
+            float a0, a1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), f), a0, a1);
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(a0, a1);
+            pk[j] = *reinterpret_cast<uint32_t *>(&v2);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            float a0, a1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), f), a0, a1);
+            __half2 v2 = __floats2half2_rn(a0, a1);
+            pk[j] = *reinterpret_cast<uint32_t *>(&v2);
+        }
     }
 }
 

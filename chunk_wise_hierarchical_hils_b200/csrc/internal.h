@@ -19,6 +19,9 @@ struct Dims {
     float scale;     // resolved: never 0
 };
 
+// Checks a problem description and derives its quantities (the validation of every entry point).
+hils_status resolve(const hils_problem *p, Dims *o);
+
 // Device-side status shared by all kernels of the library.
 struct DeviceCtl {
     unsigned int *status;   // HILS_OK or HILS_ERR_TIMEOUT, sticky until read

@@ -11,11 +11,14 @@
 // lists and the completion tickets) from a fixed array that lives in the
 // library's own device memory instead of a caller workspace.
 //
-// The array below is a host-side stand-in in host code: it must never be passed
-// to a kernel directly.  Its device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, on the first call made on the
-// device.  Every GPU that loads the library holds the array until the process
-// exits.
+// The array below is a __device__ variable.  Host code that names
+// g_noalloc_scratch sees only the runtime's host-side shadow of it, not a device
+// address, so the name is never passed to a kernel: the device address comes
+// from cudaGetSymbolAddress, looked up once per device, with that device
+// current, on the first call made on the device, and cached.  A device reset
+// (cudaDeviceReset) ends the context that address belongs to; calls after one
+// are not supported.  Every GPU that loads the library holds the array until the
+// process exits.
 #include <math.h>
 #include <mutex>
 
@@ -58,7 +61,8 @@ using namespace hils;
 extern "C" hils_status hils_decode_score_select_noalloc(const hils_problem *p, const void *Q, const void *L,
                                                         int32_t *sel_idx, float *sel_score, void *stream)
 {
-    hils_status st = hils_validate(p);
+    Dims d;
+    hils_status st = resolve(p, &d);
     if (st != HILS_OK) return st;
     if (p->N != 1) return HILS_ERR_UNSUPPORTED;   // only the single-token decode kernel needs scratch
     if (!Q || !L || !sel_score || (p->k > 0 && !sel_idx)) return HILS_ERR_INVALID_ARG;
@@ -71,12 +75,6 @@ extern "C" hils_status hils_decode_score_select_noalloc(const hils_problem *p, c
     void *scratch = nullptr;
     st = scratch_on_current_device(&scratch);
     if (st != HILS_OK) return st;
-    Dims d;
-    d.B = p->B; d.H = p->H; d.Hkv = p->Hkv; d.G = p->H / p->Hkv;
-    d.N = p->N; d.T = p->T; d.d = p->d; d.C = p->C; d.k = p->k;
-    d.nL = (p->T + p->C - 1) / p->C;
-    d.q_offset = p->q_offset;
-    d.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
     DeviceCtl ctl;
     st = device_ctl(&ctl);
     if (st != HILS_OK) return st;

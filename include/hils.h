@@ -48,6 +48,10 @@
  * failures of bounded waits are reported by hils_sync_status().
  * Thread safety: calls may come from several host threads; kernels that share
  * one workspace must not overlap on the GPU.
+ * Device state: the library looks up the device addresses of its own device
+ * variables (a status word, and the scratch array of the allocation-free entry
+ * point) once per device and caches them; a cudaDeviceReset ends the context
+ * they belong to, and calls after one are not supported.
  * Kernel choice: the tensor-core kernels run whenever they cover the problem
  * (bf16 inputs, d = 128; prefill C = 64; decode C in {64, 128}), the CUDA-core
  * kernels otherwise.  As a test control, the environment variables
@@ -131,6 +135,14 @@ HILS_API hils_status hils_score_select(const hils_problem *p, const void *Q, con
  * checks every row on the GPU, waits for the verdict (synchronising `stream`)
  * and returns HILS_ERR_INVALID_ARG, launching nothing else, when a row breaks
  * the rule.
+ * Precision: every product accumulates in float32, and the result is defined
+ * for every finite input.  On the bf16 tensor-core prefill kernel the
+ * probabilities that multiply V are rounded to 16 bits while V enters exactly:
+ * to f16 (relative error 2^-11) for a (b, kv-head) whose values all have
+ * magnitude below 65536 (V is converted to f16 in the workspace; values below
+ * 2^-14 become f16 subnormals, within 2^-25), and to bf16 (2^-9) otherwise,
+ * with V read as given.  The output error from this rounding is at most that
+ * relative error times the largest |v| the query attends to.
  */
 HILS_API hils_status hils_chunk_attend_fuse(const hils_problem *p, const void *Q, const void *K,
                                    const void *V, const int32_t *sel_idx,

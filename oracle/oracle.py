@@ -52,6 +52,10 @@ def lib():
                                                                       _D, _D, _D, _I, _D, _D, ctypes.c_int]
         L.hils_oracle_forward_window.restype = ctypes.c_int
         L.hils_oracle_landmarks.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, _D, _D, _D]
+        L.hils_oracle_select_window.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_long, ctypes.c_double, _D, _D, _D, _I, _D]
+        L.hils_oracle_attend_slots.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_long,
+                                               ctypes.c_double, _D, _I, _D, _D, _D, _D, _D, _D, _D]
         L.hils_oracle_max_threads.restype = ctypes.c_int
     return _lib
 
@@ -199,6 +203,26 @@ def attend(q, sel, Lsel, Ksel, Vsel, C, pos, scale, want_chunks=False):
     if want_chunks:
         out["oc"] = oc
     return out
+
+
+def attend_slots(q, sel, Lsel, bsel, Ksel, Vsel, C, pos, scale):
+    """Attention inside the given slots and their fusion, for one query group (the windowed form).
+
+    q [G,d]; sel [ns] chunk per slot (-1 empty); Lsel [ns,d]; bsel [ns] slot biases or None;
+    Ksel/Vsel [ns,C,d].  Returns dict s, w [G,ns], o [G,d] with s = scale q.L_c + bias_c."""
+    q = _f64(q)
+    G, d = q.shape
+    ns = len(sel)
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    Lsel, Ksel, Vsel = _f64(Lsel), _f64(Ksel), _f64(Vsel)
+    assert Ksel.shape == (ns, C, d) and Vsel.shape == (ns, C, d) and Lsel.shape == (ns, d)
+    bsel = _f64(bsel) if bsel is not None else None
+    s = np.zeros((G, ns))
+    w = np.zeros((G, ns))
+    o = np.zeros((G, d))
+    lib().hils_oracle_attend_slots(G, d, C, ns, pos, scale, _dp(q), _ip(sel), _dp(Lsel), _dp(bsel), _dp(Ksel),
+                                   _dp(Vsel), _dp(s), _dp(w), _dp(o))
+    return {"s": s, "w": w, "o": o}
 
 
 def tie_alternatives(shat, n_past, k, eps, max_alts=64):

@@ -80,9 +80,12 @@ def gather_gpu(w, O, sel_idx, sel_score, items):
 
 
 def compare(w, items, answers, sel, s, o, tol_o=None, tol_s=TOL_S, out_dtype="f32"):
-    """Check every sampled query group; returns a stats dict (failures listed in stats['fail'])."""
+    """Check every sampled query group; returns a stats dict (failures listed in stats['fail']).
+
+    tol_o: the output bound, one number for every item or a sequence with one per item."""
     if tol_o is None:
         tol_o = TOL_O[w.dtype]
+    tol_items = list(tol_o) if np.ndim(tol_o) else [tol_o] * len(items)
     st = {"n": len(items), "near_tie": 0, "overflow": 0, "max_err_O": 0.0, "max_err_s": 0.0, "fail": []}
     for n, (it, ans) in enumerate(zip(items, answers)):
         pos = ans["pos"]
@@ -130,13 +133,14 @@ def compare(w, items, answers, sel, s, o, tol_o=None, tol_s=TOL_S, out_dtype="f3
                 st["max_err_s"] = max(st["max_err_s"], e)
                 if not e <= tol_s:
                     st["fail"].append((it, "slot score", j, h, gs, os_[h, jo]))
-        allowed = tol_o
+        tol_n = tol_items[n]
+        allowed = tol_n
         if out_dtype == "bf16":
-            allowed = tol_o + np.ldexp(1.0, np.frexp(np.abs(oo))[1] - 9)   # half ulp of bf16 at |o|
+            allowed = tol_n + np.ldexp(1.0, np.frexp(np.abs(oo))[1] - 9)   # half ulp of bf16 at |o|
         e = np.abs(o[n] - oo)
         st["max_err_O"] = max(st["max_err_O"], float(np.max(e)))
         if not np.all(e <= allowed):
-            st["fail"].append((it, "output err %.3g" % float(np.max(e - allowed + tol_o))))
+            st["fail"].append((it, "output err %.3g (bound %.3g)" % (float(np.max(e - allowed + tol_n)), tol_n)))
     return st
 
 

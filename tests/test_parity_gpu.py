@@ -117,3 +117,55 @@ def test_exact_ties_lowest_index():
         assert [int(c) for c in sel[n]] == prim, (items[n], sel[n], prim)
     st = parity.compare(w, items, ans, sel, s, o)
     _check(st)
+
+
+def test_large_and_tiny_values():
+    """V entries far outside N(0,1): +-1e5 (beyond f16's range), +-3e4 (inside it) and +-1e-6 (f16
+    subnormals), planted in a few chunks of some (b, kv-head) slices, so that most rows of the blocks
+    that load those chunks did not select them.  The output is defined for every finite input
+    ("Hierarchical Sparse Attention Done Right", Sec. 3, "Hierarchical softmax"): no row may be
+    poisoned, and every row must match the oracle.
+
+    Bound per row: the value product rounds P to 16 bits (f16, relative 2^-11, or bf16, 2^-9, for a
+    slice holding a value beyond f16's range) and V enters it exactly, so the error from that rounding
+    is at most 2^-9 times the largest |v| the row attends to (its P sums to one).  Rows that attend to
+    |v| <= 8 only keep the usual 1e-2; rows that attend to a planted large value get 2^-8 times it."""
+    from synth import workloads as W
+    from synth.philox import f64_to_f32, f32_to_bf16_bits, bf16_bits_to_f64
+    w = wl("wide_values", B=2, H=8, Hkv=2, N=1024, T=1024, k=4, seed=140)
+    inp = W.full_inputs(w)
+    arr = {k: v[0].copy() for k, v in inp.items()}
+    raw = {k: v[1].copy() for k, v in inp.items()}
+
+    def plant(b, g, c, rows, cols, values):
+        for r_, c_, v_ in zip(rows, cols, values):
+            t = c * w.C + r_
+            bits = f32_to_bf16_bits(f64_to_f32(np.array([v_], dtype=np.float64)))[0]
+            raw["V"][b, g, t, c_] = bits
+            arr["V"][b, g, t, c_] = bf16_bits_to_f64(np.array([bits]))[0]
+
+    rng = np.random.default_rng(141)
+
+    def some(n, mag):
+        return (rng.integers(0, w.C, n), rng.integers(0, w.d, n), mag * rng.choice([-1.0, 1.0], n))
+
+    plant(0, 0, 5, *some(6, 1e5))          # slice (0, 0): beyond f16 -> the bf16 value product
+    plant(0, 1, 9, *some(6, 3e4))          # slice (0, 1): large but exact in f16
+    plant(1, 0, 3, *some(200, 1e-6))       # slice (1, 0): f16 subnormals
+    plant(1, 1, 12, *some(4, 1e5))         # slice (1, 1): both
+    plant(1, 1, 14, *some(200, 1e-6))
+    dev = {k: parity.to_device(v, w.dtype) for k, v in raw.items()}
+    O, sel_idx, sel_score = parity.gpu_run(w, dev)
+    assert torch.isfinite(O).all()
+    items = parity.all_items(w)
+    sel, s, o = parity.gather_gpu(w, O, sel_idx, sel_score, items)
+    ans = parity.answers_from_arrays(w, arr, items)
+    tol = []
+    for n, (b, g, i) in enumerate(items):
+        chunks = [int(c) for c in sel[n] if c >= 0] + [(w.q_offset + i) // w.C]
+        vmax = max(float(np.max(np.abs(arr["V"][b, g, c * w.C:(c + 1) * w.C]))) for c in chunks)
+        tol.append(parity.TOL_O["bf16"] if vmax <= 8.0 else 2.0 ** -8 * vmax)
+    st = parity.compare(w, items, ans, sel, s, o, tol_o=tol)
+    print({k: v for k, v in st.items() if k != "fail"}, "rows with a planted value:", sum(t > 0.01 for t in tol))
+    assert sum(t > 0.01 for t in tol) > 20     # the planted chunks were attended by some rows
+    _check(st)

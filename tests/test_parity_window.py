@@ -5,11 +5,12 @@ The window is the own chunk and the wc - 1 chunks before it, attended and fused 
 retrieval ranks only the chunks before the window, by the group score plus the chunk's bias, and the
 bias also enters every slot's fusion score ("Hierarchical Sparse Attention Done Right", Sec. 2
 Preliminary and Sec. 5 "Experimental setup" for the window, Sec. 3 "Linear surrogate for chunk mass"
-for the bias).  Checks per query group: the window slots exactly; the same retrieved chunks as the
-oracle, ranked in an order its scores allow (two chunks may swap only within the 1e-3 near-tie band),
-unless its k-th and (k+1)-th biased group scores lie within 1e-3 (such near ties at the cut are counted
-and left out); every slot's score, matched by chunk, within 1e-4; outputs within 1e-4 (float32 inputs)
-or 1e-2 (bf16).
+for the bias).  Checks for every query group: the window slots exactly; the same retrieved chunks as
+the oracle, ranked in an order its scores allow (two chunks may swap only within the 1e-3 near-tie
+band); where the oracle's biased group scores leave a near tie at the cut (within 1e-3), the GPU may
+keep any set the oracle enumerates for that band, and is then compared with the oracle run on that
+same set; every slot's score, matched by chunk, within 1e-4; outputs within 1e-4 (float32 inputs) or
+1e-2 (bf16).
 """
 import math
 
@@ -83,39 +84,73 @@ def _biased_group_scores(w, wc, arr, bias, b, g, i):
     return gs
 
 
+def _oracle_on_selection(w, wc, arr, bias, b, g, i, slots):
+    """The oracle's slot scores [G, k+wc] and outputs [G, d] for query (b, g, i) on the given slots
+    (retrieved chunks, then the window's chunks, the own chunk last)."""
+    pos = w.q_offset + i
+    ns = len(slots)
+    Ls = np.zeros((ns, w.d))
+    bs = np.zeros(ns)
+    Ks = np.zeros((ns, w.C, w.d))
+    Vs = np.zeros((ns, w.C, w.d))
+    for j, c in enumerate(slots):
+        if c < 0:
+            continue
+        t0, t1 = c * w.C, min((c + 1) * w.C, w.T)
+        Ls[j] = arr["L"][b, g, c]
+        bs[j] = bias[b, g, c] if bias is not None else 0.0
+        Ks[j, :t1 - t0] = arr["K"][b, g, t0:t1]
+        Vs[j, :t1 - t0] = arr["V"][b, g, t0:t1]
+    q = arr["Q"][b, g * w.G:(g + 1) * w.G, i]
+    r = orc.attend_slots(q, slots, Ls, bs if bias is not None else None, Ks, Vs, w.C, pos, 1.0 / math.sqrt(w.d))
+    return r["s"], r["o"]
+
+
 @pytest.mark.parametrize("case", CASES, ids=lambda c: c[0].name)
 def test_window_and_bias_match_the_oracle(case):
     w, wc, bias_scale = case
     arr, bias, ref, sel, s, O = _run(w, wc, bias_scale)
     kp = w.k + wc - 1
+    tol = 1e-4 if w.dtype == "f32" else 1e-2
     # the window slots: exact for every query group
     assert np.array_equal(sel[..., w.k:], ref["sel"][..., w.k:kp])
-    keep = np.ones((w.B, w.Hkv, w.N), dtype=bool)
+    n_alt = 0
+    max_err = 0.0
     for b in range(w.B):
         for g in range(w.Hkv):
             for i in range(w.N):
+                heads = slice(g * w.G, (g + 1) * w.G)
                 gs = _biased_group_scores(w, wc, arr, bias, b, g, i)
-                order = np.sort(gs)[::-1]
-                if w.k and len(gs) > w.k and order[w.k - 1] - order[w.k] < EPS_TIE:
-                    keep[b, g, i] = False          # near tie at the cut: either chunk may be kept
-                    continue
                 got, want = sel[b, g, i, :w.k], ref["sel"][b, g, i, :w.k]
-                assert sorted(got.tolist()) == sorted(want.tolist()), (b, g, i, got, want)
-                real = [int(c) for c in got if c >= 0]
+                m = min(w.k, len(gs))
+                real = [int(c) for c in got[:m]]
+                assert all(c == -1 for c in got[m:]), (b, g, i, got)
+                assert len(set(real)) == m and all(0 <= c < len(gs) for c in real), (b, g, i, got)
                 # rank order: by the oracle's scores, up to the near-tie band
                 assert all(gs[x] >= gs[y] - EPS_TIE for x, y in zip(real, real[1:])), (b, g, i, got)
-                assert all(c == -1 for c in got[len(real):])
+                if sorted(got.tolist()) == sorted(want.tolist()):
+                    ref_s = ref["s"][b, heads, i]
+                    ref_o = ref["O"][b, heads, i]
+                    ref_sel = [int(c) for c in ref["sel"][b, g, i]]
+                else:
+                    # a near tie at the cut: the set must be one the oracle allows for that band, and the
+                    # outputs are those of the oracle on that set
+                    alts = orc.tie_alternatives(gs, len(gs), w.k, EPS_TIE)
+                    assert alts is not None and any(sorted(a.tolist()) == sorted(got.tolist()) for a in alts), \
+                        (b, g, i, got, want)
+                    n_alt += 1
+                    ref_sel = real + [-1] * (w.k - m) + [int(c) for c in ref["sel"][b, g, i, w.k:]]
+                    ref_s, ref_o = _oracle_on_selection(w, wc, arr, bias, b, g, i, ref_sel)
                 # slot scores, matched by chunk (the window slots and the own chunk keep their places)
-                for h in range(g * w.G, (g + 1) * w.G):
-                    ref_by_chunk = {int(c): ref["s"][b, h, i, j] for j, c in enumerate(ref["sel"][b, g, i]) if c >= 0}
+                ref_by_chunk = [{c: ref_s[h, j] for j, c in enumerate(ref_sel) if c >= 0} for h in range(w.G)]
+                for h in range(w.G):
                     for j in range(kp + 1):
                         c = int(sel[b, g, i, j]) if j < kp else (w.q_offset + i) // w.C
                         if c < 0:
-                            assert np.isneginf(s[b, h, i, j])
+                            assert np.isneginf(s[b, g * w.G + h, i, j])
                         else:
-                            assert abs(s[b, h, i, j] - ref_by_chunk[c]) <= TOL_S, (b, h, i, j)
-    assert keep.mean() > 0.8, keep.mean()
-    keep_h = np.repeat(keep, w.G, axis=1)
-    tol = 1e-4 if w.dtype == "f32" else 1e-2
-    err = np.max(np.abs(O[keep_h] - ref["O"][keep_h]), initial=0.0)
-    assert err <= tol, err
+                            assert abs(s[b, g * w.G + h, i, j] - ref_by_chunk[h][c]) <= TOL_S, (b, h, i, j)
+                e = float(np.max(np.abs(O[b, heads, i] - ref_o)))
+                max_err = max(max_err, e)
+                assert e <= tol, (b, g, i, e)
+    print(w.name, "max err %.3g" % max_err, "near-tie selections compared on their own set:", n_alt)
