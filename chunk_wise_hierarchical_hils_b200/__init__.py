@@ -28,7 +28,8 @@ EXPORTS = ("hils_status_string", "hils_version", "hils_validate", "hils_score_se
            "hils_chunk_attend_fuse_workspace_size", "hils_forward_workspace_size", "hils_score_select",
            "hils_chunk_attend_fuse", "hils_forward", "hils_sync_status", "hils_set_wait_limit",
            "hils_decode_score_select_noalloc", "hils_debug_inject_stall", "hils_landmarks",
-           "hils_score_select_window", "hils_forward_window_workspace_size", "hils_forward_window")
+           "hils_score_select_window", "hils_forward_window_workspace_size", "hils_forward_window",
+           "hils_backward")
 HILS_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -74,6 +75,7 @@ def _load():
     lib.hils_score_select_window.argtypes = [P, ci, vp, vp, vp, vp, vp, vp]
     lib.hils_forward_window_workspace_size.argtypes = [P, ci, ctypes.POINTER(sz)]
     lib.hils_forward_window.argtypes = [P, ci, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.hils_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     for n in EXPORTS[2:]:
         if n not in ("hils_status_string", "hils_version"):
             getattr(lib, n).restype = ctypes.c_int
@@ -222,6 +224,12 @@ def hils_forward_window(p, window_chunks, bias, Q, K, V, L, O, workspace=None, s
     wp, wn = _ws(workspace)
     _check(_lib.hils_forward_window(ctypes.byref(p), int(window_chunks), _ptr(bias), _ptr(Q), _ptr(K), _ptr(V),
                                     _ptr(L), _ptr(O), wp, wn, _stream(stream)), "hils_forward_window")
+
+
+def hils_backward(p, Q, K, V, L, sel_idx, dO, dQ, dK, dV, dL, stream=None):
+    """Gradients dQ, dK, dV, dL (float32 tensors, written) of sum(O * dO) through the selection sel_idx."""
+    _check(_lib.hils_backward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(sel_idx), _ptr(dO), _ptr(dQ),
+                              _ptr(dK), _ptr(dV), _ptr(dL), _stream(stream)), "hils_backward")
 
 
 def problem(B, H, Hkv, N, T, d, C, k, q_offset=0, in_dtype=HILS_BF16, out_dtype=None, scale=0.0):

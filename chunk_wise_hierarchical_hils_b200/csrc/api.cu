@@ -347,6 +347,23 @@ hils_status hils_landmarks(const hils_problem *p, const void *K, const void *U, 
                                       c_end, static_cast<cudaStream_t>(stream)));
 }
 
+hils_status hils_backward(const hils_problem *p, const void *Q, const void *K, const void *V, const void *L,
+                          const int32_t *sel_idx, const void *dO, float *dQ, float *dK, float *dV, float *dL,
+                          void *stream)
+{
+    Dims d;
+    hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    if (!Q || !K || !V || !L || !dO || !dQ || !dK || !dV || !dL || (d.k > 0 && !sel_idx)) return HILS_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(L) || !aligned16(dO) || !aligned16(dQ) ||
+        !aligned16(dK) || !aligned16(dV) || !aligned16(dL) || (sel_idx && !aligned16(sel_idx)))
+        return HILS_ERR_INVALID_ARG;
+    if (backward_smem_bytes(d) > 227 * 1024) return HILS_ERR_UNSUPPORTED;
+    if ((long long)d.B * d.Hkv * d.N > 0x7FFFFFFFll) return HILS_ERR_UNSUPPORTED;
+    return from_cuda(launch_backward(d, p->in_dtype, Q, K, V, L, sel_idx, dO, dQ, dK, dV, dL,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 hils_status hils_sync_status(void *stream)
 {
     DeviceCtl ctl;

@@ -74,7 +74,7 @@
 extern "C" {
 #endif
 
-#define HILS_VERSION 110    /* 1.1.0: adds the window/bias selection and forward, and landmark generation */
+#define HILS_VERSION 120    /* 1.2.0: adds the backward pass (1.1.0: window/bias selection and forward, landmarks) */
 #define HILS_MAX_K 64       /* largest supported top-k */
 #define HILS_MAX_GROUP 16   /* largest supported H / Hkv */
 
@@ -221,6 +221,32 @@ HILS_API hils_status hils_forward_window(const hils_problem *p, int window_chunk
  */
 HILS_API hils_status hils_landmarks(const hils_problem *p, const void *K, const void *U, void *L, float *beta,
                                     int c_begin, int c_end, void *stream);
+
+/*
+ * Backward pass through a fixed selection (Sec. 3 Methodology, "Hierarchical
+ * softmax": the retrieval scores enter the output as fusion weights, so the
+ * loss trains the landmarks and the retrieval through them; a chunk that is
+ * not selected gets no gradient; the selection, a discrete choice, is held
+ * fixed).  Given the selection sel_idx [B][Hkv][N][k] (as hils_score_select
+ * writes it: -1 padded, entries -1 or past chunks of their query, no repeats;
+ * the own chunk is implied) and the upstream gradient dO [B][H][N][d]
+ * (in_dtype), writes the gradients of sum(O * dO) as float32:
+ *   dQ [B][H][N][d], dK and dV [B][Hkv][T][d], dL [B][Hkv][nL][d].
+ * With s_c = scale <q, L_c>, w = softmax over the slots of s, P^c the softmax
+ * inside chunk c and u_j = <dO, v_j>, per head and query:
+ *   dw_c = sum_j P^c_j u_j,  ds_c = w_c (dw_c - sum_c' w_c' dw_c'),
+ *   dq   = scale sum_c (ds_c L_c + sum_j dl_j k_j),  dl_j = w_c P^c_j (u_j - dw_c),
+ *   dL_c += scale ds_c q,  dk_j += scale dl_j q,  dv_j += w_c P^c_j dO,
+ * summed over the queries and heads that reach a row.  Rows of K, V and L that
+ * no query reaches get zeros.  The call zeroes dK, dV and dL and accumulates
+ * them with float32 atomics (their summation order, hence their last bits,
+ * can differ between runs); dQ is written once per row.  Shapes and dtypes as
+ * for hils_forward (out_dtype is ignored); every pointer 16-byte aligned.  No
+ * workspace; asynchronous on `stream`.  Computed on CUDA cores in float32.
+ */
+HILS_API hils_status hils_backward(const hils_problem *p, const void *Q, const void *K, const void *V,
+                                   const void *L, const int32_t *sel_idx, const void *dO, float *dQ,
+                                   float *dK, float *dV, float *dL, void *stream);
 
 /*
  * Synchronise `stream` and report device-side status since the last call:

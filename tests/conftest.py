@@ -14,10 +14,10 @@ def pytest_configure(config):
 # Suites that run after all others, in this order, so that a run stopping at its first failure has
 # already run the main forward-path suites: the prefill shapes with a single value slot, the window
 # and bias extension, landmark generation (a step before the forward path), the debug check of a
-# caller's selection, and last of all the allocation-free entry point (its first call sets up a
-# per-device array), so that every other test has run before it.
+# caller's selection, the backward pass, and last of all the allocation-free entry point (its first
+# call sets up a per-device array), so that every other test has run before it.
 RUN_LAST = ("test_parity_one_value_slot.py", "test_parity_window.py", "test_parity_landmarks.py",
-            "test_check_selection.py", "test_zz_no_alloc.py")
+            "test_check_selection.py", "test_parity_backward.py", "test_zz_no_alloc.py")
 
 
 def pytest_collection_modifyitems(config, items):

@@ -22,7 +22,7 @@ def test_header_symbols_exported():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) <= set(hils.EXPORTS) | set(names)
-    assert hils.hils_version() == 110
+    assert hils.hils_version() == 120
 
 
 def test_struct_layout_matches_header():
@@ -192,4 +192,4 @@ def test_header_is_plain_c_and_links(tmp_path):
     subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
                            "-L", libdir, "-lhils", "-Wl,-rpath," + libdir, "-o", str(exe)])
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
-    assert out[0] == "110"
+    assert out[0] == "120"
