@@ -97,6 +97,14 @@ bool check_caller_selection()
     return v && strcmp(v, "1") == 0;
 }
 
+// Test control: HILS_SELECT_KERNEL=heads keeps the prefill selection on the kernel with one product row
+// per head (the kernel used above k = 32), to cross-check it against the one with a row per query.
+bool force_select_heads()
+{
+    const char *force = getenv("HILS_SELECT_KERNEL");
+    return force && strcmp(force, "heads") == 0;
+}
+
 // Test control: HILS_DECODE_KERNEL=simt keeps decode attention on the CUDA-core kernel.
 bool force_decode_cuda_cores()
 {
@@ -119,6 +127,8 @@ hils_status do_select(const Dims &p, hils_dtype in, const void *Q, const void *L
     hils_status st = device_ctl(&ctl);
     if (st != HILS_OK) return st;
     if (p.N == 1) return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, ctl, s));
+    if (!force_cuda_cores() && !force_select_heads() && select_q_supported(p, in))
+        return from_cuda(launch_select_prefill_q(p, Q, L, sel_idx, sel_score, ctl, s));
     if (!force_cuda_cores() && select_tc_supported(p, in))
         return from_cuda(launch_select_prefill_tc(p, Q, L, sel_idx, sel_score, ctl, s));
     return from_cuda(launch_select_prefill(p, in, Q, L, sel_idx, sel_score, s));

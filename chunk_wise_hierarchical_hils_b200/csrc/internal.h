@@ -60,6 +60,10 @@ bool attend_tc_supported(const Dims &p, hils_dtype in);
 bool select_tc_supported(const Dims &p, hils_dtype in);
 cudaError_t launch_select_prefill_tc(const Dims &p, const void *Q, const void *L, int32_t *sel_idx,
                                      float *sel_score, const DeviceCtl &ctl, cudaStream_t s);
+// Prefill selection with one product row per query (group score from the mean query): bf16, d = 128, k <= 32.
+bool select_q_supported(const Dims &p, hils_dtype in);
+cudaError_t launch_select_prefill_q(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
+                                    const DeviceCtl &ctl, cudaStream_t s);
 size_t attend_tc_ws_bytes(const Dims &p);
 cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
                                      const int32_t *sel_idx, const float *sel_score, void *O, void *ws,

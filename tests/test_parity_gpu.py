@@ -70,6 +70,15 @@ def test_cuda_core_kernel_too(w, monkeypatch):
     _check(st)
 
 
+@pytest.mark.parametrize("w", [CASES[1], CASES[8], CASES[10], CASES[12]], ids=lambda w: w.name)
+def test_selection_with_a_row_per_head_too(w, monkeypatch):
+    """The tensor-core selection with one product row per head (used above k = 32), forced, on shapes the
+    kernel with one row per query normally takes."""
+    monkeypatch.setenv("HILS_SELECT_KERNEL", "heads")
+    st, _ = parity.run_small(w)
+    _check(st)
+
+
 @pytest.mark.parametrize("w", [DECODE[0], DECODE[2], DECODE[4], DECODE[5]], ids=lambda w: w.name)
 def test_cuda_core_decode_too(w, monkeypatch):
     """The CUDA-core decode attention kernel, forced, on shapes the tensor-core tile kernel normally takes."""
