@@ -89,9 +89,26 @@ def landmark_gen_bytes(w):
     return w.B * w.Hkv * (es * w.T * w.d + 2 * es * w.nL * w.d + 4 * w.nL)
 
 
+def decode_fused_applies(w, n_sm=148):
+    """Whether hils_forward runs a single-token decode as one fused kernel (bf16, d = 128, C = 64, at
+    most one (b, kv-head) pair per SM, at most 4096 landmark rows per CTA)."""
+    if w.N != 1 or w.dtype != "bf16" or w.d != 128 or w.C != 64 or w.G > 16 or w.k > 64:
+        return False
+    if os.environ.get("HILS_DECODE_FUSED") == "0":
+        return False
+    bg = w.B * w.Hkv
+    if bg > n_sm:
+        return False
+    S = min(n_sm // bg, 32)
+    n_past = w.q_offset // w.C if w.k > 0 else 0
+    return -(-n_past // 4096) <= S
+
+
 def kernels_per_step(w):
     """Kernels of this library one step launches (the input generator and copies are not counted)."""
     if w.N == 1:
+        if decode_fused_applies(w):
+            return 1      # the fused decode kernel (plus a memset of its tickets)
         return 2          # decode landmark scan + top-k, decode attention (plus two ticket memsets)
     # prefill: selection; [V to f16 (plus a memset of the slice flags) +] attention
     tc = w.dtype == "bf16" and w.d == 128 and w.G in (1, 2, 4, 8, 16) and os.environ.get("HILS_PREFILL_KERNEL") != "simt"
@@ -426,8 +443,8 @@ def measure_forward(args, w, ws, rank, local, steps=None):
         hils.hils_chunk_attend_fuse(p, dev["Q"], dev["K"], dev["V"], sel_idx, sel_score, O, ws_att)
 
     def step():
-        call_select()
-        call_attend()
+        # the public call: selection then attention (single-token decode: one fused kernel where it applies)
+        hils.hils_forward(p, dev["Q"], dev["K"], dev["V"], dev["L"], O, ws_fwd)
 
     for _ in range(args.warmup):
         step()
@@ -441,7 +458,9 @@ def measure_forward(args, w, ws, rank, local, steps=None):
             fn()
         return g_
 
-    g_step, g_sel, g_att = capture(step), capture(call_select), capture(call_attend)
+    g_step = capture(step)
+    # per-call graphs: prefill's selection and attention; decode's two-kernel path for comparison
+    g_sel, g_att = capture(call_select), capture(call_attend)
     flush = needs_flush(w)
     timer = StepTimer(flush)
     # short steps are repeated so that the clock sampler sees the GPU under load (about half a second)
@@ -505,6 +524,7 @@ def measure_forward(args, w, ws, rank, local, steps=None):
 
     pk, pk_kind = peaks()
     timed_s = total_ms * 1e-3
+    fused = w.N == 1 and decode_fused_applies(w)
     if w.N > 1:
         unit = "tokens/s"
         per_step_units = w.B * w.N
@@ -521,6 +541,18 @@ def measure_forward(args, w, ws, rank, local, steps=None):
                 "traffic": kernel_traffic("attend_prefill_tc", w.name), "peak_kind": kind,
                 "algorithmic_flops_per_launch": fl, "launch_ms": k2_avg, "select_ms": k1_avg,
                 "step_tflops": (fl + scoring_flops(w)) / (ms_step * 1e-3) / 1e12}
+    elif fused:
+        # one kernel per step (plus a memset of its tickets): its roofline is the step's bytes over the step
+        unit = "GB/s"
+        per_step_units = decode_bytes(w) / 1e9
+        peak = pk["hbm_gbs"]
+        step_gbs = decode_bytes(w) / (ms_step * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "decode_fused (selection + attention, one cooperative kernel)",
+                "achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
+                "traffic": kernel_traffic("decode_fused", w.name), "algorithmic_bytes_per_launch": decode_bytes(w),
+                "launch_ms": ms_step, "two_kernel_select_ms": k1_avg, "two_kernel_attend_ms": k2_avg,
+                "peak_kind": pk_kind + " copy", "frac_of_spec": step_gbs / HBM_SPEC_GBS, "step_gbs": step_gbs,
+                "step_frac": step_gbs / peak, "step_frac_of_spec": step_gbs / HBM_SPEC_GBS}
     else:
         unit = "GB/s"
         per_step_units = decode_bytes(w) / 1e9

@@ -97,12 +97,22 @@ bool check_caller_selection()
     return v && strcmp(v, "1") == 0;
 }
 
-// Test control: HILS_SELECT_KERNEL=heads keeps the prefill selection on the kernel with one product row
-// per head (the kernel used above k = 32), to cross-check it against the one with a row per query.
-bool force_select_heads()
+// Test control: HILS_SELECT_KERNEL=heads or =queries forces the tensor-core prefill selection with one
+// product row per head or per query (where it covers the shape), to cross-check the two.
+int forced_select_kernel()
 {
     const char *force = getenv("HILS_SELECT_KERNEL");
-    return force && strcmp(force, "heads") == 0;
+    if (force && strcmp(force, "heads") == 0) return 1;
+    if (force && strcmp(force, "queries") == 0) return 2;
+    return 0;
+}
+
+// Test control: HILS_DECODE_FUSED=0 keeps hils_forward's single-token decode on the two kernels
+// (selection, then attention) instead of the fused cooperative kernel.
+bool fused_decode_enabled()
+{
+    const char *v = getenv("HILS_DECODE_FUSED");
+    return !(v && strcmp(v, "0") == 0);
 }
 
 // Test control: HILS_DECODE_KERNEL=simt keeps decode attention on the CUDA-core kernel.
@@ -127,7 +137,8 @@ hils_status do_select(const Dims &p, hils_dtype in, const void *Q, const void *L
     hils_status st = device_ctl(&ctl);
     if (st != HILS_OK) return st;
     if (p.N == 1) return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, ctl, s));
-    if (!force_cuda_cores() && !force_select_heads() && select_q_supported(p, in))
+    const int forced = forced_select_kernel();
+    if (!force_cuda_cores() && forced != 1 && select_q_supported(p, in) && (forced == 2 || select_q_preferred(p)))
         return from_cuda(launch_select_prefill_q(p, Q, L, sel_idx, sel_score, ctl, s));
     if (!force_cuda_cores() && select_tc_supported(p, in))
         return from_cuda(launch_select_prefill_tc(p, Q, L, sel_idx, sel_score, ctl, s));
@@ -228,7 +239,8 @@ hils_status hils_forward_workspace_size(const hils_problem *p, size_t *bytes)
     if (!bytes) return HILS_ERR_INVALID_ARG;
     hils_status st = resolve(p, &d);
     if (st != HILS_OK) return st;
-    const size_t scratch = select_ws(d) > attend_ws(d, p->in_dtype) ? select_ws(d) : attend_ws(d, p->in_dtype);
+    size_t scratch = select_ws(d) > attend_ws(d, p->in_dtype) ? select_ws(d) : attend_ws(d, p->in_dtype);
+    if (decode_fused_supported(d, p->in_dtype) && decode_fused_ws_bytes(d) > scratch) scratch = decode_fused_ws_bytes(d);
     *bytes = sel_idx_bytes(d) + sel_score_bytes(d) + scratch;
     return HILS_OK;
 }
@@ -286,6 +298,12 @@ hils_status hils_forward(const hils_problem *p, const void *Q, const void *K, co
     float *sel_score = reinterpret_cast<float *>(ws + sel_idx_bytes(d));
     void *scratch = ws + sel_idx_bytes(d) + sel_score_bytes(d);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (fused_decode_enabled() && !force_decode_cuda_cores() && decode_fused_supported(d, p->in_dtype)) {
+        DeviceCtl ctl;
+        st = device_ctl(&ctl);
+        if (st != HILS_OK) return st;
+        return from_cuda(launch_decode_fused(d, p->out_dtype, Q, K, V, L, sel_idx, sel_score, O, scratch, ctl, s));
+    }
     st = do_select(d, p->in_dtype, Q, L, sel_idx, sel_score, scratch, s);
     if (st != HILS_OK) return st;
     return do_attend(d, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, scratch, s);

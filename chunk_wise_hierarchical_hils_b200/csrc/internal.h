@@ -62,6 +62,7 @@ cudaError_t launch_select_prefill_tc(const Dims &p, const void *Q, const void *L
                                      float *sel_score, const DeviceCtl &ctl, cudaStream_t s);
 // Prefill selection with one product row per query (group score from the mean query): bf16, d = 128, k <= 32.
 bool select_q_supported(const Dims &p, hils_dtype in);
+bool select_q_preferred(const Dims &p);   // where it beats the kernel with a row per head
 cudaError_t launch_select_prefill_q(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
                                     const DeviceCtl &ctl, cudaStream_t s);
 size_t attend_tc_ws_bytes(const Dims &p);
@@ -78,6 +79,14 @@ bool attend_decode_mma_supported(const Dims &p, hils_dtype in);
 cudaError_t launch_attend_decode_mma(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
                                      const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
                                      const DeviceCtl &ctl, cudaStream_t s);
+
+// Single-token decode in one cooperative kernel (selection and attention): bf16, d = 128, C = 64, with
+// B * Hkv no more than the SM count.  Writes sel_idx / sel_score (N == 1 rows) as well as O.
+bool decode_fused_supported(const Dims &p, hils_dtype in);
+size_t decode_fused_ws_bytes(const Dims &p);
+cudaError_t launch_decode_fused(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
+                                const void *L, int32_t *sel_idx, float *sel_score, void *O, void *ws,
+                                const DeviceCtl &ctl, cudaStream_t s);
 
 // TMA tile map (no interleave, 128-byte swizzle, 256-byte L2 promotion, zero fill out of bounds); rank 1..3,
 // strides in bytes for dimensions 1..rank-1.  False when the driver's encoder is missing or rejects the map.

@@ -347,45 +347,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (*abort_flag) return;
 
     // ---- per-head slot scores: scale q_h . L_c for the k selected chunks and the own chunk ------------
-    // query rows of up to kHeadBatch heads at a time in the freed stages (bf16), 16-byte pieces rotated
-    // by query so that threads of different queries read different banks
+    // query rows of up to kHeadBatch heads at a time in the freed stages (bf16, asynchronous copies),
+    // 16-byte pieces rotated by query so that threads of different queries read different banks; one
+    // thread per (query, slot), the next item's landmark row loaded while the current one is computed
     unsigned char *qrows = base;   // [head in batch][query][16 pieces] (uint4)
     const __nv_bfloat16 *Lbg = Lm + ((size_t)b * p.Hkv + g) * p.nL * kD;
+    const int n_items = nq * ns;
     for (int h0 = 0; h0 < G; h0 += kHeadBatch) {
         const int hb = min(kHeadBatch, G - h0);
         if (h0 > 0) __syncthreads();
         for (int e = tid; e < hb * nq * 16; e += kThreads) {
             const int hh = e / (nq * 16), rem = e % (nq * 16), qi = rem >> 4, seg = rem & 15;
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
-                                      Q + ((((size_t)b * p.H + (size_t)g * G + h0 + hh) * p.N) + q0 + qi) * kD) + seg);
-            *reinterpret_cast<uint4 *>(qrows + (((size_t)hh * kRows + qi) * 16 + ((seg + qi) & 15)) * 16) = v;
+            const __nv_bfloat16 *src =
+                Q + ((((size_t)b * p.H + (size_t)g * G + h0 + hh) * p.N) + q0 + qi) * kD + seg * 8;
+            const uint32_t dst = smem_addr(qrows + (((size_t)hh * kRows + qi) * 16 + ((seg + qi) & 15)) * 16);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
         }
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
         __syncthreads();
-        for (int it = tid; it < nq * ns; it += kThreads) {
+        uint4 nxt[16];
+        auto fetch = [&](int it) {
+            const int c = it < n_items ? selc[(it / ns) * ns + it % ns] : -1;
+            const uint4 *lr = reinterpret_cast<const uint4 *>(Lbg + (size_t)(c >= 0 ? c : 0) * kD);
+#pragma unroll
+            for (int seg = 0; seg < 16; ++seg) nxt[seg] = (c >= 0) ? __ldg(lr + seg) : make_uint4(0u, 0u, 0u, 0u);
+        };
+        fetch(tid);
+        for (int it = tid; it < n_items; it += kThreads) {
+            uint4 lv[16];
+#pragma unroll
+            for (int seg = 0; seg < 16; ++seg) lv[seg] = nxt[seg];
+            fetch(it + kThreads);
             const int qi = it / ns, j = it % ns;
             const int c = selc[qi * ns + j];
             float acc[kHeadBatch];
 #pragma unroll
             for (int hh = 0; hh < kHeadBatch; ++hh) acc[hh] = 0.f;
-            if (c >= 0) {
-                const uint4 *lr = reinterpret_cast<const uint4 *>(Lbg + (size_t)c * kD);
-                uint4 lv[16];
 #pragma unroll
-                for (int seg = 0; seg < 16; ++seg) lv[seg] = __ldg(lr + seg);
+            for (int seg = 0; seg < 16; ++seg) {
+                float lf[8];
+                unpack_bf16x8(lv[seg], lf);
 #pragma unroll
-                for (int seg = 0; seg < 16; ++seg) {
-                    float lf[8];
-                    unpack_bf16x8(lv[seg], lf);
+                for (int hh = 0; hh < kHeadBatch; ++hh) {
+                    if (hh < hb) {
+                        float qf[8];
+                        unpack_bf16x8(*reinterpret_cast<const uint4 *>(
+                                          qrows + (((size_t)hh * kRows + qi) * 16 + ((seg + qi) & 15)) * 16),
+                                      qf);
 #pragma unroll
-                    for (int hh = 0; hh < kHeadBatch; ++hh) {
-                        if (hh < hb) {
-                            float qf[8];
-                            unpack_bf16x8(*reinterpret_cast<const uint4 *>(
-                                              qrows + (((size_t)hh * kRows + qi) * 16 + ((seg + qi) & 15)) * 16),
-                                          qf);
-#pragma unroll
-                            for (int x = 0; x < 8; ++x) acc[hh] = fmaf(qf[x], lf[x], acc[hh]);
-                        }
+                        for (int x = 0; x < 8; ++x) acc[hh] = fmaf(qf[x], lf[x], acc[hh]);
                     }
                 }
             }
@@ -419,10 +429,20 @@ EncodeTiledFn encode_fn()
 
 }  // namespace
 
+// The kernel with one row per query pays for its G-fold smaller scan with the per-head slot scores it
+// computes afterwards on CUDA cores; the kernel with one row per head gets those with the scan.  So
+// this one is used where the scan dominates: k above 16 (the other kernel keeps larger lists in a
+// shared-memory heap) or more than 512 visible chunks.
 bool select_q_supported(const Dims &p, hils_dtype in)
 {
     if (in != HILS_BF16 || p.d != kD || p.N < 2 || p.k > 32) return false;
     return make_layout(p.k).total + 1024 <= 227 * 1024;
+}
+
+bool select_q_preferred(const Dims &p)
+{
+    const long long c_max = ((long long)p.q_offset + p.N - 1) / p.C;
+    return p.k > 16 || c_max >= 512;
 }
 
 cudaError_t launch_select_prefill_q(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,

@@ -70,13 +70,54 @@ def test_cuda_core_kernel_too(w, monkeypatch):
     _check(st)
 
 
-@pytest.mark.parametrize("w", [CASES[1], CASES[8], CASES[10], CASES[12]], ids=lambda w: w.name)
-def test_selection_with_a_row_per_head_too(w, monkeypatch):
-    """The tensor-core selection with one product row per head (used above k = 32), forced, on shapes the
-    kernel with one row per query normally takes."""
-    monkeypatch.setenv("HILS_SELECT_KERNEL", "heads")
+@pytest.mark.parametrize("kernel", ["heads", "queries"])
+@pytest.mark.parametrize("w", [CASES[1], CASES[3], CASES[5], CASES[6], CASES[7], CASES[8], CASES[10], CASES[11],
+                               CASES[12]], ids=lambda w: w.name)
+def test_both_tensor_core_selections(w, kernel, monkeypatch):
+    """Each tensor-core prefill selection forced on shapes the other one may take: one product row per
+    head (group score by a butterfly over the heads) or one per query (group score from the mean query,
+    per-head slot scores after the scan)."""
+    monkeypatch.setenv("HILS_SELECT_KERNEL", kernel)
     st, _ = parity.run_small(w)
     _check(st)
+
+
+@pytest.mark.parametrize("w", [DECODE[0], DECODE[2], DECODE[3], DECODE[4], DECODE[6]], ids=lambda w: w.name)
+def test_two_kernel_decode_too(w, monkeypatch):
+    """hils_forward's single-token decode on the two kernels (selection, then attention), forced, on shapes
+    the fused cooperative kernel normally takes."""
+    monkeypatch.setenv("HILS_DECODE_FUSED", "0")
+    st, _ = parity.run_small(w)
+    _check(st)
+
+
+@pytest.mark.parametrize("w", [DECODE[0], DECODE[4], DECODE[6]], ids=lambda w: w.name)
+def test_fused_decode_selection_equals_the_selection_call(w):
+    """The fused decode kernel writes its selection into hils_forward's workspace: it must equal
+    hils_score_select's bit for bit (same scores, same order), and its slot scores agree within 1e-6."""
+    import chunk_wise_hierarchical_hils_b200 as hils
+    from synth import workloads as W
+    inp = W.full_inputs(w)
+    dev = {k: parity.to_device(v[1], w.dtype) for k, v in inp.items()}
+    p = parity.problem_of(w)
+    sel_idx = torch.empty((w.B, w.Hkv, 1, w.k), dtype=torch.int32, device="cuda")
+    sel_score = torch.empty((w.B, w.H, 1, w.k + 1), dtype=torch.float32, device="cuda")
+    ws_sel = torch.empty(max(hils.hils_score_select_workspace_size(p), 1), dtype=torch.uint8, device="cuda")
+    hils.hils_score_select(p, dev["Q"], dev["L"], sel_idx, sel_score, ws_sel)
+    O = torch.empty((w.B, w.H, 1, w.d), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(hils.hils_forward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    hils.hils_forward(p, dev["Q"], dev["K"], dev["V"], dev["L"], O, ws)
+    assert hils.hils_sync_status() == hils.HILS_OK
+    # hils_forward keeps the selection at the start of its workspace: sel_idx rows, then (256-byte
+    # aligned) the slot scores
+    n_idx = w.B * w.Hkv * w.k
+    off = (n_idx * 4 + 255) // 256 * 256
+    f_idx = ws[:n_idx * 4].view(torch.int32).view(w.B, w.Hkv, 1, w.k)
+    f_score = ws[off:off + w.B * w.H * (w.k + 1) * 4].view(torch.float32).view(w.B, w.H, 1, w.k + 1)
+    assert torch.equal(f_idx, sel_idx)
+    fin = torch.isfinite(sel_score)
+    assert torch.equal(fin, torch.isfinite(f_score))
+    assert float((f_score[fin] - sel_score[fin]).abs().max()) <= 1e-6
 
 
 @pytest.mark.parametrize("w", [DECODE[0], DECODE[2], DECODE[4], DECODE[5]], ids=lambda w: w.name)
