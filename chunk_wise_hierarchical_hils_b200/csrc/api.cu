@@ -1,5 +1,6 @@
 // api.cu -- the C ABI of libhils.so: validation, workspace sizing, dispatch.
 #include <math.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 #include <mutex>
@@ -81,7 +82,15 @@ size_t attend_ws(const Dims &p, hils_dtype in)
     return attend_tc_supported(p, in) ? attend_tc_ws_bytes(p) : 0;
 }
 
-hils_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA; }
+// Debug control: HILS_DEBUG=1 prints the CUDA runtime's error string when a launch or runtime call
+// of an entry point fails (the status alone says only HILS_ERR_CUDA).
+hils_status from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess) return HILS_OK;
+    const char *dbg = getenv("HILS_DEBUG");
+    if (dbg && strcmp(dbg, "1") == 0) fprintf(stderr, "hils: CUDA error %d: %s\n", (int)e, cudaGetErrorString(e));
+    return HILS_ERR_CUDA;
+}
 
 // HILS_PREFILL_KERNEL=simt forces the CUDA-core prefill kernels (used to cross-check the two paths).
 bool force_cuda_cores()

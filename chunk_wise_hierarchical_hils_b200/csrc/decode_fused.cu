@@ -12,7 +12,7 @@
 // (b, g) pairs to fill the GPU, more for a few long sequences), all resident at once (a cooperative
 // launch):
 //   phase 1  CTA s streams its share of the landmark rows through a ring of bulk copies (a producer
-//            warp, eight consumer warps), scores them with the group's mean query (the same float32
+//            warp, seven consumer warps), scores them with the group's mean query (the same float32
 //            steps as the two-kernel selection, so both choose the same chunks) and keeps a local
 //            top-k; the last of the S CTAs (atomic ticket) merges the S lists, writes the selection
 //            and the per-head slot scores, and publishes them (a release flag);
@@ -37,8 +37,8 @@ namespace {
 using namespace sm100;
 using dtiles::kQPitch;
 
-constexpr int kWarps = 8;                         // consumer warps
-constexpr int kThreads = 32 * (kWarps + 1);       // + one producer warp
+constexpr int kWarps = 7;                         // consumer warps (eight warps in all: two per SM
+constexpr int kThreads = 32 * (kWarps + 1);       // sub-partition, so that each may hold 255 registers)
 constexpr int kD = 128, kC = 64;
 constexpr int kLRows = 64;                        // landmark rows per phase-1 stage
 constexpr uint32_t kLStage = kLRows * kD * 2;     // 16 KB
@@ -98,7 +98,7 @@ __device__ __forceinline__ void st_release(unsigned int *p, unsigned int v)
 }
 
 template <typename Tout>
-__global__ void __maxnreg__(224)
+__global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Dims p,
                         FusedArgs a, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ Lm,
                         int32_t *__restrict__ sel_idx, float *__restrict__ sel_score, Tout *__restrict__ O,
