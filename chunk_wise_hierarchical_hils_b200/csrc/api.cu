@@ -76,9 +76,29 @@ namespace {
 size_t sel_idx_bytes(const Dims &p) { return align_up((size_t)p.B * p.Hkv * p.N * p.k * sizeof(int32_t), 256); }
 size_t sel_score_bytes(const Dims &p) { return align_up((size_t)p.B * p.H * p.N * (p.k + 1) * sizeof(float), 256); }
 size_t select_ws(const Dims &p) { return p.N == 1 ? decode_select_ws_bytes(p) : 0; }
-size_t attend_ws(const Dims &p, hils_dtype in)
+// Test control: HILS_PREFILL_ATTEND=union or =chunk forces the tensor-core prefill attention that walks
+// each query block's chunk union, or the chunk-major one (where it covers the shape).
+int forced_prefill_attend()
+{
+    const char *force = getenv("HILS_PREFILL_ATTEND");
+    if (force && strcmp(force, "union") == 0) return 1;
+    if (force && strcmp(force, "chunk") == 0) return 2;
+    return 0;
+}
+
+bool use_chunk_major(const Dims &p, hils_dtype in)
+{
+    const char *simt = getenv("HILS_PREFILL_KERNEL");
+    if (simt && strcmp(simt, "simt") == 0) return false;
+    const int forced = forced_prefill_attend();
+    if (forced == 1 || !attend_cm_supported(p, in)) return false;
+    return forced == 2 || attend_cm_preferred(p);
+}
+
+size_t attend_ws(const Dims &p, hils_dtype in, hils_dtype out)
 {
     if (p.N == 1) return decode_attend_ws_bytes(p);
+    if (use_chunk_major(p, in)) return attend_cm_ws_bytes(p, out);
     return attend_tc_supported(p, in) ? attend_tc_ws_bytes(p) : 0;
 }
 
@@ -190,6 +210,8 @@ cudaError_t launch_attend_prefill(const Dims &p, hils_dtype in, hils_dtype out, 
                                   const void *V, const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
                                   const DeviceCtl &ctl, cudaStream_t s)
 {
+    if (use_chunk_major(p, in))
+        return launch_attend_prefill_cm(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s);
     if (!force_cuda_cores() && attend_tc_supported(p, in))
         return launch_attend_prefill_tc(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s);
     return launch_attend_prefill_simt(p, in, out, Q, K, V, sel_idx, sel_score, O, s);
@@ -238,7 +260,7 @@ hils_status hils_chunk_attend_fuse_workspace_size(const hils_problem *p, size_t 
     if (!bytes) return HILS_ERR_INVALID_ARG;
     hils_status st = resolve(p, &d);
     if (st != HILS_OK) return st;
-    *bytes = attend_ws(d, p->in_dtype);
+    *bytes = attend_ws(d, p->in_dtype, p->out_dtype);
     return HILS_OK;
 }
 
@@ -248,7 +270,7 @@ hils_status hils_forward_workspace_size(const hils_problem *p, size_t *bytes)
     if (!bytes) return HILS_ERR_INVALID_ARG;
     hils_status st = resolve(p, &d);
     if (st != HILS_OK) return st;
-    size_t scratch = select_ws(d) > attend_ws(d, p->in_dtype) ? select_ws(d) : attend_ws(d, p->in_dtype);
+    size_t scratch = select_ws(d) > attend_ws(d, p->in_dtype, p->out_dtype) ? select_ws(d) : attend_ws(d, p->in_dtype, p->out_dtype);
     if (decode_fused_supported(d, p->in_dtype) && decode_fused_ws_bytes(d) > scratch) scratch = decode_fused_ws_bytes(d);
     *bytes = sel_idx_bytes(d) + sel_score_bytes(d) + scratch;
     return HILS_OK;
@@ -279,7 +301,7 @@ hils_status hils_chunk_attend_fuse(const hils_problem *p, const void *Q, const v
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(sel_score) ||
         (sel_idx && !aligned16(sel_idx)))
         return HILS_ERR_INVALID_ARG;
-    st = check_ws(workspace, workspace_bytes, attend_ws(d, p->in_dtype));
+    st = check_ws(workspace, workspace_bytes, attend_ws(d, p->in_dtype, p->out_dtype));
     if (st != HILS_OK) return st;
     if (check_caller_selection()) {
         st = check_selection(d, sel_idx, static_cast<cudaStream_t>(stream));
@@ -338,7 +360,7 @@ hils_status hils_forward_window_workspace_size(const hils_problem *p, int window
     if (!bytes) return HILS_ERR_INVALID_ARG;
     hils_status st = resolve_window(p, window_chunks, &d, &da);
     if (st != HILS_OK) return st;
-    *bytes = sel_idx_bytes(da) + sel_score_bytes(da) + attend_ws(da, p->in_dtype);
+    *bytes = sel_idx_bytes(da) + sel_score_bytes(da) + attend_ws(da, p->in_dtype, p->out_dtype);
     return HILS_OK;
 }
 
@@ -352,7 +374,7 @@ hils_status hils_forward_window(const hils_problem *p, int window_chunks, const 
     if (!Q || !K || !V || !L || !O) return HILS_ERR_INVALID_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(L) || !aligned16(O) || !aligned4(bias))
         return HILS_ERR_INVALID_ARG;
-    const size_t need = sel_idx_bytes(da) + sel_score_bytes(da) + attend_ws(da, p->in_dtype);
+    const size_t need = sel_idx_bytes(da) + sel_score_bytes(da) + attend_ws(da, p->in_dtype, p->out_dtype);
     st = check_ws(workspace, workspace_bytes, need);
     if (st != HILS_OK) return st;
     char *ws = static_cast<char *>(workspace);

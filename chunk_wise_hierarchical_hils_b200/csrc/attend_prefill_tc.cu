@@ -730,9 +730,9 @@ size_t attend_tc_ws_bytes(const Dims &p)
     return v16_bytes(p) + align_up((size_t)p.B * p.Hkv * sizeof(unsigned int), 256);
 }
 
-cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
-                                     const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
-                                     const DeviceCtl &ctl, cudaStream_t s)
+// V converted to f16 into the workspace (the first v16_bytes), and one flag per (b, kv-head) slice
+// that holds a value f16 cannot represent (the next B * Hkv words); the flags are cleared first.
+cudaError_t launch_v_to_f16(const Dims &p, const void *V, void *ws, cudaStream_t s)
 {
     const size_t n16 = (size_t)p.B * p.Hkv * p.T * kD / 8;
     unsigned int *wide = reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + v16_bytes(p));
@@ -740,8 +740,16 @@ cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *
     if (e != cudaSuccess) return e;
     v_to_f16_kernel<<<148 * 8, 256, 0, s>>>(static_cast<const uint4 *>(V), static_cast<uint4 *>(ws), n16,
                                             (size_t)p.T * kD / 8, wide);
-    e = cudaGetLastError();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
+                                     const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
+                                     const DeviceCtl &ctl, cudaStream_t s)
+{
+    cudaError_t e = launch_v_to_f16(p, V, ws, s);
     if (e != cudaSuccess) return e;
+    unsigned int *wide = reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + v16_bytes(p));
     if (out == HILS_F32) return launch_o<float>(p, Q, K, ws, V, wide, sel_idx, sel_score, O, ctl, s);
     return launch_o<__nv_bfloat16>(p, Q, K, ws, V, wide, sel_idx, sel_score, O, ctl, s);
 }

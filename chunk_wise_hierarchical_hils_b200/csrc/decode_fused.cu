@@ -19,7 +19,7 @@
 //   phase 2  the S CTAs read the selection, split its k + 1 slots among themselves, stream their
 //            chunks' key and value tiles through the ring (TMA, 128-byte swizzle, no multicast), and
 //            attend with one warp per chunk on mma.sync tiles (decode_tiles.cuh; warp w takes chunks
-//            w, w + 4, ... from stage w, so each of its barrier waits is one phase ahead); each chunk's softmax
+//            w, w + 5, ... from stage w, so each of its barrier waits is one phase ahead); each chunk's softmax
 //            is normalised on its own and the fusion weights are known, so partial outputs add; with
 //            S > 1 the last CTA of the (b, g) adds the S partials in order.
 // Every wait is bounded: on expiry the CTA records HILS_ERR_TIMEOUT, waits (bounded) for its own
@@ -42,11 +42,11 @@ constexpr int kThreads = 32 * (kWarps + 1);       // sub-partition, so that each
 constexpr int kD = 128, kC = 64;
 constexpr int kLRows = 64;                        // landmark rows per phase-1 stage
 constexpr uint32_t kLStage = kLRows * kD * 2;     // 16 KB
-constexpr int kNL = 8;                            // phase-1 stages
+constexpr int kNL = 10;                           // phase-1 stages
 constexpr uint32_t kHalf = kC * 128;              // one 64-column half of a chunk tile
 constexpr uint32_t kCStage = 4 * kHalf;           // keys then values of one chunk: 32 KB
-constexpr int kNC = 4;                            // phase-2 stages = phase-2 consumer warps
-constexpr uint32_t kRing = 128 * 1024;
+constexpr int kNC = 5;                            // phase-2 stages = phase-2 consumer warps
+constexpr uint32_t kRing = 160 * 1024;
 constexpr int kMaxRows = 4096;                    // landmark rows per CTA
 constexpr unsigned long long kDrainNs = 2000000000ull;
 static_assert(kNL * kLStage <= kRing && kNC * kCStage <= kRing, "stages fit the ring");
@@ -255,30 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (k > 0) block_topk_desc(keys, S * k, k, s_top, hist, ctrl);
         }
     }
-    if (merger) {
-        // the selection and the per-head scores of its k slots and the own chunk; then published
-        for (int j = tid; j < k; j += kThreads) sel_idx[(size_t)bg * k + j] = key_index(s_top[j]);
-        for (int task = tid; task < G * ns; task += kThreads) {
-            const int h = task / ns, j = task % ns;
-            const int c = (j < k) ? key_index(s_top[j]) : ci;
-            float r = -INFINITY;
-            if (c >= 0) {
-                const __nv_bfloat16 *qr = Q + ((size_t)b * p.H + (size_t)g * G + h) * kD;
-                const __nv_bfloat16 *lr = Lbg + (size_t)c * kD;
-                float a0 = 0.f, a1 = 0.f;
-                for (int x = 0; x < kD; x += 2) {
-                    const int i0 = (x + task) & (kD - 1), i1 = (x + 1 + task) & (kD - 1);
-                    a0 = fmaf(__bfloat162float(qr[i0]), __bfloat162float(lr[i0]), a0);
-                    a1 = fmaf(__bfloat162float(qr[i1]), __bfloat162float(lr[i1]), a1);
-                }
-                r = (a0 + a1) * p.scale;
-            }
-            sel_score[((size_t)b * p.H + (size_t)g * G + h) * ns + j] = r;
-        }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0 && S > 1) st_release(&a.ready[bg], 1u);
-    } else if (tid == 0) {
+    if (!merger && tid == 0) {
         // wait for the merge of this (b, g) (bounded: the merging CTA is resident and running)
         const long long t0 = cycle_now();
         while (ld_acquire(&a.ready[bg]) == 0u) {
@@ -297,31 +274,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*abort_flag) return;
 
-    // ---- phase 2: this CTA's slots (j = s, s + S, ...), fusion weights of every head ------------------
-    for (int task = tid; task < G * ns; task += kThreads)
-        wsm[task] = __ldcg(sel_score + ((size_t)b * p.H + (size_t)g * G + task / ns) * ns + task % ns);
+    // ---- phase 2: this CTA's slots (j = s, s + S, ...) ------------------------------------------------
+    // the selection is known: the producer starts the chunk copies at once, while the consumer warps
+    // work out the fusion weights (the merging CTA first computes and publishes the slot scores)
     if (tid == 0) {
         int n = 0;
         for (int j = s; j < ns; j += S) {
-            const int c = (j < k) ? __ldcg(sel_idx + (size_t)bg * k + j) : ci;
+            const int c = (j < k) ? (merger ? key_index(s_top[j]) : __ldcg(sel_idx + (size_t)bg * k + j)) : ci;
             if (c >= 0) slot_c[n++] = (c << 8) | j;
         }
         *s_nmy = n;
-    }
-    __syncthreads();
-    for (int h = warp; h < G; h += kWarps + 1) {
-        float sv[3];
-#pragma unroll
-        for (int u = 0; u < 3; ++u) sv[u] = (lane + 32 * u < ns) ? wsm[h * ns + lane + 32 * u] : -INFINITY;
-        const float mx = warp_max(fmaxf(fmaxf(sv[0], sv[1]), sv[2]));
-        float z = 0.f;
-#pragma unroll
-        for (int u = 0; u < 3; ++u) z += (sv[u] == -INFINITY) ? 0.f : expf(sv[u] - mx);
-        z = warp_sum(z);
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 3; ++u)
-            if (lane + 32 * u < ns) wsm[h * ns + lane + 32 * u] = (sv[u] == -INFINITY) ? 0.f : expf(sv[u] - mx) / z;
     }
     __syncthreads();
     const int n_my = *s_nmy;
@@ -350,24 +312,83 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp < kNC) {
-        const float sl2 = p.scale * 1.4426950408889634f;
-        for (int i = warp; i < n_my; i += kNC) {
-            const int slot = i % kNC;
-            int w_ok = 1;
-            if (lane == 0) w_ok = mbar_wait(FULL2(slot), (uint32_t)((i / kNC) & 1), limit_ns, abort_flag, status);
-            if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
-                *abort_flag = 1;
-                break;
+    } else {
+        constexpr int kCons = 32 * kWarps;   // consumer threads; they meet on named barrier 1
+        if (merger) {
+            // the selection and the per-head scores of its k slots and the own chunk: the slots' landmark
+            // rows staged in shared memory (the keys are no longer needed), every load in flight at once
+            unsigned char *lrows = base + Ly.keys;   // [ns][16 pieces], bf16
+            for (int e = tid; e < ns * 16; e += kCons) {
+                const int j = e >> 4, seg = e & 15;
+                const int c = (j < k) ? key_index(s_top[j]) : ci;
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(Lbg + (size_t)(c >= 0 ? c : 0) * kD) + seg);
+                *reinterpret_cast<uint4 *>(lrows + (size_t)e * 16) = v;
             }
-            const int c = slot_c[i] >> 8, j = slot_c[i] & 255;
-            const int n_vis = (int)min((long long)kC, pos - (long long)c * kC + 1);
-            const float w0 = (gid < G) ? wsm[gid * ns + j] : 0.f;
-            const float w1 = (gid + 8 < G) ? wsm[(gid + 8) * ns + j] : 0.f;
-            const uint32_t kt = ring0 + (uint32_t)slot * kCStage;
-            dtiles::warp_chunk_mma<kC>(smem_addr(qs), kt, kt + 2 * kHalf, n_vis, sl2, w0, w1, oacc);
+            for (int j = tid; j < k; j += kCons) sel_idx[(size_t)bg * k + j] = key_index(s_top[j]);
+            asm volatile("bar.sync 1, %0;" ::"r"(kCons) : "memory");
+            for (int task = tid; task < G * ns; task += kCons) {
+                const int h = task / ns, j = task % ns;
+                const int c = (j < k) ? key_index(s_top[j]) : ci;
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+                for (int u = 0; u < 16; ++u) {
+                    const int seg = (u + j) & 15;   // rotated: threads of different slots, different banks
+                    float qf[8], lf[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(qs + h * kQPitch + seg * 16), qf);
+                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(lrows + ((size_t)j * 16 + seg) * 16), lf);
+#pragma unroll
+                    for (int x = 0; x < 8; x += 2) {
+                        a0 = fmaf(qf[x], lf[x], a0);
+                        a1 = fmaf(qf[x + 1], lf[x + 1], a1);
+                    }
+                }
+                const float r = c >= 0 ? (a0 + a1) * p.scale : -INFINITY;
+                wsm[task] = r;
+                sel_score[((size_t)b * p.H + (size_t)g * G + h) * ns + j] = r;
+            }
+            __threadfence();
+            asm volatile("bar.sync 1, %0;" ::"r"(kCons) : "memory");
+            if (tid == 0 && S > 1) st_release(&a.ready[bg], 1u);
+        } else {
+            for (int task = tid; task < G * ns; task += kCons)
+                wsm[task] = __ldcg(sel_score + ((size_t)b * p.H + (size_t)g * G + task / ns) * ns + task % ns);
+            asm volatile("bar.sync 1, %0;" ::"r"(kCons) : "memory");
+        }
+        // fusion weights of every head: softmax over its slot scores
+        for (int h = warp; h < G; h += kWarps) {
+            float sv[3];
+#pragma unroll
+            for (int u = 0; u < 3; ++u) sv[u] = (lane + 32 * u < ns) ? wsm[h * ns + lane + 32 * u] : -INFINITY;
+            const float mx = warp_max(fmaxf(fmaxf(sv[0], sv[1]), sv[2]));
+            float z = 0.f;
+#pragma unroll
+            for (int u = 0; u < 3; ++u) z += (sv[u] == -INFINITY) ? 0.f : expf(sv[u] - mx);
+            z = warp_sum(z);
             __syncwarp();
-            if (lane == 0) mbar_arrive(EMPTY2(slot));
+#pragma unroll
+            for (int u = 0; u < 3; ++u)
+                if (lane + 32 * u < ns) wsm[h * ns + lane + 32 * u] = (sv[u] == -INFINITY) ? 0.f : expf(sv[u] - mx) / z;
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(kCons) : "memory");
+        if (warp < kNC) {
+            const float sl2 = p.scale * 1.4426950408889634f;
+            for (int i = warp; i < n_my; i += kNC) {
+                const int slot = i % kNC;
+                int w_ok = 1;
+                if (lane == 0) w_ok = mbar_wait(FULL2(slot), (uint32_t)((i / kNC) & 1), limit_ns, abort_flag, status);
+                if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const int c = slot_c[i] >> 8, j = slot_c[i] & 255;
+                const int n_vis = (int)min((long long)kC, pos - (long long)c * kC + 1);
+                const float w0 = (gid < G) ? wsm[gid * ns + j] : 0.f;
+                const float w1 = (gid + 8 < G) ? wsm[(gid + 8) * ns + j] : 0.f;
+                const uint32_t kt = ring0 + (uint32_t)slot * kCStage;
+                dtiles::warp_chunk_mma<kC>(smem_addr(qs), kt, kt + 2 * kHalf, n_vis, sl2, w0, w1, oacc);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(EMPTY2(slot));
+            }
         }
     }
     __syncthreads();

@@ -65,7 +65,18 @@ bool select_q_supported(const Dims &p, hils_dtype in);
 bool select_q_preferred(const Dims &p);   // where it beats the kernel with a row per head
 cudaError_t launch_select_prefill_q(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
                                     const DeviceCtl &ctl, cudaStream_t s);
-size_t attend_tc_ws_bytes(const Dims &p);
+size_t attend_tc_ws_bytes(const Dims &p);   // V as f16 + one flag word per (b, kv-head): launch_v_to_f16's output
+// V (bf16) converted to f16 at the start of ws, and per (b, kv-head) a flag set when a value's magnitude
+// is 65536 or more (the slice then takes a bf16 value product with V as given).
+cudaError_t launch_v_to_f16(const Dims &p, const void *V, void *ws, cudaStream_t s);
+// Chunk-major prefill attention (selection inverted per chunk, tiles of gathered query rows, partial
+// outputs added in L2): bf16, d = 128, C = 64.
+bool attend_cm_supported(const Dims &p, hils_dtype in);
+bool attend_cm_preferred(const Dims &p);
+size_t attend_cm_ws_bytes(const Dims &p, hils_dtype out);
+cudaError_t launch_attend_prefill_cm(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
+                                     const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
+                                     const DeviceCtl &ctl, cudaStream_t s);
 cudaError_t launch_attend_prefill_tc(const Dims &p, hils_dtype out, const void *Q, const void *K, const void *V,
                                      const int32_t *sel_idx, const float *sel_score, void *O, void *ws,
                                      const DeviceCtl &ctl, cudaStream_t s);

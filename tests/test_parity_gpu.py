@@ -70,6 +70,23 @@ def test_cuda_core_kernel_too(w, monkeypatch):
     _check(st)
 
 
+@pytest.mark.parametrize("w", [CASES[1], CASES[3], CASES[5], CASES[6], CASES[7], CASES[8], CASES[9], CASES[10],
+                               CASES[11], CASES[12]], ids=lambda w: w.name)
+def test_chunk_major_attention_too(w, monkeypatch):
+    """The chunk-major tensor-core prefill attention (selection inverted per chunk, gathered query rows,
+    partial outputs added in L2), forced, on shapes the union kernel normally takes."""
+    monkeypatch.setenv("HILS_PREFILL_ATTEND", "chunk")
+    st, _ = parity.run_small(w)
+    _check(st)
+
+
+@pytest.mark.parametrize("attend", ["union", "chunk"])
+def test_both_prefill_attentions_with_bf16_output(attend, monkeypatch):
+    monkeypatch.setenv("HILS_PREFILL_ATTEND", attend)
+    st, _ = parity.run_small(CASES[1], out_dtype="bf16")
+    _check(st)
+
+
 @pytest.mark.parametrize("kernel", ["heads", "queries"])
 @pytest.mark.parametrize("w", [CASES[1], CASES[3], CASES[5], CASES[6], CASES[7], CASES[8], CASES[10], CASES[11],
                                CASES[12]], ids=lambda w: w.name)
@@ -169,7 +186,8 @@ def test_exact_ties_lowest_index():
     _check(st)
 
 
-def test_large_and_tiny_values():
+@pytest.mark.parametrize("attend", ["union", "chunk"])
+def test_large_and_tiny_values(attend, monkeypatch):
     """V entries far outside N(0,1): +-1e5 (beyond f16's range), +-3e4 (inside it) and +-1e-6 (f16
     subnormals), planted in a few chunks of some (b, kv-head) slices, so that most rows of the blocks
     that load those chunks did not select them.  The output is defined for every finite input
@@ -182,6 +200,7 @@ def test_large_and_tiny_values():
     |v| <= 8 only keep the usual 1e-2; rows that attend to a planted large value get 2^-8 times it."""
     from synth import workloads as W
     from synth.philox import f64_to_f32, f32_to_bf16_bits, bf16_bits_to_f64
+    monkeypatch.setenv("HILS_PREFILL_ATTEND", attend)
     w = wl("wide_values", B=2, H=8, Hkv=2, N=1024, T=1024, k=4, seed=140)
     inp = W.full_inputs(w)
     arr = {k: v[0].copy() for k, v in inp.items()}
