@@ -41,6 +41,9 @@ def parse():
                          "and prefill_256k_needles as sub-records of the same line")
     ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--min-timed-ms", type=float, default=500.0,
+                    help="decode and sub-record workloads repeat their step until the timed region lasts this "
+                         "long (so that the clock sampler sees the GPU under load); 0 times exactly --steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-blocks", type=int, default=16, help="64-query blocks in the oracle sample")
     ap.add_argument("--override", nargs="*", default=[], metavar="KEY=VALUE",
@@ -466,8 +469,9 @@ def measure_forward(args, w, ws, rank, local, steps=None):
     # short steps are repeated so that the clock sampler sees the GPU under load (about half a second)
     timer.run(g_step, 2)
     probe_ms = timer.run(g_step, 4) / 4
-    if steps is None or w.N == 1:
-        steps = max(steps or args.steps, int(0.5e3 / max(probe_ms + (0.05 if flush else 0.0), 1e-3)))
+    if (steps is None or w.N == 1) and args.min_timed_ms > 0:
+        steps = max(steps or args.steps, int(args.min_timed_ms / max(probe_ms + (0.05 if flush else 0.0), 1e-3)))
+    steps = steps or args.steps
     sampler = ClockSampler(local)
     barrier(ws)
     torch.cuda.synchronize()
@@ -509,7 +513,7 @@ def measure_forward(args, w, ws, rank, local, steps=None):
         e2e_step()
     torch.cuda.synchronize()
     barrier(ws)
-    e2e_steps = args.e2e_steps if w.N > 1 else max(args.e2e_steps, 100)
+    e2e_steps = args.e2e_steps if (w.N > 1 or args.min_timed_ms <= 0) else max(args.e2e_steps, 100)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):

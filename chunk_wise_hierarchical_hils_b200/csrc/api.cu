@@ -203,6 +203,20 @@ hils_status resolve_window(const hils_problem *p, int wc, Dims *base, Dims *att)
 
 bool aligned4(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
 
+// The windowed, biased selection: prefill on the tensor-core kernel with a row per query where it covers
+// the shape, else (decode, float32, other d or k > 32) the CUDA-core kernel.
+hils_status select_window(const Dims &p, hils_dtype in, int wc, const float *bias, const void *Q, const void *L,
+                          int32_t *sel_idx, float *sel_score, cudaStream_t s)
+{
+    if (p.N > 1 && !force_cuda_cores() && forced_select_kernel() != 1 && select_q_supported(p, in, wc)) {
+        DeviceCtl ctl;
+        hils_status st = device_ctl(&ctl);
+        if (st != HILS_OK) return st;
+        return from_cuda(launch_select_prefill_q(p, Q, L, sel_idx, sel_score, ctl, s, wc, bias));
+    }
+    return from_cuda(launch_select_window(p, in, wc, bias, Q, L, sel_idx, sel_score, s));
+}
+
 }  // namespace
 
 // Prefill dispatch: the tensor-core kernel when it covers the shape, else CUDA cores.
@@ -350,8 +364,8 @@ hils_status hils_score_select_window(const hils_problem *p, int window_chunks, c
     if (!aligned16(Q) || !aligned16(L) || (sel_idx && !aligned16(sel_idx)) || !aligned16(sel_score) ||
         !aligned4(bias))
         return HILS_ERR_INVALID_ARG;
-    return from_cuda(launch_select_window(d, p->in_dtype, window_chunks, bias, Q, L, sel_idx, sel_score,
-                                          static_cast<cudaStream_t>(stream)));
+    return select_window(d, p->in_dtype, window_chunks, bias, Q, L, sel_idx, sel_score,
+                         static_cast<cudaStream_t>(stream));
 }
 
 hils_status hils_forward_window_workspace_size(const hils_problem *p, int window_chunks, size_t *bytes)
@@ -382,7 +396,7 @@ hils_status hils_forward_window(const hils_problem *p, int window_chunks, const 
     float *sel_score = reinterpret_cast<float *>(ws + sel_idx_bytes(da));
     void *scratch = ws + sel_idx_bytes(da) + sel_score_bytes(da);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = from_cuda(launch_select_window(d, p->in_dtype, window_chunks, bias, Q, L, sel_idx, sel_score, s));
+    st = select_window(d, p->in_dtype, window_chunks, bias, Q, L, sel_idx, sel_score, s);
     if (st != HILS_OK) return st;
     return do_attend(da, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, scratch, s);
 }

@@ -61,10 +61,11 @@ bool select_tc_supported(const Dims &p, hils_dtype in);
 cudaError_t launch_select_prefill_tc(const Dims &p, const void *Q, const void *L, int32_t *sel_idx,
                                      float *sel_score, const DeviceCtl &ctl, cudaStream_t s);
 // Prefill selection with one product row per query (group score from the mean query): bf16, d = 128, k <= 32.
-bool select_q_supported(const Dims &p, hils_dtype in);
+// With wc > 1 or a bias [B][Hkv][nL] it writes the windowed selection (k + wc - 1 past slots per row).
+bool select_q_supported(const Dims &p, hils_dtype in, int wc = 1);
 bool select_q_preferred(const Dims &p);   // where it beats the kernel with a row per head
 cudaError_t launch_select_prefill_q(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
-                                    const DeviceCtl &ctl, cudaStream_t s);
+                                    const DeviceCtl &ctl, cudaStream_t s, int wc = 1, const float *bias = nullptr);
 size_t attend_tc_ws_bytes(const Dims &p);   // V as f16 + one flag word per (b, kv-head): launch_v_to_f16's output
 // V (bf16) converted to f16 at the start of ws, and per (b, kv-head) a flag set when a value's magnitude
 // is 65536 or more (the slice then takes a bf16 value product with V as given).

@@ -21,6 +21,13 @@
 // network.  Ties go to the lower chunk index through the key order.  After the scan, the per-head
 // scores of the k selected slots and the own chunk (the fusion scores the attention needs) are
 // computed on CUDA cores from the query rows staged in shared memory.
+//
+// The same kernel serves the local window and the per-chunk bias of the retrieval score (Sec. 2
+// Preliminary and Sec. 5 "Experimental setup": a chunk-aligned window of the own chunk and the wc - 1
+// chunks before it is always attended, and retrieval ranks only the chunks before it; Sec. 3 "Linear
+// surrogate for chunk mass": the bias of chunk c is added to every head's score of c): the candidates
+// are c <= c_i - wc, the bias is added to each candidate's group score and to every slot score, and a
+// row holds k + wc - 1 past slots (the retrieved chunks, then the window's past chunks ascending).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -50,7 +57,7 @@ struct Layout {
 
 // Shared memory: qbar (64 KB), the landmark stages, barriers, the candidate queue, then the rows'
 // selected chunks.  After the scan the first kQbarBytes + kNSL * kTileBytes bytes hold query rows.
-__host__ __device__ inline Layout make_layout(int k)
+__host__ __device__ inline Layout make_layout(int k, int wc = 1)
 {
     Layout L;
     L.qbar = 0;
@@ -59,7 +66,7 @@ __host__ __device__ inline Layout make_layout(int k)
     L.misc = L.bar + 16 * 8;
     L.queue = L.misc + 16;
     L.selc = L.queue + 8u * kQueue * kRows;
-    L.total = L.selc + 4u * (uint32_t)(k + 1) * kRows;
+    L.total = L.selc + 4u * (uint32_t)(k + wc) * kRows;
     return L;
 }
 static_assert(kHeadBatch * kRows * kD * 2 <= kQbarBytes + kNSL * kTileBytes, "query rows fit the freed stages");
@@ -103,24 +110,25 @@ __device__ __forceinline__ void list_sort_desc(uint64_t (&a)[RK])
     }
 }
 
-template <int RK>
+template <int RK, bool BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
     select_q_kernel(const __grid_constant__ CUtensorMap tmL, Dims p, const __nv_bfloat16 *__restrict__ Q,
                     const __nv_bfloat16 *__restrict__ Lm, int32_t *__restrict__ sel_idx,
-                    float *__restrict__ sel_score, unsigned int *status, unsigned long long limit_ns)
+                    float *__restrict__ sel_score, int wc, const float *__restrict__ bias, unsigned int *status,
+                    unsigned long long limit_ns)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    const Layout Ly = make_layout(p.k);
-    const int G = p.G, ns = p.k + 1;
+    const Layout Ly = make_layout(p.k, wc);
+    const int G = p.G, ns = p.k + wc, kp = p.k + wc - 1;   // slots per row; past slots per row
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q0 = blockIdx.x * kRows, g = blockIdx.y, b = blockIdx.z;
     const int nq = min(kRows, p.N - q0);
     const int c_hi = (int)(((long long)p.q_offset + q0 + nq - 1) / p.C);   // own chunk of the last query
-    // candidates are chunks c < c_i <= c_hi; without any (k = 0, or the block's queries all in chunk
-    // 0) the scan is skipped and only the own chunk's slot score is written
-    const int n_tiles = (p.k > 0 && c_hi > 0) ? (c_hi - 1) / kTile + 1 : 0;
+    // candidates are chunks c <= c_i - wc <= c_hi - wc; without any (k = 0, or the block's queries all
+    // inside their first wc chunks) the scan is skipped and only the window's slot scores are written
+    const int n_tiles = (p.k > 0 && c_hi - wc >= 0) ? (c_hi - wc) / kTile + 1 : 0;
     const int ksteps = G == 1 ? 8 : 16;   // with one head qbar = q is exact in bf16: lo = 0
 
     const uint32_t sQ = smem_addr(base + Ly.qbar), sL = smem_addr(base + Ly.l), bar0 = smem_addr(base + Ly.bar);
@@ -128,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 8);
     uint64_t *queue = reinterpret_cast<uint64_t *>(base + Ly.queue);
     int *selc = reinterpret_cast<int *>(base + Ly.selc);
+    const float *bias_bg = BIAS ? bias + ((size_t)b * p.Hkv + g) * p.nL : nullptr;
     auto L_FULL = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto L_EMPTY = [&](int s) { return bar0 + 8u * (uint32_t)(kNSL + s); };
     auto S_FULL = [&](int s) { return bar0 + 8u * (uint32_t)(2 * kNSL + s); };
@@ -264,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid = r < nq;
         const long long pos = (long long)p.q_offset + q0 + r;
         const int ci = (int)(pos / p.C);
+        const int c_lim = ci - wc + 1;   // candidates c < c_lim
         const uint32_t trow = tmem + ((uint32_t)(32 * qq) << 16);
         uint64_t *hk = queue + r;
         uint64_t top[RK];
@@ -289,6 +299,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) mbar_arrive(S_FREE(t & 1));
                 }
                 const int cb = t * kTile + 32 * part;
+                float bv[BIAS ? 32 : 1];   // the 32 chunks' biases (the same address in every lane: broadcast)
+                if constexpr (BIAS) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) bv[j] = cb + j < p.nL ? __ldg(bias_bg + cb + j) : 0.f;
+                }
                 int qn = 0;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
@@ -310,8 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         qn = 0;
                     }
                     const int c = cb + j;
-                    const uint64_t key = make_key(__uint_as_float(sv[j]) * p.scale, c);
-                    if (valid && c < ci && key > top[RK - 1]) {
+                    float sc = __uint_as_float(sv[j]) * p.scale;
+                    if constexpr (BIAS) sc += bv[j];
+                    const uint64_t key = make_key(sc, c);
+                    if (valid && c < c_lim && key > top[RK - 1]) {
                         hk[qn * kRows] = key;
                         ++qn;
                     }
@@ -324,18 +341,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (!ok) *abort_flag = 1;
-        // the selection: chunk indices in rank order (k < RK: the list's first k keys), own chunk last
+        // the selection: chunk indices in rank order (k < RK: the list's first k keys), then the window's
+        // past chunks ascending, own chunk last
         if (valid) {
             const size_t row_g = (((size_t)b * p.Hkv + g) * p.N) + q0 + r;
 #pragma unroll
             for (int j = 0; j < RK; ++j) {
                 if (j < p.k) {
                     const int c = key_index(top[j]);
-                    sel_idx[row_g * p.k + j] = c;
+                    sel_idx[row_g * kp + j] = c;
                     selc[r * ns + j] = c;
                 }
             }
-            selc[r * ns + p.k] = ci;
+            for (int j = p.k; j < kp; ++j) {
+                const int c = ci - wc + 1 + (j - p.k);
+                sel_idx[row_g * kp + j] = c >= 0 ? c : -1;
+                selc[r * ns + j] = c >= 0 ? c : -1;
+            }
+            selc[r * ns + kp] = ci;
         }
     }
     tc_fence_before();
@@ -403,7 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int hh = 0; hh < kHeadBatch; ++hh) {
                 if (hh < hb) {
                     const size_t row_h = (((size_t)b * p.H + (size_t)g * G + h0 + hh) * p.N) + q0 + qi;
-                    sel_score[row_h * ns + j] = c >= 0 ? acc[hh] * p.scale : -INFINITY;
+                    sel_score[row_h * ns + j] =
+                        c >= 0 ? acc[hh] * p.scale + (BIAS ? __ldg(bias_bg + c) : 0.f) : -INFINITY;
                 }
             }
         }
@@ -433,10 +457,10 @@ EncodeTiledFn encode_fn()
 // computes afterwards on CUDA cores; the kernel with one row per head gets those with the scan.  So
 // this one is used where the scan dominates: k above 16 (the other kernel keeps larger lists in a
 // shared-memory heap) or more than 512 visible chunks.
-bool select_q_supported(const Dims &p, hils_dtype in)
+bool select_q_supported(const Dims &p, hils_dtype in, int wc)
 {
-    if (in != HILS_BF16 || p.d != kD || p.N < 2 || p.k > 32) return false;
-    return make_layout(p.k).total + 1024 <= 227 * 1024;
+    if (in != HILS_BF16 || p.d != kD || p.N < 2 || p.k > 32 || wc < 1) return false;
+    return make_layout(p.k, wc).total + 1024 <= 227 * 1024;
 }
 
 bool select_q_preferred(const Dims &p)
@@ -446,7 +470,7 @@ bool select_q_preferred(const Dims &p)
 }
 
 cudaError_t launch_select_prefill_q(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
-                                    const DeviceCtl &ctl, cudaStream_t s)
+                                    const DeviceCtl &ctl, cudaStream_t s, int wc, const float *bias)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorInvalidValue;
@@ -459,20 +483,23 @@ cudaError_t launch_select_prefill_q(const Dims &p, const void *Q, const void *L,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const size_t smem = make_layout(p.k).total + 1024;
+    const size_t smem = make_layout(p.k, wc).total + 1024;
     dim3 grid((p.N + kRows - 1) / kRows, p.Hkv, p.B);
     cudaError_t e;
-#define HILS_LAUNCH_SELQ(RKV)                                                                                \
+#define HILS_LAUNCH_SELQ(RKV, BV)                                                                            \
     {                                                                                                        \
-        auto kern = select_q_kernel<RKV>;                                                                    \
+        auto kern = select_q_kernel<RKV, BV>;                                                                \
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);              \
         if (e != cudaSuccess) return e;                                                                      \
         kern<<<grid, kThreads, smem, s>>>(tl, p, static_cast<const __nv_bfloat16 *>(Q),                      \
-                                          static_cast<const __nv_bfloat16 *>(L), sel_idx, sel_score,         \
-                                          ctl.status, (unsigned long long)ctl.wait_limit);                   \
+                                          static_cast<const __nv_bfloat16 *>(L), sel_idx, sel_score, wc,     \
+                                          bias, ctl.status, (unsigned long long)ctl.wait_limit);             \
     }
-    if (p.k <= 16) HILS_LAUNCH_SELQ(16)
-    else HILS_LAUNCH_SELQ(32)
+    if (p.k <= 16) {
+        if (bias) HILS_LAUNCH_SELQ(16, true) else HILS_LAUNCH_SELQ(16, false)
+    } else {
+        if (bias) HILS_LAUNCH_SELQ(32, true) else HILS_LAUNCH_SELQ(32, false)
+    }
 #undef HILS_LAUNCH_SELQ
     return cudaGetLastError();
 }

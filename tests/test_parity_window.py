@@ -108,6 +108,18 @@ def _oracle_on_selection(w, wc, arr, bias, b, g, i, slots):
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: c[0].name)
 def test_window_and_bias_match_the_oracle(case):
+    _check_window_case(case)
+
+
+@pytest.mark.parametrize("case", [c for c in CASES if c[0].N > 1 and c[0].dtype == "bf16"], ids=lambda c: c[0].name)
+def test_window_on_the_cuda_core_selection_too(case, monkeypatch):
+    """The bf16 prefill window selection normally runs on the tensor-core kernel with a row per query;
+    the CUDA-core kernel (forced here) must agree with the oracle as well."""
+    monkeypatch.setenv("HILS_SELECT_KERNEL", "heads")
+    _check_window_case(case)
+
+
+def _check_window_case(case):
     w, wc, bias_scale = case
     arr, bias, ref, sel, s, O = _run(w, wc, bias_scale)
     kp = w.k + wc - 1
