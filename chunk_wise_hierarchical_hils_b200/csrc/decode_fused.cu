@@ -30,6 +30,7 @@
 #include "common.cuh"
 #include "decode_tiles.cuh"
 #include "sm100.cuh"
+#include "warp_topk.cuh"
 
 namespace hils {
 namespace {
@@ -54,7 +55,7 @@ static_assert(kNC * 16 * kD * 4 <= kRing, "the warps' partial outputs fit the ri
 static_assert(kNC <= kWarps, "a consumer warp per phase-2 stage");
 
 struct Layout {
-    uint32_t ring, keys, qs, qbar, wsm, slot_c, top, hist, ctrl, bars, misc, total;
+    uint32_t ring, keys, qs, qbar, wsm, slot_c, top, wl, bars, misc, total;
 };
 
 __host__ __device__ inline Layout make_layout()
@@ -67,9 +68,8 @@ __host__ __device__ inline Layout make_layout()
     L.wsm = L.qbar + kD * 4;
     L.slot_c = L.wsm + HILS_MAX_GROUP * (HILS_MAX_K + 1) * 4;
     L.top = (L.slot_c + (HILS_MAX_K + 1) * 4 + 7) & ~7u;
-    L.hist = L.top + HILS_MAX_K * 8;
-    L.ctrl = L.hist + 256 * 4;
-    L.bars = L.ctrl + 4 * 8;
+    L.wl = L.top + HILS_MAX_K * 8;
+    L.bars = L.wl + kWarps * HILS_MAX_K * 8;
     L.misc = L.bars + (2 * kNL + 2 * kNC) * 8;
     L.total = L.misc + 32;
     return L;
@@ -97,7 +97,34 @@ __device__ __forceinline__ void st_release(unsigned int *p, unsigned int v)
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-template <typename Tout>
+// The k largest of n keys (kWarps warps each keep a list over a strided share, warp 0 merges the
+// lists) into out[0 .. 32 KR), descending; every thread of the block calls it.
+template <int KR>
+__device__ __forceinline__ void topk_warps(const uint64_t *keys, int n, uint64_t *wl, uint64_t *out)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < kWarps) {
+        wtopk::List<KR> L;
+        L.clear();
+        for (int e0 = warp * 32; e0 < n; e0 += kWarps * 32) L.add(e0 + lane < n ? keys[e0 + lane] : 0ull);
+#pragma unroll
+        for (int r = 0; r < KR; ++r) wl[warp * 64 + r * 32 + lane] = L.v[r];
+    }
+    __syncthreads();
+    if (warp == 0) {
+        wtopk::List<KR> L;
+#pragma unroll
+        for (int r = 0; r < KR; ++r) L.v[r] = wl[r * 32 + lane];
+        for (int w = 1; w < kWarps; ++w)
+#pragma unroll
+            for (int r = 0; r < KR; ++r) L.add(wl[w * 64 + r * 32 + lane]);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) out[r * 32 + lane] = r < KR ? L.v[r] : 0ull;
+    }
+    __syncthreads();
+}
+
+template <typename Tout, int KR>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Dims p,
                         FusedArgs a, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ Lm,
@@ -113,8 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *wsm = reinterpret_cast<float *>(base + Ly.wsm);
     int *slot_c = reinterpret_cast<int *>(base + Ly.slot_c);
     uint64_t *s_top = reinterpret_cast<uint64_t *>(base + Ly.top);
-    unsigned int *hist = reinterpret_cast<unsigned int *>(base + Ly.hist);
-    unsigned long long *ctrl = reinterpret_cast<unsigned long long *>(base + Ly.ctrl);
+    uint64_t *wl = reinterpret_cast<uint64_t *>(base + Ly.wl);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc);
     int *s_flag = reinterpret_cast<int *>(base + Ly.misc + 4);
     int *s_nmy = reinterpret_cast<int *>(base + Ly.misc + 8);
@@ -237,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // local top-k, then the merge by the last CTA of the (b, g)
-    block_topk_desc(keys, n_local, min(k, max(n_local, 1)), s_top, hist, ctrl);
+    topk_warps<KR>(keys, n_local, wl, s_top);
     bool merger = true;
     if (S > 1) {
         uint64_t *mine = a.cand + ((size_t)bg * S + s) * k;
@@ -252,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t *all = a.cand + (size_t)bg * S * k;
             for (int e = tid; e < S * k; e += kThreads) keys[e] = __ldcg(all + e);
             __syncthreads();
-            if (k > 0) block_topk_desc(keys, S * k, k, s_top, hist, ctrl);
+            topk_warps<KR>(keys, S * k, wl, s_top);
         }
     }
     if (!merger && tid == 0) {
@@ -525,19 +551,20 @@ cudaError_t launch_decode_fused(const Dims &p, hils_dtype out, const void *Q, co
     cfg.numAttrs = 1;
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(Q), *l = static_cast<const __nv_bfloat16 *>(L);
     const unsigned long long lim = (unsigned long long)ctl.wait_limit;
-    if (out == HILS_F32) {
-        auto kern = decode_fused_kernel<float>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        e = cudaLaunchKernelEx(&cfg, kern, tk, tv, p, a, q, l, sel_idx, sel_score, static_cast<float *>(O), ctl.status,
-                               lim);
-    } else {
-        auto kern = decode_fused_kernel<__nv_bfloat16>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        e = cudaLaunchKernelEx(&cfg, kern, tk, tv, p, a, q, l, sel_idx, sel_score, static_cast<__nv_bfloat16 *>(O),
-                               ctl.status, lim);
+#define HILS_LAUNCH_FUSED(TOUT, KRV)                                                                         \
+    {                                                                                                        \
+        auto kern = decode_fused_kernel<TOUT, KRV>;                                                          \
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);              \
+        if (e != cudaSuccess) return e;                                                                      \
+        e = cudaLaunchKernelEx(&cfg, kern, tk, tv, p, a, q, l, sel_idx, sel_score, static_cast<TOUT *>(O),   \
+                               ctl.status, lim);                                                             \
     }
+    if (out == HILS_F32) {
+        if (p.k <= 32) HILS_LAUNCH_FUSED(float, 1) else HILS_LAUNCH_FUSED(float, 2)
+    } else {
+        if (p.k <= 32) HILS_LAUNCH_FUSED(__nv_bfloat16, 1) else HILS_LAUNCH_FUSED(__nv_bfloat16, 2)
+    }
+#undef HILS_LAUNCH_FUSED
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
