@@ -18,10 +18,13 @@
 //              (TMA), computes S = Q K^T (tcgen05, M = 128 rows, N = 64 keys) into TMEM; the softmax warps
 //              write P = w_c softmax(S) (the fusion weight folded in, f16) to shared memory; then
 //              O^T = V^T P^T (tcgen05, M = d = 128, N = 128 rows, K = 64 keys), so that TMEM lane x
-//              holds column x of every row's chunk output; the epilogue warps add it into a float32
-//              accumulator with one coalesced 128-byte reduction per warp and row;
+//              holds column x of every row's chunk output; the epilogue warps copy it, half a tile at
+//              a time, into the tile's query buffer (free once S is computed) as rows of d floats, and
+//              one thread adds each query's G rows into a float32 accumulator [B][Hkv][N][G][d] with a
+//              single bulk reduction (cp.reduce.async.bulk ... add.f32, G * d * 4 bytes, no multicast);
 //   ordering   tiles go (kv-group, query range, chunk): the accumulator rows of one query range
-//              (about 32 MB) stay in L2 while its tiles run, so the reductions do not reach HBM.
+//              (about 32 MB) stay in L2 while its tiles run, so the reductions do not reach HBM;
+//   finalize   the accumulator is permuted to O [B][H][N][d] in the output type.
 // Each chunk's softmax is normalised on its own and the fusion weights are known, so the partial
 // outputs simply add (in no fixed order: the last bits of the float32 sums may differ between runs).
 // A slice of V holding a value f16 cannot represent takes the bf16 value product (V as given).
@@ -56,7 +59,8 @@ constexpr uint32_t IDESC_PV_BF16 = idesc_bf16_f32(128, 128, true, false);
 constexpr uint32_t OFF_Q = 0;                               // 2 query tiles
 constexpr uint32_t OFF_KV = OFF_Q + 2 * kQTile;             // 2 key/value tiles
 constexpr uint32_t OFF_P = OFF_KV + 2 * kKVTile;            // 2 probability tiles
-constexpr uint32_t OFF_RQ = OFF_P + 2 * kPTile;             // [2][128] int: accumulator row, -1 = none
+constexpr uint32_t OFF_RQ = OFF_P + 2 * kPTile;             // [2][128] int: per tile query q: its accumulator
+                                                            // block (b Hkv + g) N + i, -1 = none
 constexpr uint32_t OFF_RW = OFF_RQ + 2 * kRows * 4;         // [2][128] float: fusion weight
 constexpr uint32_t OFF_RN = OFF_RW + 2 * kRows * 4;         // [2][128] int: visible keys
 constexpr uint32_t OFF_BAR = OFF_RN + 2 * kRows * 4;
@@ -76,6 +80,28 @@ enum {
     B_KVPFREE = 16,  // value product done: key/value tile and P tile free (MMA commit)
     B_MMADONE = 18
 };
+
+// the epilogue's four warps meet on named barrier 3; the OR of their flags says whether any stops
+__device__ __forceinline__ bool epilogue_bar_any(bool flag)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 3, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(flag ? 1u : 0u)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, uint32_t src, uint32_t bytes)
+{
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+                 ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
 
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, unsigned long long lim, volatile int *abort_flag,
                                           unsigned int *status)
@@ -247,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 nvis = own ? (int)(pos - (long long)c * kC + 1) : kC;
                 wt = __expf(__ldg(sel_score + (size_t)row * ns + j) - __ldg(lse + row));
             }
-            rq[b * kRows + r] = row;
+            if (h == 0) rq[b * kRows + ql] = i >= 0 ? bg * p.N + i : -1;
             rw[b * kRows + r] = wt;
             rn[b * kRows + r] = nvis;
             mbar_arrive(BAR(B_ROW + b));
@@ -307,31 +333,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(BAR(B_PFULL + b));
         }
     } else if (warp >= 12) {
-        // ---- epilogue: lane x of warp e holds column 32 e + x of every row's chunk output; each row is
-        // added into the accumulator by one coalesced 128-byte reduction of the warp
+        // ---- epilogue: lane x of warp e holds column 32 e + x of every row's chunk output.  Half a tile
+        // (64 rows) at a time: rows of d floats into the tile's query buffer, then one bulk reduction per
+        // query (its G rows, contiguous in the buffer and in the accumulator)
         const int e = warp & 3;
         const uint32_t lane_off = (uint32_t)(32 * e) << 16;
+        const int Gq = p.G;
         for (int t = 0; tile_of(t) < n_tiles; ++t) {
             const int b = t & 1;
             const uint32_t ph = (uint32_t)((t >> 1) & 1);
-            if (!wait_warp(BAR(B_OFULL + b), ph, limit_ns, abort_flag, status)) break;
-            if (!wait_warp(BAR(B_ROW + b), ph, limit_ns, abort_flag, status)) break;
+            bool ok = wait_warp(BAR(B_OFULL + b), ph, limit_ns, abort_flag, status) &&
+                      wait_warp(BAR(B_ROW + b), ph, limit_ns, abort_flag, status);
+            if (epilogue_bar_any(!ok || *abort_flag)) break;
             tc_fence_after();
+            float *stage = reinterpret_cast<float *>(base + OFF_Q + (size_t)b * kQTile);   // [64][kD]
+            const uint32_t stage_s = sQ + (uint32_t)b * kQTile;
+            for (int half = 0; half < 2; ++half) {
 #pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_off + kColO + (uint32_t)b * 128u + 32u * (uint32_t)cb, v);
-                tmem_wait_ld();
+                for (int cb = 0; cb < 2; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_off + kColO + (uint32_t)b * 128u + 64u * (uint32_t)half + 32u * (uint32_t)cb, v);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    const int row = rq[b * kRows + 32 * cb + x];
-                    if (row >= 0) atomicAdd(acc + (size_t)row * kD + 32 * e + lane, __uint_as_float(v[x]));
+                    for (int x = 0; x < 32; ++x) stage[(32 * cb + x) * kD + 32 * e + lane] = __uint_as_float(v[x]);
                 }
+                fence_proxy_async_smem();
+                epilogue_bar_any(false);
+                if (warp == 12 && lane == 0) {
+                    const int q0 = 64 * half / Gq, q1 = 64 * (half + 1) / Gq;
+                    for (int q = q0; q < q1; ++q) {
+                        const int blk = rq[b * kRows + q];
+                        if (blk >= 0)
+                            bulk_reduce_add_f32(acc + (size_t)blk * Gq * kD, stage_s + (uint32_t)((q * Gq - 64 * half) * kD * 4),
+                                                (uint32_t)(Gq * kD * 4));
+                    }
+                    asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group.read 0;" ::: "memory");
+                }
+                epilogue_bar_any(false);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR(B_OFREE + b));
         }
+        if (warp == 12 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
@@ -478,15 +522,29 @@ __global__ void cm_scatter_kernel(Dims p, int RQ, int R, const int32_t *__restri
     }
 }
 
-// float32 accumulator -> bf16 output, 8 elements per thread step
-__global__ void cm_finalize_kernel(const float4 *__restrict__ acc, uint4 *__restrict__ out, size_t n8)
+// the accumulator [B][Hkv][N][G][d] (float32) -> O [B][H][N][d], 8 elements per thread step
+template <typename Tout>
+__global__ void cm_finalize_kernel(Dims p, const float4 *__restrict__ acc, Tout *__restrict__ O)
 {
+    const size_t n8 = (size_t)p.B * p.H * p.N * kD / 8;
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n8; e += (size_t)gridDim.x * blockDim.x) {
-        const float4 a = __ldg(acc + 2 * e), z = __ldg(acc + 2 * e + 1);
-        __nv_bfloat162 v0 = __floats2bfloat162_rn(a.x, a.y), v1 = __floats2bfloat162_rn(a.z, a.w),
-                       v2 = __floats2bfloat162_rn(z.x, z.y), v3 = __floats2bfloat162_rn(z.z, z.w);
-        out[e] = make_uint4(*reinterpret_cast<uint32_t *>(&v0), *reinterpret_cast<uint32_t *>(&v1),
-                            *reinterpret_cast<uint32_t *>(&v2), *reinterpret_cast<uint32_t *>(&v3));
+        const size_t o = e * 8, row = o / kD;           // O row (b H + h) N + i
+        const int x = (int)(o % kD);
+        const int i = (int)(row % p.N), bh = (int)(row / p.N), b = bh / p.H, h = bh % p.H;
+        const int g = h / p.G, hh = h % p.G;
+        const size_t src = ((((size_t)b * p.Hkv + g) * p.N + i) * p.G + hh) * kD + x;
+        const float4 a = __ldg(acc + src / 4), z = __ldg(acc + src / 4 + 1);
+        if constexpr (sizeof(Tout) == 4) {
+            float4 *dst = reinterpret_cast<float4 *>(O + o);
+            dst[0] = a;
+            dst[1] = z;
+        } else {
+            __nv_bfloat162 v0 = __floats2bfloat162_rn(a.x, a.y), v1 = __floats2bfloat162_rn(a.z, a.w),
+                           v2 = __floats2bfloat162_rn(z.x, z.y), v3 = __floats2bfloat162_rn(z.z, z.w);
+            *reinterpret_cast<uint4 *>(O + o) =
+                make_uint4(*reinterpret_cast<uint32_t *>(&v0), *reinterpret_cast<uint32_t *>(&v1),
+                           *reinterpret_cast<uint32_t *>(&v2), *reinterpret_cast<uint32_t *>(&v3));
+        }
     }
 }
 
@@ -516,7 +574,7 @@ CmWs cm_ws(const Dims &p, hils_dtype out, void *ws)
     w.lse = reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * 4));
     w.entries = reinterpret_cast<int *>(take((size_t)p.B * p.Hkv * p.N * p.k * 4 + 4));
     w.tiles = reinterpret_cast<int4 *>(take((size_t)c.max_tiles * 16));
-    w.acc = out == HILS_F32 ? nullptr : reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * kD * 4));
+    w.acc = reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * kD * 4));
     w.total = off;
     return w;
 }
@@ -554,7 +612,7 @@ cudaError_t launch_attend_prefill_cm(const Dims &p, hils_dtype out, const void *
     if (e != cudaSuccess) return e;
     const unsigned int *wide = reinterpret_cast<const unsigned int *>(
         static_cast<char *>(ws) + align_up((size_t)p.B * p.Hkv * p.T * kD * 2, 256));
-    float *acc = out == HILS_F32 ? static_cast<float *>(O) : w.acc;
+    float *acc = w.acc;
     const long long groups = (long long)p.B * p.Hkv * p.N;
     e = cudaMemsetAsync(w.cnt, 0, (size_t)c.M * 4, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(acc, 0, (size_t)p.B * p.H * p.N * kD * 4, s);
@@ -586,9 +644,12 @@ cudaError_t launch_attend_prefill_cm(const Dims &p, hils_dtype out, const void *
                                                         w.lse, w.entries, w.tiles, w.n_tiles, wide, acc, ctl.status,
                                                         (unsigned long long)ctl.wait_limit);
     e = cudaGetLastError();
-    if (e != cudaSuccess || out == HILS_F32) return e;
-    const size_t n8 = (size_t)p.B * p.H * p.N * kD / 8;
-    cm_finalize_kernel<<<148 * 8, 256, 0, s>>>(reinterpret_cast<const float4 *>(acc), static_cast<uint4 *>(O), n8);
+    if (e != cudaSuccess) return e;
+    if (out == HILS_F32)
+        cm_finalize_kernel<float><<<148 * 8, 256, 0, s>>>(p, reinterpret_cast<const float4 *>(acc), static_cast<float *>(O));
+    else
+        cm_finalize_kernel<__nv_bfloat16>
+            <<<148 * 8, 256, 0, s>>>(p, reinterpret_cast<const float4 *>(acc), static_cast<__nv_bfloat16 *>(O));
     return cudaGetLastError();
 }
 
