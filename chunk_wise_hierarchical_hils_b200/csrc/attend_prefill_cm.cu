@@ -63,7 +63,8 @@ constexpr uint32_t OFF_RQ = OFF_P + 2 * kPTile;             // [2][128] int: per
                                                             // block (b Hkv + g) N + i, -1 = none
 constexpr uint32_t OFF_RW = OFF_RQ + 2 * kRows * 4;         // [2][128] float: fusion weight
 constexpr uint32_t OFF_RN = OFF_RW + 2 * kRows * 4;         // [2][128] int: visible keys
-constexpr uint32_t OFF_BAR = OFF_RN + 2 * kRows * 4;
+constexpr uint32_t OFF_TM = OFF_RN + 2 * kRows * 4;          // [2] int4: the tile's kv-group, chunk, -, V flag
+constexpr uint32_t OFF_BAR = OFF_TM + 2 * 16;
 constexpr uint32_t OFF_MISC = OFF_BAR + 32 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
 
@@ -114,7 +115,7 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, unsigne
 __global__ void __launch_bounds__(kThreads, 1)
     attend_cm_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV16,
                      const __grid_constant__ CUtensorMap tmVb, Dims p, const __nv_bfloat16 *__restrict__ Q,
-                     const float *__restrict__ sel_score, const float *__restrict__ lse,
+                     const float *__restrict__ ew, const float *__restrict__ ow,
                      const int *__restrict__ entries, const int4 *__restrict__ tiles, const int *__restrict__ n_tiles_p,
                      const unsigned int *__restrict__ wide_flags, float *__restrict__ acc, unsigned int *status,
                      unsigned long long limit_ns)
@@ -126,12 +127,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *rq = reinterpret_cast<int *>(base + OFF_RQ);
     float *rw = reinterpret_cast<float *>(base + OFF_RW);
     int *rn = reinterpret_cast<int *>(base + OFF_RN);
+    int4 *tm = reinterpret_cast<int4 *>(base + OFF_TM);
     const uint32_t bar0 = smem_addr(base + OFF_BAR);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + OFF_MISC + 4);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
     const int n_tiles = __ldg(n_tiles_p);
-    const int ns = p.k + 1, G = p.G;
+    const int G = p.G;
     auto tile_of = [&](int t) { return (int)blockIdx.x + t * (int)gridDim.x; };
 
     if (tid == 0) {
@@ -214,8 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(BAR(B_PFULL + b), ph, limit_ns, abort_flag, status)) return false;
                 if (t >= 2 && !mbar_wait(BAR(B_OFREE + b), ph ^ 1u, limit_ns, abort_flag, status)) return false;
                 tc_fence_after();
-                const int4 d = __ldg(tiles + tile_of(t));
-                const uint32_t idesc = __ldg(wide_flags + d.x) ? IDESC_PV_BF16 : IDESC_PV;
+                const uint32_t idesc = tm[b].w ? IDESC_PV_BF16 : IDESC_PV;   // published with the rows
                 const uint32_t va = sKV + (uint32_t)b * kKVTile + 16384u, pa = sP + (uint32_t)b * kPTile;
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
@@ -254,24 +255,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 d = __ldg(tiles + tile_of(t));
             const int bg = d.x, c = d.y & ~kOwnBit, own = (d.y & kOwnBit) != 0, start = d.z, count = d.w;
             const int bb = bg / p.Hkv, g = bg % p.Hkv;
-            int i = -1, j = p.k;
+            const int hh = g * G + h;
+            int i = -1;
+            float wt = 0.f;
             if (ql < count) {
                 if (own) {
                     i = start + ql;
+                    wt = __ldg(ow + ((size_t)bb * p.H + hh) * p.N + i);
                 } else {
+                    // the entry and its fusion weights come from the inversion, loaded together
                     const int e = __ldg(entries + start + ql);
+                    wt = __ldg(ew + (size_t)(start + ql) * G + h);
                     i = e >> 6;
-                    j = e & 63;
                 }
             }
-            const int hh = g * G + h;
+            if (r == 0) tm[b] = make_int4(bg, c, own, (int)__ldg(wide_flags + bg));
             int row = -1, nvis = 0;
-            float wt = 0.f;
             if (i >= 0) {
                 row = (bb * p.H + hh) * p.N + i;
                 const long long pos = (long long)p.q_offset + i;
                 nvis = own ? (int)(pos - (long long)c * kC + 1) : kC;
-                wt = __expf(__ldg(sel_score + (size_t)row * ns + j) - __ldg(lse + row));
             }
             if (h == 0) rq[b * kRows + ql] = i >= 0 ? bg * p.N + i : -1;
             rw[b * kRows + r] = wt;
@@ -314,8 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(BAR(B_SFREE + b));
             const float w = rw[b * kRows + r];
             const int nvis = rn[b * kRows + r];
-            const int4 d = __ldg(tiles + tile_of(t));
-            const bool wide = __ldg(wide_flags + d.x) != 0u;
+            const bool wide = tm[b].w != 0;
             uint32_t pk[32];
             if (w > 0.f) {
                 chunk_softmax_row<kPolyPairEvery>(sv, nvis, w, sl2, pk, wide);
@@ -412,9 +414,10 @@ CmPlan cm_plan(const Dims &p)
 }
 
 // per query group: count its selected chunks per (kv-group, range, chunk) list, and each head's
-// log-sum-exp of its slot scores (the fusion weights' normaliser)
+// log-sum-exp of its slot scores (the fusion weights' normaliser) and own chunk's fusion weight
 __global__ void cm_count_kernel(Dims p, int RQ, int R, const int32_t *__restrict__ sel_idx,
-                                const float *__restrict__ sel_score, int *__restrict__ cnt, float *__restrict__ lse)
+                                const float *__restrict__ sel_score, int *__restrict__ cnt, float *__restrict__ lse,
+                                float *__restrict__ ow)
 {
     const long long qg = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     if (qg >= (long long)p.B * p.Hkv * p.N) return;
@@ -434,7 +437,9 @@ __global__ void cm_count_kernel(Dims p, int RQ, int R, const int32_t *__restrict
         for (int j = 0; j < ns; ++j) m = fmaxf(m, sr[j]);
         float z = 0.f;
         for (int j = 0; j < ns; ++j) z += (sr[j] == -INFINITY) ? 0.f : __expf(sr[j] - m);
-        lse[row] = m + __logf(z);
+        const float l = m + __logf(z);
+        lse[row] = l;
+        ow[row] = __expf(sr[p.k] - l);   // the own chunk's fusion weight
     }
 }
 
@@ -504,20 +509,27 @@ __global__ void cm_tiles_kernel(Dims p, int RQ, int R, int Mq, int M, const int 
     for (int u = 0; u < n_ret; u += Mq) tiles[t++] = make_int4(bg, c, eoff[m] + u, min(Mq, n_ret - u));
 }
 
-// each selected (query, slot) into its chunk's list: entry = query << 6 | slot
-__global__ void cm_scatter_kernel(Dims p, int RQ, int R, const int32_t *__restrict__ sel_idx, int *__restrict__ fill,
-                                  int *__restrict__ entries)
+// each selected (query, slot) into its chunk's list: entry = query << 6 | slot, and beside it the
+// slot's fusion weight for each of the group's G heads
+__global__ void cm_scatter_kernel(Dims p, int RQ, int R, const int32_t *__restrict__ sel_idx,
+                                  const float *__restrict__ sel_score, const float *__restrict__ lse,
+                                  int *__restrict__ fill, int *__restrict__ entries, float *__restrict__ ew)
 {
     const long long qg = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     if (qg >= (long long)p.B * p.Hkv * p.N) return;
     const int i = (int)(qg % p.N);
     const long long bg = qg / p.N;
-    const int r = i / RQ;
+    const int b = (int)(bg / p.Hkv), g = (int)(bg % p.Hkv);
+    const int r = i / RQ, ns = p.k + 1;
     for (int j = 0; j < p.k; ++j) {
         const int c = sel_idx[qg * p.k + j];
         if (c >= 0) {
             const int at = atomicAdd(fill + ((bg * R + r) * p.nL + c), 1);
             entries[at] = (i << 6) | j;
+            for (int h = 0; h < p.G; ++h) {
+                const size_t row = ((size_t)b * p.H + (size_t)g * p.G + h) * p.N + i;
+                ew[(size_t)at * p.G + h] = __expf(sel_score[row * ns + j] - lse[row]);
+            }
         }
     }
 }
@@ -550,7 +562,7 @@ __global__ void cm_finalize_kernel(Dims p, const float4 *__restrict__ acc, Tout 
 
 struct CmWs {
     int *cnt, *eoff, *fill, *toff, *n_tiles, *entries;
-    float *lse, *acc;
+    float *lse, *ow, *ew, *acc;
     int4 *tiles;
     size_t total;
 };
@@ -572,7 +584,9 @@ CmWs cm_ws(const Dims &p, hils_dtype out, void *ws)
     w.toff = reinterpret_cast<int *>(take((size_t)c.M * 4));
     w.n_tiles = reinterpret_cast<int *>(take(4));
     w.lse = reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * 4));
+    w.ow = reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * 4));
     w.entries = reinterpret_cast<int *>(take((size_t)p.B * p.Hkv * p.N * p.k * 4 + 4));
+    w.ew = reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * p.k * 4 + 4));
     w.tiles = reinterpret_cast<int4 *>(take((size_t)c.max_tiles * 16));
     w.acc = reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * kD * 4));
     w.total = off;
@@ -617,10 +631,12 @@ cudaError_t launch_attend_prefill_cm(const Dims &p, hils_dtype out, const void *
     e = cudaMemsetAsync(w.cnt, 0, (size_t)c.M * 4, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(acc, 0, (size_t)p.B * p.H * p.N * kD * 4, s);
     if (e != cudaSuccess) return e;
-    cm_count_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, s>>>(p, c.RQ, c.R, sel_idx, sel_score, w.cnt, w.lse);
+    cm_count_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, s>>>(p, c.RQ, c.R, sel_idx, sel_score, w.cnt, w.lse,
+                                                                     w.ow);
     cm_scan_kernel<<<1, 1024, 0, s>>>(p, c.RQ, c.R, c.Mq, c.M, w.cnt, w.eoff, w.fill, w.toff, w.n_tiles);
     cm_tiles_kernel<<<(c.M + 255) / 256, 256, 0, s>>>(p, c.RQ, c.R, c.Mq, c.M, w.cnt, w.eoff, w.toff, w.tiles);
-    cm_scatter_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, s>>>(p, c.RQ, c.R, sel_idx, w.fill, w.entries);
+    cm_scatter_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, s>>>(p, c.RQ, c.R, sel_idx, sel_score, w.lse,
+                                                                       w.fill, w.entries, w.ew);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     CUtensorMap tk, tv16, tvb;
@@ -640,8 +656,8 @@ cudaError_t launch_attend_prefill_cm(const Dims &p, hils_dtype out, const void *
     e = cudaFuncSetAttribute(attend_cm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int grid = (int)min((long long)n_sm, c.max_tiles);
-    attend_cm_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tk, tv16, tvb, p, static_cast<const __nv_bfloat16 *>(Q), sel_score,
-                                                        w.lse, w.entries, w.tiles, w.n_tiles, wide, acc, ctl.status,
+    attend_cm_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tk, tv16, tvb, p, static_cast<const __nv_bfloat16 *>(Q), w.ew,
+                                                        w.ow, w.entries, w.tiles, w.n_tiles, wide, acc, ctl.status,
                                                         (unsigned long long)ctl.wait_limit);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

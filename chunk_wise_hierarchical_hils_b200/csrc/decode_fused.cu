@@ -49,6 +49,7 @@ constexpr uint32_t kCStage = 4 * kHalf;           // keys then values of one chu
 constexpr int kNC = 5;                            // phase-2 stages = phase-2 consumer warps
 constexpr uint32_t kRing = 160 * 1024;
 constexpr int kMaxRows = 4096;                    // landmark rows per CTA
+constexpr int kPrefetch = 12;                     // selected chunks prefetched into L2 ahead of their copies
 constexpr unsigned long long kDrainNs = 2000000000ull;
 static_assert(kNL * kLStage <= kRing && kNC * kCStage <= kRing, "stages fit the ring");
 static_assert(kNC * 16 * kD * 4 <= kRing, "the warps' partial outputs fit the ring");
@@ -76,6 +77,7 @@ __host__ __device__ inline Layout make_layout()
 }
 
 struct FusedArgs {
+    const __nv_bfloat16 *K, *V;   // the caches (L2 prefetches of the selected chunks)
     uint64_t *cand;          // [BG][S][k] local top-k keys
     float *part;             // [BG][S][G][d] partial outputs (S > 1)
     unsigned int *tick1;     // [BG] scan tickets
@@ -322,8 +324,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 4; ++e) oacc[nd][e] = 0.f;
     if (warp == kWarps) {
         if (lane == 0) {
+            // the chunks are scattered over a cache of many GB: their first touch is slow (address
+            // translation and DRAM latency), so each one's rows are prefetched into L2 well before its
+            // tile copy, keeping many chunks in flight per SM without shared memory for them
+            auto prefetch = [&](int u) {
+                const int c = slot_c[u] >> 8;
+                const int rows = (int)min((long long)kC, (long long)p.T - (long long)c * kC);
+                const size_t off = ((size_t)bg * p.T + (size_t)c * kC) * kD;
+                const uint32_t bytes = (uint32_t)rows * kD * 2;
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.K + off), "r"(bytes) : "memory");
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.V + off), "r"(bytes) : "memory");
+            };
+            for (int u = 0; u < min(kPrefetch, n_my); ++u) prefetch(u);
             int &issued = issued2;
             for (; issued < n_my; ++issued) {
+                if (issued + kPrefetch < n_my) prefetch(issued + kPrefetch);
                 const int slot = issued % kNC;
                 if (issued >= kNC &&
                     !mbar_wait(EMPTY2(slot), (uint32_t)(((issued / kNC) - 1) & 1), limit_ns, abort_flag, status))
@@ -520,6 +535,8 @@ cudaError_t launch_decode_fused(const Dims &p, hils_dtype out, const void *Q, co
     const size_t BG = (size_t)p.B * p.Hkv;
     char *w = static_cast<char *>(ws);
     FusedArgs a;
+    a.K = static_cast<const __nv_bfloat16 *>(K);
+    a.V = static_cast<const __nv_bfloat16 *>(V);
     a.cand = reinterpret_cast<uint64_t *>(w);
     w += align_up(BG * f.S * p.k * 8, 256);
     a.part = reinterpret_cast<float *>(w);
