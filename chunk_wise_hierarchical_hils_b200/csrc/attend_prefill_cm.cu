@@ -413,33 +413,64 @@ CmPlan cm_plan(const Dims &p)
     return c;
 }
 
+constexpr int kHistBins = 8192;   // shared-memory histogram of a block's lists (32 KB)
+
+// The lists a block of consecutive query groups touches, (kv-group, range) pairs pr_lo .. pr_hi: when they
+// fit the shared-memory histogram, the block counts there and adds each list's count to global memory
+// once (the same few hundred lists are hit by every query of a block), else it counts in global memory.
+__device__ __forceinline__ void block_pairs(const Dims &p, int RQ, int R, long long qg0, int &pr_lo, int &pr_hi)
+{
+    const long long groups = (long long)p.B * p.Hkv * p.N;
+    const long long qa = qg0, qz = min(qg0 + (long long)blockDim.x, groups) - 1;
+    pr_lo = (int)((qa / p.N) * R + (qa % p.N) / RQ);
+    pr_hi = (int)((qz / p.N) * R + (qz % p.N) / RQ);
+}
+
 // per query group: count its selected chunks per (kv-group, range, chunk) list, and each head's
 // log-sum-exp of its slot scores (the fusion weights' normaliser) and own chunk's fusion weight
 __global__ void cm_count_kernel(Dims p, int RQ, int R, const int32_t *__restrict__ sel_idx,
                                 const float *__restrict__ sel_score, int *__restrict__ cnt, float *__restrict__ lse,
                                 float *__restrict__ ow)
 {
-    const long long qg = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-    if (qg >= (long long)p.B * p.Hkv * p.N) return;
-    const int i = (int)(qg % p.N);
-    const long long bg = qg / p.N;
-    const int b = (int)(bg / p.Hkv), g = (int)(bg % p.Hkv);
-    const int r = i / RQ;
-    for (int j = 0; j < p.k; ++j) {
-        const int c = sel_idx[qg * p.k + j];
-        if (c >= 0) atomicAdd(cnt + ((bg * R + r) * p.nL + c), 1);
+    __shared__ int hist[kHistBins];
+    const long long qg0 = (long long)blockIdx.x * blockDim.x, qg = qg0 + threadIdx.x;
+    const bool valid = qg < (long long)p.B * p.Hkv * p.N;
+    int pr_lo, pr_hi;
+    block_pairs(p, RQ, R, qg0, pr_lo, pr_hi);
+    const int span = (pr_hi - pr_lo + 1) * p.nL;
+    const bool local = span <= kHistBins;
+    if (local) {
+        for (int x = threadIdx.x; x < span; x += blockDim.x) hist[x] = 0;
+        __syncthreads();
     }
-    const int ns = p.k + 1;
-    for (int h = 0; h < p.G; ++h) {
-        const size_t row = ((size_t)b * p.H + (size_t)g * p.G + h) * p.N + i;
-        const float *sr = sel_score + row * ns;
-        float m = -INFINITY;
-        for (int j = 0; j < ns; ++j) m = fmaxf(m, sr[j]);
-        float z = 0.f;
-        for (int j = 0; j < ns; ++j) z += (sr[j] == -INFINITY) ? 0.f : __expf(sr[j] - m);
-        const float l = m + __logf(z);
-        lse[row] = l;
-        ow[row] = __expf(sr[p.k] - l);   // the own chunk's fusion weight
+    if (valid) {
+        const int i = (int)(qg % p.N);
+        const long long bg = qg / p.N;
+        const int b = (int)(bg / p.Hkv), g = (int)(bg % p.Hkv);
+        const int pr = (int)(bg * R + i / RQ);
+        for (int j = 0; j < p.k; ++j) {
+            const int c = sel_idx[qg * p.k + j];
+            if (c < 0) continue;
+            if (local) atomicAdd(hist + (pr - pr_lo) * p.nL + c, 1);
+            else atomicAdd(cnt + (size_t)pr * p.nL + c, 1);
+        }
+        const int ns = p.k + 1;
+        for (int h = 0; h < p.G; ++h) {
+            const size_t row = ((size_t)b * p.H + (size_t)g * p.G + h) * p.N + i;
+            const float *sr = sel_score + row * ns;
+            float m = -INFINITY;
+            for (int j = 0; j < ns; ++j) m = fmaxf(m, sr[j]);
+            float z = 0.f;
+            for (int j = 0; j < ns; ++j) z += (sr[j] == -INFINITY) ? 0.f : __expf(sr[j] - m);
+            const float l = m + __logf(z);
+            lse[row] = l;
+            ow[row] = __expf(sr[p.k] - l);   // the own chunk's fusion weight
+        }
+    }
+    if (local) {
+        __syncthreads();
+        for (int x = threadIdx.x; x < span; x += blockDim.x)
+            if (hist[x]) atomicAdd(cnt + (size_t)pr_lo * p.nL + x, hist[x]);
     }
 }
 
@@ -510,26 +541,53 @@ __global__ void cm_tiles_kernel(Dims p, int RQ, int R, int Mq, int M, const int 
 }
 
 // each selected (query, slot) into its chunk's list: entry = query << 6 | slot, and beside it the
-// slot's fusion weight for each of the group's G heads
+// slot's fusion weight for each of the group's G heads.  Positions are reserved per list once per block
+// (a shared-memory count, one global atomic per list, then shared-memory atomics), where the block's
+// lists fit the histogram; otherwise one global atomic per entry.
 __global__ void cm_scatter_kernel(Dims p, int RQ, int R, const int32_t *__restrict__ sel_idx,
                                   const float *__restrict__ sel_score, const float *__restrict__ lse,
                                   int *__restrict__ fill, int *__restrict__ entries, float *__restrict__ ew)
 {
-    const long long qg = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-    if (qg >= (long long)p.B * p.Hkv * p.N) return;
-    const int i = (int)(qg % p.N);
-    const long long bg = qg / p.N;
-    const int b = (int)(bg / p.Hkv), g = (int)(bg % p.Hkv);
-    const int r = i / RQ, ns = p.k + 1;
+    __shared__ int hist[kHistBins];
+    const long long qg0 = (long long)blockIdx.x * blockDim.x, qg = qg0 + threadIdx.x;
+    const bool valid = qg < (long long)p.B * p.Hkv * p.N;
+    int pr_lo, pr_hi;
+    block_pairs(p, RQ, R, qg0, pr_lo, pr_hi);
+    const int span = (pr_hi - pr_lo + 1) * p.nL;
+    const bool local = span <= kHistBins;
+    int i = 0, b = 0, g = 0, pr = 0;
+    long long bg = 0;
+    if (valid) {
+        i = (int)(qg % p.N);
+        bg = qg / p.N;
+        b = (int)(bg / p.Hkv);
+        g = (int)(bg % p.Hkv);
+        pr = (int)(bg * R + i / RQ);
+    }
+    if (local) {
+        for (int x = threadIdx.x; x < span; x += blockDim.x) hist[x] = 0;
+        __syncthreads();
+        if (valid)
+            for (int j = 0; j < p.k; ++j) {
+                const int c = sel_idx[qg * p.k + j];
+                if (c >= 0) atomicAdd(hist + (pr - pr_lo) * p.nL + c, 1);
+            }
+        __syncthreads();
+        for (int x = threadIdx.x; x < span; x += blockDim.x)
+            if (hist[x]) hist[x] = atomicAdd(fill + (size_t)pr_lo * p.nL + x, hist[x]);
+        __syncthreads();
+    }
+    if (!valid) return;
+    const int ns = p.k + 1;
     for (int j = 0; j < p.k; ++j) {
         const int c = sel_idx[qg * p.k + j];
-        if (c >= 0) {
-            const int at = atomicAdd(fill + ((bg * R + r) * p.nL + c), 1);
-            entries[at] = (i << 6) | j;
-            for (int h = 0; h < p.G; ++h) {
-                const size_t row = ((size_t)b * p.H + (size_t)g * p.G + h) * p.N + i;
-                ew[(size_t)at * p.G + h] = __expf(sel_score[row * ns + j] - lse[row]);
-            }
+        if (c < 0) continue;
+        const int at = local ? atomicAdd(hist + (pr - pr_lo) * p.nL + c, 1)
+                             : atomicAdd(fill + (size_t)pr * p.nL + c, 1);
+        entries[at] = (i << 6) | j;
+        for (int h = 0; h < p.G; ++h) {
+            const size_t row = ((size_t)b * p.H + (size_t)g * p.G + h) * p.N + i;
+            ew[(size_t)at * p.G + h] = __expf(sel_score[row * ns + j] - lse[row]);
         }
     }
 }
@@ -607,11 +665,13 @@ bool attend_cm_supported(const Dims &p, hils_dtype in)
 // Chunk-major work grows with the selected pairs, the union kernel's with the chunks its query blocks
 // cover; with uncorrelated selections a block covers about every visible chunk, so the union kernel
 // does about (mean visible chunks) / (k + 1) times the useful work.  The chunk-major kernel pays a
-// float32 reduction per selected pair instead; it is chosen when that ratio exceeds 3.
+// float32 reduction per selected pair and an inversion instead.  Measured on B200: at a ratio of
+// about 4 (8K prefill, k = 16) the union kernel is 2.8 times faster, at about 62 (256K prefill,
+// k = 32) the chunk-major kernel is 1.45 times faster; the switch is placed at 16, between the two.
 bool attend_cm_preferred(const Dims &p)
 {
     const double mean_visible = ((double)p.q_offset + 0.5 * p.N) / p.C + 0.5;
-    return mean_visible > 3.0 * (p.k + 1);
+    return mean_visible > 16.0 * (p.k + 1);
 }
 
 size_t attend_cm_ws_bytes(const Dims &p, hils_dtype out) { return cm_ws(p, out, nullptr).total; }

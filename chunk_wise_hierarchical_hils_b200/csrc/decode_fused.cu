@@ -41,22 +41,23 @@ using dtiles::kQPitch;
 constexpr int kWarps = 7;                         // consumer warps (eight warps in all: two per SM
 constexpr int kThreads = 32 * (kWarps + 1);       // sub-partition, so that each may hold 255 registers)
 constexpr int kD = 128, kC = 64;
-constexpr int kLRows = 64;                        // landmark rows per phase-1 stage
-constexpr uint32_t kLStage = kLRows * kD * 2;     // 16 KB
-constexpr int kNL = 10;                           // phase-1 stages
+constexpr int kLRows = 8 * kWarps;                // landmark rows per phase-1 stage: 8 per consumer warp
+constexpr uint32_t kLStage = kLRows * kD * 2;     // 14 KB
+constexpr int kNL = 11;                           // phase-1 stages
 constexpr uint32_t kHalf = kC * 128;              // one 64-column half of a chunk tile
 constexpr uint32_t kCStage = 4 * kHalf;           // keys then values of one chunk: 32 KB
 constexpr int kNC = 5;                            // phase-2 stages = phase-2 consumer warps
 constexpr uint32_t kRing = 160 * 1024;
-constexpr int kMaxRows = 4096;                    // landmark rows per CTA
+constexpr int kKeys = 4096;                       // keys region: S x k merged keys, then the slots' rows
 constexpr int kPrefetch = 12;                     // selected chunks prefetched into L2 ahead of their copies
 constexpr unsigned long long kDrainNs = 2000000000ull;
 static_assert(kNL * kLStage <= kRing && kNC * kCStage <= kRing, "stages fit the ring");
 static_assert(kNC * 16 * kD * 4 <= kRing, "the warps' partial outputs fit the ring");
 static_assert(kNC <= kWarps, "a consumer warp per phase-2 stage");
+static_assert((HILS_MAX_K + 1) * kD * 2 <= kKeys * 8 && 32 * HILS_MAX_K <= kKeys, "the keys region holds both uses");
 
 struct Layout {
-    uint32_t ring, keys, qs, qbar, wsm, slot_c, top, wl, bars, misc, total;
+    uint32_t ring, keys, qs, qbar, wsm, slot_c, top, wl, cbuf, bars, misc, total;
 };
 
 __host__ __device__ inline Layout make_layout()
@@ -64,13 +65,14 @@ __host__ __device__ inline Layout make_layout()
     Layout L;
     L.ring = 0;
     L.keys = kRing;
-    L.qs = L.keys + kMaxRows * 8;
+    L.qs = L.keys + kKeys * 8;
     L.qbar = L.qs + 16 * kQPitch;
     L.wsm = L.qbar + kD * 4;
     L.slot_c = L.wsm + HILS_MAX_GROUP * (HILS_MAX_K + 1) * 4;
     L.top = (L.slot_c + (HILS_MAX_K + 1) * 4 + 7) & ~7u;
     L.wl = L.top + HILS_MAX_K * 8;
-    L.bars = L.wl + kWarps * HILS_MAX_K * 8;
+    L.cbuf = L.wl + kWarps * HILS_MAX_K * 8;
+    L.bars = L.cbuf + kWarps * 64 * 8;
     L.misc = L.bars + (2 * kNL + 2 * kNC) * 8;
     L.total = L.misc + 32;
     return L;
@@ -99,31 +101,65 @@ __device__ __forceinline__ void st_release(unsigned int *p, unsigned int v)
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// The k largest of n keys (kWarps warps each keep a list over a strided share, warp 0 merges the
-// lists) into out[0 .. 32 KR), descending; every thread of the block calls it.
+// Warp 0 merges the consumer warps' lists (wl[w][0 .. 32 KR), descending) into out[0 .. 64), descending,
+// zero padded; every thread of the block calls it.
 template <int KR>
-__device__ __forceinline__ void topk_warps(const uint64_t *keys, int n, uint64_t *wl, uint64_t *out)
+__device__ __forceinline__ void merge_lists(const uint64_t *wl, uint64_t *cbuf, uint64_t *out)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (warp == 0) {
+        wtopk::Stream<KR> tk;
+        tk.init(cbuf);
+#pragma unroll
+        for (int r = 0; r < KR; ++r) tk.L.v[r] = wl[r * 32 + lane];
+        tk.thr = tk.L.last();
+        for (int w = 1; w < kWarps; ++w)
+#pragma unroll
+            for (int r = 0; r < KR; ++r) tk.offer(wl[w * 64 + r * 32 + lane]);
+        tk.flush();
+#pragma unroll
+        for (int r = 0; r < 2; ++r) out[r * 32 + lane] = r < KR ? tk.L.v[r] : 0ull;
+    }
+    __syncthreads();
+}
+
+// The k largest of n keys in shared memory (each consumer warp streams a strided share, then
+// merge_lists) into out[0 .. 64); every thread of the block calls it.
+template <int KR>
+__device__ __forceinline__ void topk_array(const uint64_t *keys, int n, uint64_t *wl, uint64_t *cbuf, uint64_t *out)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp < kWarps) {
-        wtopk::List<KR> L;
-        L.clear();
-        for (int e0 = warp * 32; e0 < n; e0 += kWarps * 32) L.add(e0 + lane < n ? keys[e0 + lane] : 0ull);
+        wtopk::Stream<KR> tk;
+        tk.init(cbuf + warp * 64);
+        for (int e0 = warp * 32; e0 < n; e0 += kWarps * 32) tk.offer(e0 + lane < n ? keys[e0 + lane] : 0ull);
+        tk.flush();
 #pragma unroll
-        for (int r = 0; r < KR; ++r) wl[warp * 64 + r * 32 + lane] = L.v[r];
+        for (int r = 0; r < KR; ++r) wl[warp * 64 + r * 32 + lane] = tk.L.v[r];
     }
-    __syncthreads();
-    if (warp == 0) {
-        wtopk::List<KR> L;
-#pragma unroll
-        for (int r = 0; r < KR; ++r) L.v[r] = wl[r * 32 + lane];
-        for (int w = 1; w < kWarps; ++w)
-#pragma unroll
-            for (int r = 0; r < KR; ++r) L.add(wl[w * 64 + r * 32 + lane]);
-#pragma unroll
-        for (int r = 0; r < 2; ++r) out[r * 32 + lane] = r < KR ? L.v[r] : 0ull;
+    merge_lists<KR>(wl, cbuf, out);
+}
+
+// Bounded wait of one thread until *flag >= target (set by another CTA of the same (b, g), resident
+// and running); false, with the abort flag set, on a device error or expiry.
+__device__ __forceinline__ bool wait_flag(const unsigned int *flag, unsigned int target, unsigned long long limit_ns,
+                                          volatile int *abort_flag, unsigned int *status)
+{
+    const long long t0 = cycle_now();
+    while (ld_acquire(flag) < target) {
+        if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
+            *abort_flag = 1;
+            return false;
+        }
+        if (past_limit(t0, limit_ns)) {
+            *abort_flag = 1;
+            atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
+            return false;
+        }
+        __nanosleep(64);
     }
-    __syncthreads();
+    return true;
 }
 
 template <typename Tout, int KR>
@@ -143,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *slot_c = reinterpret_cast<int *>(base + Ly.slot_c);
     uint64_t *s_top = reinterpret_cast<uint64_t *>(base + Ly.top);
     uint64_t *wl = reinterpret_cast<uint64_t *>(base + Ly.wl);
+    uint64_t *cbuf = reinterpret_cast<uint64_t *>(base + Ly.cbuf);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc);
     int *s_flag = reinterpret_cast<int *>(base + Ly.misc + 4);
     int *s_nmy = reinterpret_cast<int *>(base + Ly.misc + 8);
@@ -218,12 +255,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // 16 lanes per landmark row, 8 elements each, two rows per warp step: the same products, order
-        // and butterfly as the two-kernel selection
-        const int sub = lane & 15;
+        // warp w scores rows 8w .. 8w + 7 of every stage: 16 lanes per landmark row, 8 elements each, four
+        // rows per half warp at once (per row the same products, order and butterfly as the two-kernel
+        // selection), and offers the keys to its streaming top-k list
+        const int sub = lane & 15, rb = warp * 8 + (lane >> 4) * 4;
         float qv[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) qv[u] = qbar[sub * 8 + u];
+        wtopk::Stream<KR> tk;
+        tk.init(cbuf + warp * 64);
         for (int st = 0; st < n_st; ++st) {
             const int slot = st % kNL;
             int w_ok = 1;
@@ -234,24 +274,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int r0 = st * kLRows, nr = min(kLRows, n_local - r0);
             const __nv_bfloat16 *stg = reinterpret_cast<const __nv_bfloat16 *>(base + Ly.ring + (size_t)slot * kLStage);
-            for (int rw = warp * 2; rw < nr; rw += kWarps * 2) {
-                const int rr = rw + (lane >> 4);
+            float acc[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
                 float lv[8];
-                if (rr < nr) {
-                    lds8(stg + (size_t)rr * kD + sub * 8, lv);
+                if (rb + u < nr) {
+                    lds8(stg + (size_t)(rb + u) * kD + sub * 8, lv);
                 } else {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) lv[u] = 0.f;
+                    for (int x = 0; x < 8; ++x) lv[x] = 0.f;
                 }
-                float acc = 0.f;
+                float a0 = 0.f;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) acc = fmaf(qv[u], lv[u], acc);
-#pragma unroll
-                for (int o = 8; o; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-                if (sub == 0 && rr < nr) keys[r0 + rr] = make_key(acc, c0 + r0 + rr);
+                for (int x = 0; x < 8; ++x) a0 = fmaf(qv[x], lv[x], a0);
+                acc[u] = a0;
             }
+#pragma unroll
+            for (int o = 8; o; o >>= 1)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], o);
             __syncwarp();
             if (lane == 0) mbar_arrive(EMPTY1(slot));
+            // lanes 0-3 of each half warp offer its four rows
+            const int u = lane & 3;
+            const float mine = u == 0 ? acc[0] : (u == 1 ? acc[1] : (u == 2 ? acc[2] : acc[3]));
+            tk.offer((sub < 4 && rb + u < nr) ? make_key(mine, c0 + r0 + rb + u) : 0ull);
+        }
+        if (ok) {
+            tk.flush();
+#pragma unroll
+            for (int r = 0; r < KR; ++r) wl[warp * 64 + r * 32 + lane] = tk.L.v[r];
         }
         if (!ok) *abort_flag = 1;
     }
@@ -264,8 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
 
-    // local top-k, then the merge by the last CTA of the (b, g)
-    topk_warps<KR>(keys, n_local, wl, s_top);
+    // local top-k (the warps' lists merged), then the merge by the last CTA of the (b, g)
+    merge_lists<KR>(wl, cbuf, s_top);
     bool merger = true;
     if (S > 1) {
         uint64_t *mine = a.cand + ((size_t)bg * S + s) * k;
@@ -280,24 +332,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t *all = a.cand + (size_t)bg * S * k;
             for (int e = tid; e < S * k; e += kThreads) keys[e] = __ldcg(all + e);
             __syncthreads();
-            topk_warps<KR>(keys, S * k, wl, s_top);
+            topk_array<KR>(keys, S * k, wl, cbuf, s_top);
         }
     }
-    if (!merger && tid == 0) {
-        // wait for the merge of this (b, g) (bounded: the merging CTA is resident and running)
-        const long long t0 = cycle_now();
-        while (ld_acquire(&a.ready[bg]) == 0u) {
-            if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
-                *abort_flag = 1;
-                break;
-            }
-            if (past_limit(t0, limit_ns)) {
-                *abort_flag = 1;
-                atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
-                break;
-            }
-            __nanosleep(64);
+    unsigned char *lrows = base + Ly.keys;   // [ns][16 pieces], bf16: the slots' landmark rows
+    if (merger) {
+        // the selection is written and published (other CTAs of the (b, g) start their chunk copies),
+        // then the slots' landmark rows are staged for the slot scores before this CTA's own chunk copies
+        // start (behind them these loads would wait for the copies' bytes)
+        for (int j = tid; j < k; j += kThreads) sel_idx[(size_t)bg * k + j] = key_index(s_top[j]);
+        if (S > 1) {
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) st_release(&a.ready[bg], 1u);
         }
+        uint4 lv[5];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+            const int e = tid + i * kThreads;
+            if (e < ns * 16) {
+                const int j = e >> 4, seg = e & 15;
+                const int c = (j < k) ? key_index(s_top[j]) : ci;
+                lv[i] = __ldg(reinterpret_cast<const uint4 *>(Lbg + (size_t)(c >= 0 ? c : 0) * kD) + seg);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+            const int e = tid + i * kThreads;
+            if (e < ns * 16) *reinterpret_cast<uint4 *>(lrows + (size_t)e * 16) = lv[i];
+        }
+    } else if (tid == 0) {
+        wait_flag(&a.ready[bg], 1u, limit_ns, abort_flag, status);   // the selection of this (b, g)
     }
     __syncthreads();
     if (*abort_flag) return;
@@ -356,17 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         constexpr int kCons = 32 * kWarps;   // consumer threads; they meet on named barrier 1
         if (merger) {
-            // the selection and the per-head scores of its k slots and the own chunk: the slots' landmark
-            // rows staged in shared memory (the keys are no longer needed), every load in flight at once
-            unsigned char *lrows = base + Ly.keys;   // [ns][16 pieces], bf16
-            for (int e = tid; e < ns * 16; e += kCons) {
-                const int j = e >> 4, seg = e & 15;
-                const int c = (j < k) ? key_index(s_top[j]) : ci;
-                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(Lbg + (size_t)(c >= 0 ? c : 0) * kD) + seg);
-                *reinterpret_cast<uint4 *>(lrows + (size_t)e * 16) = v;
-            }
-            for (int j = tid; j < k; j += kCons) sel_idx[(size_t)bg * k + j] = key_index(s_top[j]);
-            asm volatile("bar.sync 1, %0;" ::"r"(kCons) : "memory");
+            // the per-head scores of the k slots and the own chunk, from the staged landmark rows
             for (int task = tid; task < G * ns; task += kCons) {
                 const int h = task / ns, j = task % ns;
                 const int c = (j < k) ? key_index(s_top[j]) : ci;
@@ -387,12 +442,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wsm[task] = r;
                 sel_score[((size_t)b * p.H + (size_t)g * G + h) * ns + j] = r;
             }
-            __threadfence();
+            if (S > 1) __threadfence();   // other CTAs of the (b, g) read the scores
             asm volatile("bar.sync 1, %0;" ::"r"(kCons) : "memory");
-            if (tid == 0 && S > 1) st_release(&a.ready[bg], 1u);
+            if (tid == 0 && S > 1) st_release(&a.ready[bg], 2u);
         } else {
-            for (int task = tid; task < G * ns; task += kCons)
-                wsm[task] = __ldcg(sel_score + ((size_t)b * p.H + (size_t)g * G + task / ns) * ns + task % ns);
+            if (tid == 0) wait_flag(&a.ready[bg], 2u, limit_ns, abort_flag, status);   // the slot scores
+            asm volatile("bar.sync 1, %0;" ::"r"(kCons) : "memory");
+            if (!*abort_flag)
+                for (int task = tid; task < G * ns; task += kCons)
+                    wsm[task] = __ldcg(sel_score + ((size_t)b * p.H + (size_t)g * G + task / ns) * ns + task % ns);
             asm volatile("bar.sync 1, %0;" ::"r"(kCons) : "memory");
         }
         // fusion weights of every head: softmax over its slot scores
@@ -500,9 +558,6 @@ FusedPlan fused_plan(const Dims &p)
     const int n_past = p.k > 0 ? (int)((long long)p.q_offset / kC) : 0;
     int S = n_sm / BG;
     if (S > 32) S = 32;
-    // no CTA scans more than kMaxRows landmark rows
-    const int need = (n_past + kMaxRows - 1) / kMaxRows;
-    if (need > S) return f;
     // no more CTAs than there are rows or slots to share
     const int useful = max(1, max((n_past + kLRows - 1) / kLRows, p.k + 1));
     if (S > useful) S = useful;

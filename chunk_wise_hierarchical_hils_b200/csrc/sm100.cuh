@@ -94,19 +94,23 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 
 // Bounded wait: returns false (and raises the CTA's abort flag and the device
 // status) when the phase has not completed within limit_ns.  It also returns
-// false once another role of the CTA aborted, or once any CTA recorded a
-// timeout in the device status word, so that one failure ends the whole grid
-// quickly instead of costing every CTA its own time limit.
+// false once another role of the CTA aborted, or, in a wait that has lasted
+// more than about 10 us, once any CTA recorded a timeout in the device status
+// word, so that one failure ends the whole grid quickly instead of costing every
+// CTA its own time limit.  The status word is a global load: short waits, the
+// common case, never issue it (under heavy traffic it takes a microsecond or
+// more, and a phase that completes meanwhile would be seen only after it).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long limit_ns,
                                           volatile int *abort_flag, unsigned int *status)
 {
     // a short spin first: most phases this wait is used for complete within a few hundred cycles
     for (int i = 0; i < 32; ++i)
         if (mbar_test(bar, parity)) return true;
-    if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = cycle_now();
     for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 200u)) return true;
         if (*abort_flag) return false;
+        if (clock64() - t0 < 20000) continue;
         if (*reinterpret_cast<volatile unsigned int *>(status) != 0u) {
             *abort_flag = 1;
             return false;
@@ -116,7 +120,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
             atomicExch(status, 4u /* HILS_ERR_TIMEOUT */);
             return false;
         }
-        if (mbar_try_wait_sleep(bar, parity, 500u)) return true;
     }
 }
 

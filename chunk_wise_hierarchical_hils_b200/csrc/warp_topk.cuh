@@ -106,5 +106,59 @@ struct List {
     }
 };
 
+// A list fed one key per lane at a time (0 = none): keys that do not beat the list's last element are
+// dropped at once (they cannot enter: the list only improves), the others wait in a per-warp buffer
+// of 64 keys in shared memory and are merged 32 at a time, so that the sorting networks run about
+// k ln(n / k) / 32 times for n keys instead of n / 32.
+template <int KR>
+struct Stream {
+    List<KR> L;
+    uint64_t thr;    // the list's last element (warp-uniform)
+    int n;           // keys waiting in buf (warp-uniform)
+    uint64_t *buf;   // this warp's 64 places
+
+    __device__ __forceinline__ void init(uint64_t *b)
+    {
+        L.clear();
+        thr = 0ull;
+        n = 0;
+        buf = b;
+    }
+
+    __device__ __forceinline__ void offer(uint64_t x)
+    {
+        const bool pass = x > thr;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, pass);
+        if (!m) return;
+        const int lane = threadIdx.x & 31;
+        if (pass) buf[n + __popc(m & ((1u << lane) - 1u))] = x;
+        n += __popc(m);
+        if (n >= 32) {
+            __syncwarp();
+            const uint64_t b = buf[lane];
+            const uint64_t rest = (lane + 32 < n) ? buf[lane + 32] : 0ull;
+            __syncwarp();
+            L.add(b);
+            thr = L.last();
+            n -= 32;
+            if (lane < n) buf[lane] = rest;
+            __syncwarp();
+        }
+    }
+
+    __device__ __forceinline__ void flush()
+    {
+        if (n > 0) {
+            __syncwarp();
+            const int lane = threadIdx.x & 31;
+            const uint64_t b = lane < n ? buf[lane] : 0ull;
+            __syncwarp();
+            L.add(b);
+            thr = L.last();
+            n = 0;
+        }
+    }
+};
+
 }  // namespace wtopk
 }  // namespace hils
