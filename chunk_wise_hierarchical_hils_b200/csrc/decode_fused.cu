@@ -289,16 +289,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int x = 0; x < 8; ++x) a0 = fmaf(qv[x], lv[x], a0);
                 acc[u] = a0;
             }
-#pragma unroll
-            for (int o = 8; o; o >>= 1)
-#pragma unroll
-                for (int u = 0; u < 4; ++u) acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], o);
+            // the rows' sums over the half warp's 16 lanes: per row the pairwise additions of a butterfly
+            // over lane distances 8, 4, 2, 1 (float addition commutes, so every lane that forms a pair
+            // gets the same value), with the rows spread over the lanes as the distance halves: 4
+            // shuffles instead of 16; lane bits 3 and 2 then name the row the lane holds
+            const bool b3 = (lane & 8) != 0, b2 = (lane & 4) != 0;
+            const float v0 = (b3 ? acc[2] : acc[0]) + __shfl_xor_sync(0xFFFFFFFFu, b3 ? acc[0] : acc[2], 8);
+            const float v1 = (b3 ? acc[3] : acc[1]) + __shfl_xor_sync(0xFFFFFFFFu, b3 ? acc[1] : acc[3], 8);
+            float rs = (b2 ? v1 : v0) + __shfl_xor_sync(0xFFFFFFFFu, b2 ? v0 : v1, 4);
+            rs += __shfl_xor_sync(0xFFFFFFFFu, rs, 2);
+            rs += __shfl_xor_sync(0xFFFFFFFFu, rs, 1);
             __syncwarp();
             if (lane == 0) mbar_arrive(EMPTY1(slot));
-            // lanes 0-3 of each half warp offer its four rows
-            const int u = lane & 3;
-            const float mine = u == 0 ? acc[0] : (u == 1 ? acc[1] : (u == 2 ? acc[2] : acc[3]));
-            tk.offer((sub < 4 && rb + u < nr) ? make_key(mine, c0 + r0 + rb + u) : 0ull);
+            // lane 4u' of each half warp (u' = 2 b3 + b2) offers row rb + u'
+            const int u = (b3 ? 2 : 0) + (b2 ? 1 : 0);
+            tk.offer(((lane & 3) == 0 && rb + u < nr) ? make_key(rs, c0 + r0 + rb + u) : 0ull);
         }
         if (ok) {
             tk.flush();

@@ -25,6 +25,9 @@
 // index through the key order.
 #include <cuda.h>
 
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -127,12 +130,65 @@ __device__ __forceinline__ void list_sort_desc(uint64_t (&a)[RK], float (&ap)[RK
     }
 }
 
-template <int G, int NSL, int RK>
-__global__ void __launch_bounds__(kThreads, 1)
+// The group sums of G adjacent score columns over the G lanes of a query (lane h holds head h's
+// scores v[0..G) of the columns): after the rounds lane h holds the sum over the G heads of column h.
+// Round r pairs lanes 2^r apart, as the butterfly sum over heads does, so each column's sum is
+// associated exactly as that butterfly associates it (float addition commutes: both lanes of a pair
+// form the same value); each round halves the columns a lane keeps, so G - 1 shuffles serve G columns.
+template <int G>
+__device__ __forceinline__ float head_sum_transposed(float (&v)[G], int h)
+{
+#pragma unroll
+    for (int r = 0, n = G; (1 << r) < G; ++r, n >>= 1) {
+        const bool bit = ((h >> r) & 1) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float keep = bit ? v[2 * i + 1] : v[2 * i];
+            const float send = bit ? v[2 * i] : v[2 * i + 1];
+            v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 1 << r);
+        }
+    }
+    return v[0];
+}
+
+__device__ __forceinline__ uint64_t shfl_xor_key(uint64_t v, int m)
+{
+    const uint32_t lo = __shfl_xor_sync(0xFFFFFFFFu, (uint32_t)v, m);
+    const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, (uint32_t)(v >> 32), m);
+    return ((uint64_t)hi << 32) | lo;
+}
+
+// a (descending, 16 keys) becomes the 16 largest of a and the lane's (lane ^ m) list, descending: the
+// elementwise maximum of a and the other list reversed is bitonic and holds them; a merge network sorts it
+__device__ __forceinline__ void merge_with_lane(uint64_t (&a)[16], int m)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint64_t x = shfl_xor_key(a[15 - i], m), y = shfl_xor_key(a[i], m);
+        a[i] = a[i] > x ? a[i] : x;
+        a[15 - i] = a[15 - i] > y ? a[15 - i] : y;
+    }
+#pragma unroll
+    for (int stride = 8; stride > 0; stride >>= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if ((i & stride) == 0) {
+                const uint64_t x = a[i], y = a[i + stride];
+                a[i] = x > y ? x : y;
+                a[i + stride] = x > y ? y : x;
+            }
+}
+
+// RES (k <= 16, G >= 2, every landmark tile of the CTA kept in TMEM): the G lanes of a query split the
+// score columns (lane h ranks the columns congruent to h mod G, from the transposed head sums), merge
+// their lists at the end, and read the per-head slot scores back from the resident tiles.
+template <int G, int NSL, int RK, bool RES>
+__global__ void __launch_bounds__(kThreads, RES ? 2 : 1)
     select_tc_kernel(const __grid_constant__ CUtensorMap tmL, Dims p, const __nv_bfloat16 *__restrict__ Q,
                      int32_t *__restrict__ sel_idx, float *__restrict__ sel_score, unsigned int *status,
-                     unsigned long long limit_ns)
+                     unsigned long long limit_ns, uint32_t tmem_cols)
 {
+    static_assert(!RES || (RK == 16 && G >= 2), "resident tiles: register lists and two or more heads");
     constexpr int BQ = kRows / G;
     constexpr int RKN = RK > 0 ? RK : 1;   // register list length (unused when RK = 0)
     extern __shared__ unsigned char smem_raw[];
@@ -172,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tmL);
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(tmem_holder), kTmemCols);
+        tmem_alloc(smem_addr(tmem_holder), tmem_cols);
         tmem_relinquish();
     }
     if (RK == 0)
@@ -235,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t la = sL + (uint32_t)st * kTileBytes;
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16_ss(tmem + (uint32_t)(t & 1) * kTile,
+                    mma_bf16_ss(tmem + (uint32_t)(RES ? t : (t & 1)) * kTile,
                                 smem_desc_sw128(sQ + (s >> 2) * 16384u + (s & 3) * 32u, 16, 1024),
                                 smem_desc_sw128(la + (s >> 2) * (kTileBytes / 2) + (s & 3) * 32u, 16, 1024), IDESC,
                                 s > 0 ? 1u : 0u);
@@ -248,7 +304,122 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_drain(L_FULL(u % NSL), (uint32_t)((u / NSL) & 1), kDrainNs);
         }
         __syncwarp();
-    } else if (warp >= 2) {
+    } else if (RES && warp >= 2) {
+        const int qq = warp & 3;
+        const int r = 32 * qq + lane, qi = r / G, h = r % G;
+        const bool valid = qi < nq;
+        const long long pos = (long long)p.q_offset + q0 + qi;
+        const int ci = (int)(pos / p.C);
+        const float sc_g = p.scale / (float)G;
+        const uint32_t trow = tmem + ((uint32_t)(32 * qq) << 16);
+        uint64_t *hk = keys + r;
+        uint64_t top[16];
+        float dummy[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            top[i] = 0ull;
+            dummy[i] = 0.f;
+        }
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            int w_ok = 1;
+            if (lane == 0) w_ok = mbar_wait(S_FULL(t & 1), (uint32_t)((t >> 1) & 1), limit_ns, abort_flag, status);
+            if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[32];
+                tmem_ld32(trow + (uint32_t)t * kTile + 32u * half, sv);
+                tmem_wait_ld();
+                if (half == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(S_FREE(t & 1));
+                }
+                int qn = 0;
+#pragma unroll
+                for (int grp = 0; grp < 32 / G; ++grp) {
+                    float v[G];
+#pragma unroll
+                    for (int x = 0; x < G; ++x) v[x] = __uint_as_float(sv[grp * G + x]);
+                    const float gs = head_sum_transposed<G>(v, h);
+                    const int c = t * kTile + 32 * half + grp * G + h;
+                    const uint64_t key = make_key(gs * sc_g, c);
+                    if (valid && c < ci && p.k > 0 && key > top[15]) {
+                        hk[qn * kRows] = key;
+                        ++qn;
+                    }
+                }
+                // at most 32 / G <= 16 queued keys: the first block fills the empty list by a sort
+                // network, later blocks insert theirs
+                if (t == 0 && half == 0) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) top[i] = i < qn ? hk[i * kRows] : 0ull;
+                    list_sort_desc<16>(top, dummy);
+                } else {
+                    const int m = __reduce_max_sync(0xFFFFFFFFu, qn);
+                    for (int i = 0; i < m; ++i) {
+                        const bool on = i < qn;
+                        list_insert<16>(top, dummy, on ? hk[i * kRows] : 0ull, 0.f, on);
+                    }
+                }
+            }
+        }
+        if (__all_sync(0xFFFFFFFFu, ok)) {
+            // the query's G lists into one, in every lane of the query
+#pragma unroll
+            for (int o = 1; o < G; o <<= 1) merge_with_lane(top, o);
+            // the per-head scores of the selected chunks and of the own chunk, from the resident tiles:
+            // each lane's row of a tile is staged in shared memory (the query tile's space, free once
+            // the last product is done; element x of lane l at l * 64 + (x ^ l), so that neither the
+            // stores nor the reads conflict) and the lane picks its columns
+            float *stg = reinterpret_cast<float *>(base + Ly.q) + qq * 32 * 64;
+            int cj[16];   // the selected chunks, -1 for an empty slot
+            float pay[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                cj[j] = key_index(top[j]);
+                pay[j] = -INFINITY;
+            }
+            float own = -INFINITY;
+            for (int t = 0; t < n_tiles; ++t) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t sv[32];
+                    tmem_ld32(trow + (uint32_t)t * kTile + 32u * half, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) stg[lane * 64 + ((32 * half + x) ^ lane)] = __uint_as_float(sv[x]);
+                }
+                __syncwarp();
+                const int c0 = t * kTile;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int dd = cj[j] - c0;
+                    if (dd >= 0 && dd < kTile) pay[j] = stg[lane * 64 + (dd ^ lane)] * p.scale;
+                }
+                const int dd = ci - c0;
+                if (dd >= 0 && dd < kTile) own = stg[lane * 64 + (dd ^ lane)] * p.scale;
+                __syncwarp();
+            }
+            if (valid) {
+                const size_t row_g = (((size_t)b * p.Hkv + g) * p.N) + q0 + qi;
+                const size_t row_h = (((size_t)b * p.H + (size_t)g * G + h) * p.N) + q0 + qi;
+                const int ns = p.k + 1;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    if (j < p.k) {
+                        if (h == 0) sel_idx[row_g * p.k + j] = cj[j];
+                        sel_score[row_h * ns + j] = pay[j];   // -inf for an empty slot
+                    }
+                }
+                sel_score[row_h * ns + p.k] = own;
+            }
+        }
+    } else if (!RES && warp >= 2) {
         const int qq = warp & 3;
         const int r = 32 * qq + lane, qi = r / G, h = r % G;
         const bool valid = qi < nq;
@@ -379,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, tmem_cols);
     }
 }
 
@@ -402,6 +573,13 @@ EncodeTiledFn encode_fn()
 
 int stages_for(int k) { return k <= 32 ? 2 : 4; }
 
+// Test control: HILS_SELECT_RESIDENT=0 keeps the per-row lists of the streaming epilogue.
+bool res_disabled()
+{
+    const char *v = getenv("HILS_SELECT_RESIDENT");
+    return v && strcmp(v, "0") == 0;
+}
+
 template <int G>
 cudaError_t launch_g(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
                      const DeviceCtl &ctl, cudaStream_t s)
@@ -420,20 +598,29 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *L, int32_t *sel_i
         return cudaErrorInvalidValue;
     const int nsl = stages_for(p.k);
     const int rk = p.k <= 16 ? 16 : 0;   // register list for k <= 16, shared-memory heap above
-    const size_t smem = make_layout(rk ? kQueue : p.k, nsl).total + 1024;
+    size_t smem = make_layout(rk ? kQueue : p.k, nsl).total + 1024;
     dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
+    // every tile of a CTA resident in TMEM when they fit (at most 8 tiles of 64 columns)
+    const int n_tiles_max = (int)(((long long)p.q_offset + p.N - 1) / p.C / kTile) + 1;
+    const bool res = rk == 16 && G >= 2 && n_tiles_max <= 8 && !res_disabled();
+    uint32_t tcols = kTmemCols;
+    if (res) {
+        while (tcols < (uint32_t)n_tiles_max * kTile) tcols <<= 1;
+        if (tcols > 256 && smem < 120 * 1024) smem = 120 * 1024;   // 512 columns: one CTA per SM
+    }
     cudaError_t e;
-#define HILS_LAUNCH_SEL(NS, RKV)                                                                             \
+#define HILS_LAUNCH_SEL(NS, RKV, RESV)                                                                       \
     {                                                                                                        \
-        auto kern = select_tc_kernel<G, NS, RKV>;                                                            \
+        auto kern = select_tc_kernel<G, NS, RKV, RESV>;                                                      \
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);              \
         if (e != cudaSuccess) return e;                                                                      \
         kern<<<grid, kThreads, smem, s>>>(tl, p, static_cast<const __nv_bfloat16 *>(Q), sel_idx, sel_score,  \
-                                          ctl.status, (unsigned long long)ctl.wait_limit);                   \
+                                          ctl.status, (unsigned long long)ctl.wait_limit, tcols);            \
     }
-    if (rk) HILS_LAUNCH_SEL(2, 16)
-    else if (nsl == 2) HILS_LAUNCH_SEL(2, 0)
-    else HILS_LAUNCH_SEL(4, 0)
+    if (rk && res) HILS_LAUNCH_SEL(2, 16, G >= 2)
+    else if (rk) HILS_LAUNCH_SEL(2, 16, false)
+    else if (nsl == 2) HILS_LAUNCH_SEL(2, 0, false)
+    else HILS_LAUNCH_SEL(4, 0, false)
 #undef HILS_LAUNCH_SEL
     return cudaGetLastError();
 }

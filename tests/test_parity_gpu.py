@@ -87,14 +87,25 @@ def test_both_prefill_attentions_with_bf16_output(attend, monkeypatch):
     _check(st)
 
 
-@pytest.mark.parametrize("kernel", ["heads", "queries"])
+# chunked prefill over 3 and 6 landmark tiles of 64 (256 and 512 resident TMEM columns)
+RESIDENT = [
+    wl("g4_c32_three_tiles", B=1, H=8, Hkv=2, N=300, T=6000, q_offset=5700, C=32, k=8, seed=113),
+    wl("g2_c32_six_tiles", B=1, H=4, Hkv=2, N=260, T=12000, q_offset=11740, C=32, k=16, seed=114, l_mode="iid"),
+]
+
+
+@pytest.mark.parametrize("kernel", ["heads", "heads_streaming", "queries"])
 @pytest.mark.parametrize("w", [CASES[1], CASES[3], CASES[5], CASES[6], CASES[7], CASES[8], CASES[10], CASES[11],
-                               CASES[12]], ids=lambda w: w.name)
+                               CASES[12]] + RESIDENT, ids=lambda w: w.name)
 def test_both_tensor_core_selections(w, kernel, monkeypatch):
     """Each tensor-core prefill selection forced on shapes the other one may take: one product row per
-    head (group score by a butterfly over the heads) or one per query (group score from the mean query,
-    per-head slot scores after the scan)."""
-    monkeypatch.setenv("HILS_SELECT_KERNEL", kernel)
+    head (group score by a butterfly over the heads; with k <= 16 and at most 8 landmark tiles the tiles
+    stay in TMEM and the G lanes of a query split the columns, "heads_streaming" forces the per-row
+    lists instead) or one per query (group score from the mean query, per-head slot scores after the
+    scan)."""
+    monkeypatch.setenv("HILS_SELECT_KERNEL", "heads" if kernel.startswith("heads") else kernel)
+    if kernel == "heads_streaming":
+        monkeypatch.setenv("HILS_SELECT_RESIDENT", "0")
     st, _ = parity.run_small(w)
     _check(st)
 
