@@ -10,7 +10,8 @@
 //   beta_c = -sum_t p_t ln p_t
 //
 // HBM-bound: every key row is read once.  One warp per chunk; each lane owns d/32 consecutive columns.
-// Key rows are taken eight at a time (eight independent loads in flight per lane); the eight logits are
+// Key rows are taken eight at a time, and the next eight rows' loads are issued before the current
+// eight are used (sixteen rows in flight per lane while the warp computes); the eight logits are
 // finished by butterfly sums, so every lane holds all of them, and the chunk's softmax runs online
 // across the blocks of eight: running max m, running normaliser z = sum e^{s-m}, running
 // y = sum e^{s-m} (s - m) for the entropy, and the lane's columns of sum e^{s-m} k.  When the max moves
@@ -56,6 +57,45 @@ __device__ __forceinline__ void load_cols(const __nv_bfloat16 *p, float *o)
     }
 }
 
+// The raw (not yet widened) E elements of a lane, so that loads can be issued a block ahead.
+template <typename Tin, int E>
+struct Raw;
+template <>
+struct Raw<float, 4> {
+    float4 v;
+    __device__ __forceinline__ void load(const float *p) { v = __ldg(reinterpret_cast<const float4 *>(p)); }
+    __device__ __forceinline__ void zero() { v = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void widen(float *o) const { o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w; }
+};
+template <>
+struct Raw<float, 2> {
+    float2 v;
+    __device__ __forceinline__ void load(const float *p) { v = __ldg(reinterpret_cast<const float2 *>(p)); }
+    __device__ __forceinline__ void zero() { v = make_float2(0.f, 0.f); }
+    __device__ __forceinline__ void widen(float *o) const { o[0] = v.x; o[1] = v.y; }
+};
+template <>
+struct Raw<__nv_bfloat16, 4> {
+    uint2 v;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) { v = __ldg(reinterpret_cast<const uint2 *>(p)); }
+    __device__ __forceinline__ void zero() { v = make_uint2(0u, 0u); }
+    __device__ __forceinline__ void widen(float *o) const
+    {
+        o[0] = __uint_as_float(v.x << 16); o[1] = __uint_as_float(v.x & 0xFFFF0000u);
+        o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xFFFF0000u);
+    }
+};
+template <>
+struct Raw<__nv_bfloat16, 2> {
+    uint32_t v;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) { v = __ldg(reinterpret_cast<const unsigned int *>(p)); }
+    __device__ __forceinline__ void zero() { v = 0u; }
+    __device__ __forceinline__ void widen(float *o) const
+    {
+        o[0] = __uint_as_float(v << 16); o[1] = __uint_as_float(v & 0xFFFF0000u);
+    }
+};
+
 template <int E>
 __device__ __forceinline__ void store_cols(float *p, const float *v)
 {
@@ -86,7 +126,7 @@ struct LandmarkArgs {
 };
 
 template <typename Tin, int D>
-__global__ void __launch_bounds__(32 * kWarps)
+__global__ void __launch_bounds__(32 * kWarps, sizeof(Tin) == 2 ? 3 : 2)
 landmarks_kernel(const Tin *__restrict__ K, const Tin *__restrict__ U, Tin *__restrict__ L,
                  float *__restrict__ beta, LandmarkArgs a)
 {
@@ -110,22 +150,30 @@ landmarks_kernel(const Tin *__restrict__ K, const Tin *__restrict__ U, Tin *__re
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
 
+    Raw<Tin, E> nxt[kRows];   // the next block's rows, loaded one block ahead
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) {
+        if (j < rows) nxt[j].load(kc + (size_t)j * D);
+        else nxt[j].zero();
+    }
     for (int t0 = 0; t0 < rows; t0 += kRows) {
-        float kv[kRows][E], s[kRows];
+        Raw<Tin, E> cur[kRows];   // kept raw (widened where used) to hold the registers down
+        float s[kRows];
+#pragma unroll
+        for (int j = 0; j < kRows; ++j) cur[j] = nxt[j];
 #pragma unroll
         for (int j = 0; j < kRows; ++j) {
-            if (t0 + j < rows) {
-                load_cols<E>(kc + (size_t)(t0 + j) * D, kv[j]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < E; ++e) kv[j][e] = 0.f;
-            }
+            const int t = t0 + kRows + j;
+            if (t < rows) nxt[j].load(kc + (size_t)t * D);
+            else nxt[j].zero();
         }
 #pragma unroll
         for (int j = 0; j < kRows; ++j) {
+            float kv[E];
+            cur[j].widen(kv);
             float part = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) part = fmaf(u[e], kv[j][e], part);
+            for (int e = 0; e < E; ++e) part = fmaf(u[e], kv[e], part);
             s[j] = part;
         }
 #pragma unroll
@@ -155,8 +203,10 @@ landmarks_kernel(const Tin *__restrict__ K, const Tin *__restrict__ U, Tin *__re
                 const float w = expf(x);
                 z += w;
                 y = fmaf(w, x, y);
+                float kv[E];
+                cur[j].widen(kv);
 #pragma unroll
-                for (int e = 0; e < E; ++e) acc[e] = fmaf(w, kv[j][e], acc[e]);
+                for (int e = 0; e < E; ++e) acc[e] = fmaf(w, kv[e], acc[e]);
             }
         }
     }

@@ -158,6 +158,54 @@ __device__ __forceinline__ uint64_t shfl_xor_key(uint64_t v, int m)
     return ((uint64_t)hi << 32) | lo;
 }
 
+__device__ __forceinline__ void cas_desc(uint64_t &x, uint64_t &y)
+{
+    const uint64_t a = x, b = y;
+    x = a > b ? a : b;
+    y = a > b ? b : a;
+}
+
+// a bitonic sequence of 16 keys, sorted descending in place
+__device__ __forceinline__ void bitonic_merge16_desc(uint64_t (&a)[16])
+{
+#pragma unroll
+    for (int stride = 8; stride > 0; stride >>= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if ((i & stride) == 0) cas_desc(a[i], a[i + stride]);
+}
+
+// N keys (N a power of two), sorted descending in place by a bitonic network
+template <int N>
+__device__ __forceinline__ void sort_desc(uint64_t (&q)[N])
+{
+#pragma unroll
+    for (int size = 2; size <= N; size <<= 1)
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    if ((i & size) == 0 || size == N) cas_desc(q[i], q[j]);
+                    else cas_desc(q[j], q[i]);
+                }
+            }
+}
+
+// a (descending, 16 keys) takes the 16 largest of itself and q (descending, N <= 16 keys): the tail
+// of a against q reversed, elementwise maximum, is bitonic with the head of a; a merge network sorts it
+template <int N>
+__device__ __forceinline__ void merge_sorted(uint64_t (&a)[16], const uint64_t (&q)[N])
+{
+#pragma unroll
+    for (int m = 0; m < N; ++m) {
+        const uint64_t x = q[N - 1 - m];
+        a[16 - N + m] = a[16 - N + m] > x ? a[16 - N + m] : x;
+    }
+    bitonic_merge16_desc(a);
+}
+
 // a (descending, 16 keys) becomes the 16 largest of a and the lane's (lane ^ m) list, descending: the
 // elementwise maximum of a and the other list reversed is bitonic and holds them; a merge network sorts it
 __device__ __forceinline__ void merge_with_lane(uint64_t (&a)[16], int m)
@@ -168,15 +216,7 @@ __device__ __forceinline__ void merge_with_lane(uint64_t (&a)[16], int m)
         a[i] = a[i] > x ? a[i] : x;
         a[15 - i] = a[15 - i] > y ? a[15 - i] : y;
     }
-#pragma unroll
-    for (int stride = 8; stride > 0; stride >>= 1)
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if ((i & stride) == 0) {
-                const uint64_t x = a[i], y = a[i + stride];
-                a[i] = x > y ? x : y;
-                a[i + stride] = x > y ? y : x;
-            }
+    bitonic_merge16_desc(a);
 }
 
 // RES (k <= 16, G >= 2, every landmark tile of the CTA kept in TMEM): the G lanes of a query split the
@@ -314,12 +354,8 @@ __global__ void __launch_bounds__(kThreads, RES ? 2 : 1)
         const uint32_t trow = tmem + ((uint32_t)(32 * qq) << 16);
         uint64_t *hk = keys + r;
         uint64_t top[16];
-        float dummy[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            top[i] = 0ull;
-            dummy[i] = 0.f;
-        }
+        for (int i = 0; i < 16; ++i) top[i] = 0ull;
         bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
             int w_ok = 1;
@@ -353,18 +389,15 @@ __global__ void __launch_bounds__(kThreads, RES ? 2 : 1)
                         ++qn;
                     }
                 }
-                // at most 32 / G <= 16 queued keys: the first block fills the empty list by a sort
-                // network, later blocks insert theirs
-                if (t == 0 && half == 0) {
+                // the block's queued keys (at most 32 / G <= 16) sorted by a network and merged into the
+                // list
+                if (__any_sync(0xFFFFFFFFu, qn > 0)) {
+                    constexpr int QN = 32 / G;
+                    uint64_t qk[QN];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) top[i] = i < qn ? hk[i * kRows] : 0ull;
-                    list_sort_desc<16>(top, dummy);
-                } else {
-                    const int m = __reduce_max_sync(0xFFFFFFFFu, qn);
-                    for (int i = 0; i < m; ++i) {
-                        const bool on = i < qn;
-                        list_insert<16>(top, dummy, on ? hk[i * kRows] : 0ull, 0.f, on);
-                    }
+                    for (int i = 0; i < QN; ++i) qk[i] = i < qn ? hk[i * kRows] : 0ull;
+                    sort_desc<QN>(qk);
+                    merge_sorted<QN>(top, qk);
                 }
             }
         }
