@@ -121,11 +121,12 @@ def kernels_per_step(w):
 def kernel_traffic(kernel, workload):
     """DRAM bytes per launch from an ncu capture committed in profiles/traffic.json, or None.
 
-    The entry names the source files the kernel is built from with their SHA-256 at the time of the
+    Entries are keyed "kernel@workload" (or "kernel" alone).  The entry names the source files the kernel is built from with their SHA-256 at the time of the
     capture; it is used only while every one of them is unchanged, and for the same workload."""
     import hashlib
     try:
-        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
+        data = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        rec = data.get(kernel + "@" + workload) or data[kernel]
         csrc = os.path.join(ROOT, "chunk_wise_hierarchical_hils_b200", "csrc")
         for f, sha in rec["sources"].items():
             if hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest() != sha:
@@ -436,6 +437,7 @@ def measure_forward(args, w, ws, rank, local, steps=None):
     ws_sel = torch.empty(max(hils.hils_score_select_workspace_size(p), 16), dtype=torch.uint8, device="cuda")
     ws_att = torch.empty(max(hils.hils_chunk_attend_fuse_workspace_size(p), 16), dtype=torch.uint8, device="cuda")
     ws_fwd = torch.empty(hils.hils_forward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    plan = hils.hils_describe(p)   # the kernels the library runs for this problem
     # Timing: every timed region replays a CUDA graph of the library calls (captured once after
     # warm-up), so the device times below are the kernels' and not the host's launch gaps.
     # The step graph times the whole path; a graph per call gives each call's average duration.
@@ -540,9 +542,12 @@ def measure_forward(args, w, ws, rank, local, steps=None):
         else:
             peak, kind = tensor_peak(pk, pk_kind, timed_s)
         achieved = fl / (k2_avg * 1e-3) / 1e12
-        roof = {"bound": "tensor", "kernel": "chunk_attend_fuse (prefill)", "achieved": achieved, "peak": peak,
+        cm = "attend=chunk-major" in plan
+        roof = {"bound": "tensor", "kernel": "chunk_attend_fuse (prefill, %s)" % ("chunk-major" if cm else "union"),
+                "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "frac_of_spec": achieved / TENSOR_SPEC_TFLOPS,
-                "traffic": kernel_traffic("attend_prefill_tc", w.name), "peak_kind": kind,
+                "traffic": kernel_traffic("attend_prefill_cm" if cm else "attend_prefill_tc", w.name),
+                "peak_kind": kind,
                 "algorithmic_flops_per_launch": fl, "launch_ms": k2_avg, "select_ms": k1_avg,
                 "step_tflops": (fl + scoring_flops(w)) / (ms_step * 1e-3) / 1e12}
     elif fused:
@@ -577,6 +582,7 @@ def measure_forward(args, w, ws, rank, local, steps=None):
                     "algorithmic_bytes_per_launch": lb, "launch_ms": k1_avg, "attend_ms": k2_avg}
         roof.update({"peak_kind": pk_kind + " copy", "frac_of_spec": achieved / HBM_SPEC_GBS,
                      "step_gbs": step_gbs, "step_frac": step_gbs / peak, "step_frac_of_spec": step_gbs / HBM_SPEC_GBS})
+    roof["plan"] = plan
     units_all = ws * per_step_units
     if args.scaling == "strong" and ws > 1:
         units_all = per_step_units * full_B / w.B   # ranks hold slices of one batch (equal slices assumed)

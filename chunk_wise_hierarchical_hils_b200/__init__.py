@@ -24,7 +24,7 @@ HILS_F32, HILS_BF16 = 0, 1
 HILS_MAX_K = 64
 HILS_MAX_GROUP = 16
 
-EXPORTS = ("hils_status_string", "hils_version", "hils_validate", "hils_score_select_workspace_size",
+EXPORTS = ("hils_status_string", "hils_version", "hils_validate", "hils_describe", "hils_score_select_workspace_size",
            "hils_chunk_attend_fuse_workspace_size", "hils_forward_workspace_size", "hils_score_select",
            "hils_chunk_attend_fuse", "hils_forward", "hils_sync_status", "hils_set_wait_limit",
            "hils_decode_score_select_noalloc", "hils_debug_inject_stall", "hils_landmarks",
@@ -127,6 +127,14 @@ def hils_status_string(status):
 
 def hils_version():
     return _lib.hils_version()
+
+
+def hils_describe(p):
+    """The kernels the library runs for problem p, e.g. "forward=two-call select=tc-heads-resident
+    attend=union-tc" (see include/hils.h)."""
+    buf = ctypes.create_string_buffer(128)
+    _check(_lib.hils_describe(ctypes.byref(p), buf, ctypes.c_size_t(len(buf))), "hils_describe")
+    return buf.value.decode()
 
 
 def hils_validate(p):

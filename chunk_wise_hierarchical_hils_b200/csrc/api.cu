@@ -159,19 +159,50 @@ hils_status check_ws(void *ws, size_t have, size_t need)
     return HILS_OK;
 }
 
+// The selection kernel for a problem (one decision, used by the launch and by hils_describe).
+enum class SelKind { DecodeScan, Queries, Heads, CudaCores };
+
+SelKind select_kind(const Dims &p, hils_dtype in)
+{
+    if (p.N == 1) return SelKind::DecodeScan;
+    const int forced = forced_select_kernel();
+    if (!force_cuda_cores() && forced != 1 && select_q_supported(p, in) && (forced == 2 || select_q_preferred(p)))
+        return SelKind::Queries;
+    if (!force_cuda_cores() && select_tc_supported(p, in)) return SelKind::Heads;
+    return SelKind::CudaCores;
+}
+
 hils_status do_select(const Dims &p, hils_dtype in, const void *Q, const void *L, int32_t *sel_idx,
                       float *sel_score, void *ws, cudaStream_t s)
 {
     DeviceCtl ctl;
     hils_status st = device_ctl(&ctl);
     if (st != HILS_OK) return st;
-    if (p.N == 1) return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, ctl, s));
-    const int forced = forced_select_kernel();
-    if (!force_cuda_cores() && forced != 1 && select_q_supported(p, in) && (forced == 2 || select_q_preferred(p)))
-        return from_cuda(launch_select_prefill_q(p, Q, L, sel_idx, sel_score, ctl, s));
-    if (!force_cuda_cores() && select_tc_supported(p, in))
-        return from_cuda(launch_select_prefill_tc(p, Q, L, sel_idx, sel_score, ctl, s));
-    return from_cuda(launch_select_prefill(p, in, Q, L, sel_idx, sel_score, s));
+    switch (select_kind(p, in)) {
+    case SelKind::DecodeScan: return from_cuda(launch_select_decode(p, in, Q, L, sel_idx, sel_score, ws, ctl, s));
+    case SelKind::Queries: return from_cuda(launch_select_prefill_q(p, Q, L, sel_idx, sel_score, ctl, s));
+    case SelKind::Heads: return from_cuda(launch_select_prefill_tc(p, Q, L, sel_idx, sel_score, ctl, s));
+    default: return from_cuda(launch_select_prefill(p, in, Q, L, sel_idx, sel_score, s));
+    }
+}
+
+// The attention kernel for a problem (hils_chunk_attend_fuse), likewise.
+enum class AttKind { DecodeMma, DecodeCudaCores, ChunkMajor, Union, CudaCores };
+
+AttKind attend_kind(const Dims &p, hils_dtype in)
+{
+    if (p.N == 1)
+        return (!force_decode_cuda_cores() && attend_decode_mma_supported(p, in)) ? AttKind::DecodeMma
+                                                                                   : AttKind::DecodeCudaCores;
+    if (use_chunk_major(p, in)) return AttKind::ChunkMajor;
+    if (!force_cuda_cores() && attend_tc_supported(p, in)) return AttKind::Union;
+    return AttKind::CudaCores;
+}
+
+// hils_forward's single-token decode runs the fused kernel where it applies.
+bool forward_fused(const Dims &p, hils_dtype in)
+{
+    return p.N == 1 && fused_decode_enabled() && !force_decode_cuda_cores() && decode_fused_supported(p, in);
 }
 
 hils_status do_attend(const Dims &p, hils_dtype in, hils_dtype out, const void *Q, const void *K,
@@ -181,12 +212,13 @@ hils_status do_attend(const Dims &p, hils_dtype in, hils_dtype out, const void *
     DeviceCtl ctl;
     hils_status st = device_ctl(&ctl);
     if (st != HILS_OK) return st;
-    if (p.N == 1) {
-        if (!force_decode_cuda_cores() && attend_decode_mma_supported(p, in))
-            return from_cuda(launch_attend_decode_mma(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
+    switch (attend_kind(p, in)) {
+    case AttKind::DecodeMma:
+        return from_cuda(launch_attend_decode_mma(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
+    case AttKind::DecodeCudaCores:
         return from_cuda(launch_attend_decode(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
+    default: return from_cuda(launch_attend_prefill(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
     }
-    return from_cuda(launch_attend_prefill(p, in, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s));
 }
 
 // The problem the chunk attention sees under a window of wc chunks: k + wc - 1 past slots per query.
@@ -256,6 +288,37 @@ hils_status hils_validate(const hils_problem *p)
 {
     Dims d;
     return resolve(p, &d);
+}
+
+hils_status hils_describe(const hils_problem *p, char *buf, size_t len)
+{
+    if (!buf) return HILS_ERR_INVALID_ARG;
+    Dims d;
+    const hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    const hils_dtype in = p->in_dtype;
+    const char *sel = "cuda-cores";
+    switch (select_kind(d, in)) {
+    case SelKind::DecodeScan: sel = "decode-scan"; break;
+    case SelKind::Queries: sel = "tc-queries"; break;
+    case SelKind::Heads: sel = select_tc_resident(d) ? "tc-heads-resident" : "tc-heads"; break;
+    default: break;
+    }
+    const char *att = "cuda-cores";
+    switch (attend_kind(d, in)) {
+    case AttKind::DecodeMma: att = "decode-mma"; break;
+    case AttKind::DecodeCudaCores: att = "decode-cuda-cores"; break;
+    case AttKind::ChunkMajor: att = "chunk-major"; break;
+    case AttKind::Union: att = "union-tc"; break;
+    default: break;
+    }
+    const int n = snprintf(buf, len, "forward=%s select=%s attend=%s", forward_fused(d, in) ? "decode-fused" : "two-call",
+                           sel, att);
+    if (n < 0 || (size_t)n >= len) {
+        if (len) buf[0] = 0;
+        return HILS_ERR_INVALID_ARG;
+    }
+    return HILS_OK;
 }
 
 hils_status hils_score_select_workspace_size(const hils_problem *p, size_t *bytes)
@@ -343,7 +406,7 @@ hils_status hils_forward(const hils_problem *p, const void *Q, const void *K, co
     float *sel_score = reinterpret_cast<float *>(ws + sel_idx_bytes(d));
     void *scratch = ws + sel_idx_bytes(d) + sel_score_bytes(d);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (fused_decode_enabled() && !force_decode_cuda_cores() && decode_fused_supported(d, p->in_dtype)) {
+    if (forward_fused(d, p->in_dtype)) {
         DeviceCtl ctl;
         st = device_ctl(&ctl);
         if (st != HILS_OK) return st;

@@ -58,6 +58,7 @@ cudaError_t launch_attend_prefill_simt(const Dims &p, hils_dtype in, hils_dtype 
                                        const float *sel_score, void *O, cudaStream_t s);
 bool attend_tc_supported(const Dims &p, hils_dtype in);
 bool select_tc_supported(const Dims &p, hils_dtype in);
+bool select_tc_resident(const Dims &p);   // the heads kernel keeps every landmark tile in TMEM
 cudaError_t launch_select_prefill_tc(const Dims &p, const void *Q, const void *L, int32_t *sel_idx,
                                      float *sel_score, const DeviceCtl &ctl, cudaStream_t s);
 // Prefill selection with one product row per query (group score from the mean query): bf16, d = 128, k <= 32.

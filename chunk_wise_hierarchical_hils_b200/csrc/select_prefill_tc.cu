@@ -613,6 +613,16 @@ bool res_disabled()
     return v && strcmp(v, "0") == 0;
 }
 
+int max_tiles(const Dims &p) { return (int)(((long long)p.q_offset + p.N - 1) / p.C / kTile) + 1; }
+
+}  // namespace
+
+// Every tile of a CTA resident in TMEM (at most 8 tiles of 64 columns), register lists (k <= 16), and
+// two or more heads per group to split the columns.
+bool select_tc_resident(const Dims &p) { return p.k <= 16 && p.G >= 2 && max_tiles(p) <= 8 && !res_disabled(); }
+
+namespace {
+
 template <int G>
 cudaError_t launch_g(const Dims &p, const void *Q, const void *L, int32_t *sel_idx, float *sel_score,
                      const DeviceCtl &ctl, cudaStream_t s)
@@ -633,9 +643,8 @@ cudaError_t launch_g(const Dims &p, const void *Q, const void *L, int32_t *sel_i
     const int rk = p.k <= 16 ? 16 : 0;   // register list for k <= 16, shared-memory heap above
     size_t smem = make_layout(rk ? kQueue : p.k, nsl).total + 1024;
     dim3 grid((p.N + BQ - 1) / BQ, p.Hkv, p.B);
-    // every tile of a CTA resident in TMEM when they fit (at most 8 tiles of 64 columns)
-    const int n_tiles_max = (int)(((long long)p.q_offset + p.N - 1) / p.C / kTile) + 1;
-    const bool res = rk == 16 && G >= 2 && n_tiles_max <= 8 && !res_disabled();
+    const int n_tiles_max = max_tiles(p);
+    const bool res = select_tc_resident(p);
     uint32_t tcols = kTmemCols;
     if (res) {
         while (tcols < (uint32_t)n_tiles_max * kTile) tcols <<= 1;

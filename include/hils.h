@@ -74,7 +74,7 @@
 extern "C" {
 #endif
 
-#define HILS_VERSION 120    /* 1.2.0: adds the backward pass (1.1.0: window/bias selection and forward, landmarks) */
+#define HILS_VERSION 121    /* 1.2.1: adds hils_describe (1.2.0: the backward pass; 1.1.0: window/bias selection and forward, landmarks) */
 #define HILS_MAX_K 64       /* largest supported top-k */
 #define HILS_MAX_GROUP 16   /* largest supported H / Hkv */
 
@@ -110,6 +110,18 @@ HILS_API int hils_version(void);
 
 /* Check a problem description without launching anything. */
 HILS_API hils_status hils_validate(const hils_problem *p);
+
+/*
+ * The kernels the library would run for problem p with the current test controls, as text:
+ * "forward=<k> select=<k> attend=<k>", where forward is "decode-fused" (one cooperative kernel for
+ * single-token decode) or "two-call", select is one of "decode-scan", "tc-queries",
+ * "tc-heads-resident", "tc-heads", "cuda-cores", and attend is one of "decode-mma", "decode-cuda-cores",
+ * "chunk-major", "union-tc", "cuda-cores" (select and attend name what hils_score_select and
+ * hils_chunk_attend_fuse run).  Writes at most len bytes including the terminating zero into buf
+ * (host memory, owned by the caller); HILS_ERR_INVALID_ARG if buf is NULL or len is too small for the
+ * text (at most 80 bytes), the problem's own error if it is invalid.  Launches nothing.
+ */
+HILS_API hils_status hils_describe(const hils_problem *p, char *buf, size_t len);
 
 /* Workspace bytes each entry point needs for problem p (may be 0). */
 HILS_API hils_status hils_score_select_workspace_size(const hils_problem *p, size_t *bytes);

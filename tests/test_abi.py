@@ -22,7 +22,7 @@ def test_header_symbols_exported():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) <= set(hils.EXPORTS) | set(names)
-    assert hils.hils_version() == 120
+    assert hils.hils_version() == 121
 
 
 def test_struct_layout_matches_header():
@@ -192,4 +192,44 @@ def test_header_is_plain_c_and_links(tmp_path):
     subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
                            "-L", libdir, "-lhils", "-Wl,-rpath," + libdir, "-o", str(exe)])
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
-    assert out[0] == "120"
+    assert out[0] == "121"
+
+
+def _bf16(**kw):
+    p = prob(**kw)
+    p.in_dtype = hils.HILS_BF16
+    p.out_dtype = hils.HILS_BF16
+    return p
+
+
+@pytest.mark.parametrize("kw,env,want", [
+    # 8K prefill, k = 16: every landmark tile fits TMEM, the union kernel (visible / selected about 4)
+    (dict(B=4, H=32, Hkv=8, N=8192, T=8192, k=16), {}, "select=tc-heads-resident attend=union-tc"),
+    (dict(B=4, H=32, Hkv=8, N=8192, T=8192, k=16), {"HILS_SELECT_RESIDENT": "0"}, "select=tc-heads attend=union-tc"),
+    (dict(B=4, H=32, Hkv=8, N=8192, T=8192, k=16), {"HILS_PREFILL_ATTEND": "chunk"},
+     "select=tc-heads-resident attend=chunk-major"),
+    # 256K prefill, k = 32: the per-query selection (k > 16) and chunk-major attention (ratio about 62)
+    (dict(B=1, H=16, Hkv=4, N=262144, T=262144, k=32), {}, "select=tc-queries attend=chunk-major"),
+    (dict(B=1, H=16, Hkv=4, N=262144, T=262144, k=32), {"HILS_PREFILL_ATTEND": "union"},
+     "select=tc-queries attend=union-tc"),
+    # single-token decode (the fused kernel needs a device, so forward is not checked here)
+    (dict(B=16, H=32, Hkv=8, N=1, T=131072, q_offset=131071, k=32), {}, "select=decode-scan attend=decode-mma"),
+])
+def test_describe(kw, env, want, monkeypatch):
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    text = hils.hils_describe(_bf16(**kw))
+    assert text.startswith("forward=")
+    assert text.split(" ", 1)[1] == want, text
+
+
+def test_describe_float32_and_errors():
+    p = prob()
+    p.in_dtype = hils.HILS_F32
+    p.out_dtype = hils.HILS_F32
+    assert hils.hils_describe(p).endswith("select=cuda-cores attend=cuda-cores")
+    buf = ctypes.create_string_buffer(8)
+    lib = ctypes.CDLL(hils.LIB_PATH)
+    assert lib.hils_describe(ctypes.byref(prob()), buf, ctypes.c_size_t(8)) == hils.HILS_ERR_INVALID_ARG
+    assert lib.hils_describe(ctypes.byref(prob()), None, ctypes.c_size_t(64)) == hils.HILS_ERR_INVALID_ARG
+    assert lib.hils_describe(ctypes.byref(prob(N=0)), buf, ctypes.c_size_t(8)) == hils.HILS_ERR_INVALID_ARG
