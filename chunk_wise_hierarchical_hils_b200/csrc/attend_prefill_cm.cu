@@ -482,47 +482,122 @@ __device__ __forceinline__ void own_range(const Dims &p, int RQ, int r, int c, i
     hi = (int)min(min(z, (long long)(r + 1) * RQ), (long long)p.N);
 }
 
-// one block: exclusive scans of the list sizes (entry offsets) and of the tiles per list
-__global__ void __launch_bounds__(1024) cm_scan_kernel(Dims p, int RQ, int R, int Mq, int M, const int *__restrict__ cnt,
-                                                       int *__restrict__ eoff, int *__restrict__ fill,
-                                                       int *__restrict__ toff, int *__restrict__ n_tiles)
+// Exclusive scans of the list sizes (entry offsets) and of the tiles per list, in three launches: each
+// block of cm_scan_sums adds up its kScanSeg consecutive lists, cm_scan_top scans the block sums, and
+// cm_scan_out scans each segment again from its block's offset.  Lists are read in rounds of 1024
+// consecutive ones (coalesced), each round a block-wide scan.
+constexpr int kScanSeg = 4096;   // lists per block: 4 rounds of 1024
+
+__device__ __forceinline__ void list_size(const Dims &p, int RQ, int R, int Mq, int M, int m, const int *cnt,
+                                          long long &ne, long long &nt)
 {
-    __shared__ long long s_e[1024], s_t[1024];
-    const int tid = threadIdx.x;
-    const int per = (M + 1023) / 1024;
-    const int m0 = min(tid * per, M), m1 = min(m0 + per, M);
-    long long se = 0, st = 0;
-    for (int m = m0; m < m1; ++m) {
-        const int c = m % p.nL, r = (m / p.nL) % R;
-        int lo, hi;
-        own_range(p, RQ, r, c, lo, hi);
-        const int n_own = max(hi - lo, 0), n_ret = cnt[m];
-        se += n_ret;
-        st += (n_ret + Mq - 1) / Mq + (n_own + Mq - 1) / Mq;
+    ne = 0;
+    nt = 0;
+    if (m >= M) return;
+    const int c = m % p.nL, r = (m / p.nL) % R;
+    int lo, hi;
+    own_range(p, RQ, r, c, lo, hi);
+    const int n_own = max(hi - lo, 0), n_ret = cnt[m];
+    ne = n_ret;
+    nt = (n_ret + Mq - 1) / Mq + (n_own + Mq - 1) / Mq;
+}
+
+// exclusive block-wide scan of two values per thread (1024 threads); the block totals in ta, tb
+__device__ __forceinline__ void block_scan2(long long &a, long long &b, long long &ta, long long &tb)
+{
+    __shared__ long long wa[32], wb[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long xa = __shfl_up_sync(0xFFFFFFFFu, ia, o), xb = __shfl_up_sync(0xFFFFFFFFu, ib, o);
+        if (lane >= o) {
+            ia += xa;
+            ib += xb;
+        }
     }
-    s_e[tid] = se;
-    s_t[tid] = st;
+    if (lane == 31) {
+        wa[warp] = ia;
+        wb[warp] = ib;
+    }
     __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-        const long long ae = tid >= o ? s_e[tid - o] : 0, at = tid >= o ? s_t[tid - o] : 0;
-        __syncthreads();
-        s_e[tid] += ae;
-        s_t[tid] += at;
-        __syncthreads();
+    if (warp == 0) {
+        long long va = wa[lane], vb = wb[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long xa = __shfl_up_sync(0xFFFFFFFFu, va, o), xb = __shfl_up_sync(0xFFFFFFFFu, vb, o);
+            if (lane >= o) {
+                va += xa;
+                vb += xb;
+            }
+        }
+        wa[lane] = va;
+        wb[lane] = vb;
     }
-    long long e = s_e[tid] - se, t = s_t[tid] - st;
-    for (int m = m0; m < m1; ++m) {
-        const int c = m % p.nL, r = (m / p.nL) % R;
-        int lo, hi;
-        own_range(p, RQ, r, c, lo, hi);
-        const int n_own = max(hi - lo, 0), n_ret = cnt[m];
-        eoff[m] = (int)e;
-        fill[m] = (int)e;
-        toff[m] = (int)t;
-        e += n_ret;
-        t += (n_ret + Mq - 1) / Mq + (n_own + Mq - 1) / Mq;
+    __syncthreads();
+    const long long pa = warp ? wa[warp - 1] : 0, pb = warp ? wb[warp - 1] : 0;
+    ta = wa[31];
+    tb = wb[31];
+    a = pa + ia - a;
+    b = pb + ib - b;
+    __syncthreads();   // wa, wb are reused by the next call
+}
+
+__global__ void __launch_bounds__(1024) cm_scan_sums(Dims p, int RQ, int R, int Mq, int M, const int *__restrict__ cnt,
+                                                     long long *__restrict__ bsum)
+{
+    long long se = 0, st = 0;
+    for (int j = 0; j < kScanSeg / 1024; ++j) {
+        long long ne, nt;
+        list_size(p, RQ, R, Mq, M, blockIdx.x * kScanSeg + j * 1024 + threadIdx.x, cnt, ne, nt);
+        long long te, tt;
+        block_scan2(ne, nt, te, tt);
+        se += te;
+        st += tt;
     }
-    if (tid == 1023) *n_tiles = (int)s_t[1023];
+    if (threadIdx.x == 0) {
+        bsum[2 * blockIdx.x] = se;
+        bsum[2 * blockIdx.x + 1] = st;
+    }
+}
+
+__global__ void __launch_bounds__(1024) cm_scan_top(int nb, long long *__restrict__ bsum, int *__restrict__ n_tiles)
+{
+    long long ce = 0, ct = 0;
+    for (int base = 0; base < nb; base += 1024) {
+        const int i = base + threadIdx.x;
+        long long e = i < nb ? bsum[2 * i] : 0, t = i < nb ? bsum[2 * i + 1] : 0;
+        long long te, tt;
+        block_scan2(e, t, te, tt);
+        if (i < nb) {
+            bsum[2 * i] = ce + e;
+            bsum[2 * i + 1] = ct + t;
+        }
+        ce += te;
+        ct += tt;
+    }
+    if (threadIdx.x == 0) *n_tiles = (int)ct;
+}
+
+__global__ void __launch_bounds__(1024) cm_scan_out(Dims p, int RQ, int R, int Mq, int M, const int *__restrict__ cnt,
+                                                    const long long *__restrict__ bsum, int *__restrict__ eoff,
+                                                    int *__restrict__ fill, int *__restrict__ toff)
+{
+    long long ce = bsum[2 * blockIdx.x], ct = bsum[2 * blockIdx.x + 1];
+    for (int j = 0; j < kScanSeg / 1024; ++j) {
+        const int m = blockIdx.x * kScanSeg + j * 1024 + threadIdx.x;
+        long long ne, nt;
+        list_size(p, RQ, R, Mq, M, m, cnt, ne, nt);
+        long long te, tt;
+        block_scan2(ne, nt, te, tt);
+        if (m < M) {
+            eoff[m] = (int)(ce + ne);
+            fill[m] = (int)(ce + ne);
+            toff[m] = (int)(ct + nt);
+        }
+        ce += te;
+        ct += tt;
+    }
 }
 
 // tile descriptors of each list: its own-chunk tiles, then its retrieved tiles
@@ -620,6 +695,7 @@ __global__ void cm_finalize_kernel(Dims p, const float4 *__restrict__ acc, Tout 
 
 struct CmWs {
     int *cnt, *eoff, *fill, *toff, *n_tiles, *entries;
+    long long *bsum;
     float *lse, *ow, *ew, *acc;
     int4 *tiles;
     size_t total;
@@ -641,6 +717,7 @@ CmWs cm_ws(const Dims &p, hils_dtype out, void *ws)
     w.fill = reinterpret_cast<int *>(take((size_t)c.M * 4));
     w.toff = reinterpret_cast<int *>(take((size_t)c.M * 4));
     w.n_tiles = reinterpret_cast<int *>(take(4));
+    w.bsum = reinterpret_cast<long long *>(take((size_t)((c.M + kScanSeg - 1) / kScanSeg) * 16));
     w.lse = reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * 4));
     w.ow = reinterpret_cast<float *>(take((size_t)p.B * p.H * p.N * 4));
     w.entries = reinterpret_cast<int *>(take((size_t)p.B * p.Hkv * p.N * p.k * 4 + 4));
@@ -693,7 +770,10 @@ cudaError_t launch_attend_prefill_cm(const Dims &p, hils_dtype out, const void *
     if (e != cudaSuccess) return e;
     cm_count_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, s>>>(p, c.RQ, c.R, sel_idx, sel_score, w.cnt, w.lse,
                                                                      w.ow);
-    cm_scan_kernel<<<1, 1024, 0, s>>>(p, c.RQ, c.R, c.Mq, c.M, w.cnt, w.eoff, w.fill, w.toff, w.n_tiles);
+    const int nb = (c.M + kScanSeg - 1) / kScanSeg;
+    cm_scan_sums<<<nb, 1024, 0, s>>>(p, c.RQ, c.R, c.Mq, c.M, w.cnt, w.bsum);
+    cm_scan_top<<<1, 1024, 0, s>>>(nb, w.bsum, w.n_tiles);
+    cm_scan_out<<<nb, 1024, 0, s>>>(p, c.RQ, c.R, c.Mq, c.M, w.cnt, w.bsum, w.eoff, w.fill, w.toff);
     cm_tiles_kernel<<<(c.M + 255) / 256, 256, 0, s>>>(p, c.RQ, c.R, c.Mq, c.M, w.cnt, w.eoff, w.toff, w.tiles);
     cm_scatter_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, s>>>(p, c.RQ, c.R, sel_idx, sel_score, w.lse,
                                                                        w.fill, w.entries, w.ew);
