@@ -26,7 +26,7 @@ HILS_MAX_GROUP = 16
 
 EXPORTS = ("hils_status_string", "hils_version", "hils_validate", "hils_describe", "hils_score_select_workspace_size",
            "hils_chunk_attend_fuse_workspace_size", "hils_forward_workspace_size", "hils_score_select",
-           "hils_chunk_attend_fuse", "hils_forward", "hils_sync_status", "hils_set_wait_limit",
+           "hils_chunk_attend_fuse", "hils_forward", "hils_forward_host_workspace_size", "hils_forward_host", "hils_sync_status", "hils_set_wait_limit",
            "hils_decode_score_select_noalloc", "hils_debug_inject_stall", "hils_landmarks",
            "hils_score_select_window", "hils_forward_window_workspace_size", "hils_forward_window",
            "hils_backward")
@@ -66,6 +66,9 @@ def _load():
     lib.hils_score_select.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
     lib.hils_chunk_attend_fuse.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hils_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.hils_forward_host_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+    lib.hils_forward_host.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.hils_describe.argtypes = [P, ctypes.c_char_p, sz]
     lib.hils_sync_status.argtypes = [vp]
     lib.hils_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.hils_decode_score_select_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
@@ -175,6 +178,18 @@ def hils_forward(p, Q, K, V, L, O, workspace=None, stream=None):
     wp, wn = _ws(workspace)
     _check(_lib.hils_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(O), wp, wn,
                              _stream(stream)), "hils_forward")
+
+
+def hils_forward_host_workspace_size(p):
+    return _size(_lib.hils_forward_host_workspace_size, p)
+
+
+def hils_forward_host(p, Q, K, V, L, O, workspace=None, stream=None):
+    """hils_forward on host tensors (page-locked for overlapped copies): Q, K, V, L are read from and O is
+    written to host memory, with copies and compute of batch slices overlapped (see include/hils.h)."""
+    wp, wn = _ws(workspace)
+    _check(_lib.hils_forward_host(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(O), wp, wn,
+                                  _stream(stream)), "hils_forward_host")
 
 
 def hils_sync_status(stream=None):

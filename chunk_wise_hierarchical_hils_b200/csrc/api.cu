@@ -265,6 +265,99 @@ cudaError_t launch_attend_prefill(const Dims &p, hils_dtype in, hils_dtype out, 
 
 }  // namespace hils
 
+namespace hils {
+namespace {
+
+// ---- forward from host buffers -----------------------------------------------------------------------
+
+constexpr int kHostSlices = 8;   // slices a batch is cut into (fewer when it has fewer units)
+
+struct HostPlan {
+    hils_problem slice;                              // the problem of one slice
+    int slices;                                      // slices in the batch
+    size_t q_bytes, kv_bytes, l_bytes, o_bytes;      // one slice's bytes of Q, K (and V), L, O
+    size_t slot_bytes;                               // one device slot: Q, K, V, L, O, each 256-aligned
+    size_t fwd_ws;                                   // the slice forward's workspace
+};
+
+size_t dtype_bytes(hils_dtype t) { return t == HILS_F32 ? 4 : 2; }
+
+hils_status host_plan(const hils_problem *p, HostPlan *hp)
+{
+    Dims d;
+    hils_status st = resolve(p, &d);
+    if (st != HILS_OK) return st;
+    // slices of `per` consecutive (b, g) units, each a problem of its own: per divides Hkv (groups
+    // g0 .. g0 + per - 1 of one batch element) or is a multiple of Hkv (whole batch elements); the
+    // units of a slice are contiguous in every tensor, at offset (first unit) x (bytes per unit)
+    const long long units = (long long)d.B * d.Hkv;
+    const long long want = (units + kHostSlices - 1) / kHostSlices;
+    long long per = units;
+    for (long long c = want; c < units; ++c)
+        if ((c <= d.Hkv && d.Hkv % c == 0) || (c % d.Hkv == 0 && units % c == 0)) {
+            per = c;
+            break;
+        }
+    hils_problem s = *p;
+    if (per <= d.Hkv) {
+        s.B = 1;
+        s.Hkv = (int)per;
+        s.H = (int)per * d.G;
+    } else {
+        s.B = (int)(per / d.Hkv);
+    }
+    hp->slice = s;
+    hp->slices = (int)(units / per);
+    const size_t ei = dtype_bytes(p->in_dtype), eo = dtype_bytes(p->out_dtype);
+    hp->q_bytes = (size_t)per * d.G * d.N * d.d * ei;
+    hp->kv_bytes = (size_t)per * d.T * d.d * ei;
+    hp->l_bytes = (size_t)per * d.nL * d.d * ei;
+    hp->o_bytes = (size_t)per * d.G * d.N * d.d * eo;
+    hp->slot_bytes = align_up(hp->q_bytes, 256) + 2 * align_up(hp->kv_bytes, 256) + align_up(hp->l_bytes, 256) +
+                     align_up(hp->o_bytes, 256);
+    size_t fw = 0;
+    st = hils_forward_workspace_size(&s, &fw);
+    if (st != HILS_OK) return st;
+    hp->fwd_ws = align_up(fw, 256);
+    return HILS_OK;
+}
+
+// The internal copy streams and the events of the two slots, per device, created on first use.
+struct HostStreams {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, end = nullptr, in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+};
+
+std::mutex g_host_mu;   // held while a call enqueues: the events are re-recorded in call order
+
+hils_status host_streams(HostStreams **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HILS_ERR_CUDA;
+    static HostStreams hs[64];
+    if (dev < 0 || dev >= 64) return HILS_ERR_UNSUPPORTED;
+    HostStreams &h = hs[dev];
+    if (!h.in) {
+        bool ok = cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&h.start, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&h.end, cudaEventDisableTiming) == cudaSuccess;
+        for (int k = 0; k < 2 && ok; ++k)
+            ok = cudaEventCreateWithFlags(&h.in_done[k], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&h.comp_done[k], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&h.out_done[k], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            h = HostStreams();   // handles created before the failure stay with the process
+            return HILS_ERR_CUDA;
+        }
+    }
+    *out = &h;
+    return HILS_OK;
+}
+
+}  // namespace
+}  // namespace hils
+
 using namespace hils;
 
 extern "C" {
@@ -415,6 +508,71 @@ hils_status hils_forward(const hils_problem *p, const void *Q, const void *K, co
     st = do_select(d, p->in_dtype, Q, L, sel_idx, sel_score, scratch, s);
     if (st != HILS_OK) return st;
     return do_attend(d, p->in_dtype, p->out_dtype, Q, K, V, sel_idx, sel_score, O, scratch, s);
+}
+
+hils_status hils_forward_host_workspace_size(const hils_problem *p, size_t *bytes)
+{
+    if (!bytes) return HILS_ERR_INVALID_ARG;
+    HostPlan hp;
+    const hils_status st = host_plan(p, &hp);
+    if (st != HILS_OK) return st;
+    *bytes = 2 * hp.slot_bytes + hp.fwd_ws;
+    return HILS_OK;
+}
+
+hils_status hils_forward_host(const hils_problem *p, const void *Q, const void *K, const void *V, const void *L,
+                              void *O, void *workspace, size_t workspace_bytes, void *stream)
+{
+    HostPlan hp;
+    hils_status st = host_plan(p, &hp);
+    if (st != HILS_OK) return st;
+    if (!Q || !K || !V || !L || !O) return HILS_ERR_INVALID_ARG;
+    st = check_ws(workspace, workspace_bytes, 2 * hp.slot_bytes + hp.fwd_ws);
+    if (st != HILS_OK) return st;
+    std::lock_guard<std::mutex> lk(g_host_mu);
+    HostStreams *h = nullptr;
+    st = host_streams(&h);
+    if (st != HILS_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    void *fws = ws + 2 * hp.slot_bytes;
+    const char *qh = static_cast<const char *>(Q), *kh = static_cast<const char *>(K);
+    const char *vh = static_cast<const char *>(V), *lh = static_cast<const char *>(L);
+    char *oh = static_cast<char *>(O);
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    if (!ok(cudaEventRecord(h->start, s)) || !ok(cudaStreamWaitEvent(h->in, h->start, 0)) ||
+        !ok(cudaStreamWaitEvent(h->out, h->start, 0)))
+        return HILS_ERR_CUDA;
+    for (int i = 0; i < hp.slices; ++i) {
+        const int k = i & 1;
+        char *dq = ws + (size_t)k * hp.slot_bytes;
+        char *dk = dq + align_up(hp.q_bytes, 256);
+        char *dv = dk + align_up(hp.kv_bytes, 256);
+        char *dl = dv + align_up(hp.kv_bytes, 256);
+        char *dout = dl + align_up(hp.l_bytes, 256);
+        // copies in: after slice i - 2's forward has read this slot
+        if (i >= 2 && !ok(cudaStreamWaitEvent(h->in, h->comp_done[k], 0))) return HILS_ERR_CUDA;
+        if (!ok(cudaMemcpyAsync(dq, qh + (size_t)i * hp.q_bytes, hp.q_bytes, cudaMemcpyHostToDevice, h->in)) ||
+            !ok(cudaMemcpyAsync(dk, kh + (size_t)i * hp.kv_bytes, hp.kv_bytes, cudaMemcpyHostToDevice, h->in)) ||
+            !ok(cudaMemcpyAsync(dv, vh + (size_t)i * hp.kv_bytes, hp.kv_bytes, cudaMemcpyHostToDevice, h->in)) ||
+            !ok(cudaMemcpyAsync(dl, lh + (size_t)i * hp.l_bytes, hp.l_bytes, cudaMemcpyHostToDevice, h->in)) ||
+            !ok(cudaEventRecord(h->in_done[k], h->in)))
+            return HILS_ERR_CUDA;
+        // the forward: after its inputs landed and slice i - 2's output left this slot
+        if (!ok(cudaStreamWaitEvent(s, h->in_done[k], 0))) return HILS_ERR_CUDA;
+        if (i >= 2 && !ok(cudaStreamWaitEvent(s, h->out_done[k], 0))) return HILS_ERR_CUDA;
+        st = hils_forward(&hp.slice, dq, dk, dv, dl, dout, fws, hp.fwd_ws, stream);
+        if (st != HILS_OK) return st;
+        if (!ok(cudaEventRecord(h->comp_done[k], s))) return HILS_ERR_CUDA;
+        // copy out
+        if (!ok(cudaStreamWaitEvent(h->out, h->comp_done[k], 0)) ||
+            !ok(cudaMemcpyAsync(oh + (size_t)i * hp.o_bytes, dout, hp.o_bytes, cudaMemcpyDeviceToHost, h->out)) ||
+            !ok(cudaEventRecord(h->out_done[k], h->out)))
+            return HILS_ERR_CUDA;
+    }
+    // the caller's stream continues once the last output copy is done (the copy stream runs in order)
+    if (!ok(cudaEventRecord(h->end, h->out)) || !ok(cudaStreamWaitEvent(s, h->end, 0))) return HILS_ERR_CUDA;
+    return HILS_OK;
 }
 
 hils_status hils_score_select_window(const hils_problem *p, int window_chunks, const float *bias, const void *Q,

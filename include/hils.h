@@ -74,7 +74,7 @@
 extern "C" {
 #endif
 
-#define HILS_VERSION 121    /* 1.2.1: adds hils_describe (1.2.0: the backward pass; 1.1.0: window/bias selection and forward, landmarks) */
+#define HILS_VERSION 122    /* 1.2.2: adds hils_forward_host (1.2.1: hils_describe; 1.2.0: the backward pass; 1.1.0: window/bias selection and forward, landmarks) */
 #define HILS_MAX_K 64       /* largest supported top-k */
 #define HILS_MAX_GROUP 16   /* largest supported H / Hkv */
 
@@ -169,6 +169,27 @@ HILS_API hils_status hils_chunk_attend_fuse(const hils_problem *p, const void *Q
 HILS_API hils_status hils_forward(const hils_problem *p, const void *Q, const void *K, const void *V,
                          const void *L, void *O, void *workspace, size_t workspace_bytes,
                          void *stream);
+
+/*
+ * hils_forward on HOST buffers: Q, K, V, L are read from and O is written to host memory (page-locked
+ * for the copies to overlap; pageable memory works but serialises them).  The (batch, kv-group) pairs
+ * are independent problems [Sec. 4, Architecture: a group's heads share its selection, groups share
+ * nothing], so the batch is cut into about eight slices of consecutive pairs; each slice's inputs are
+ * copied into one of two device slots on an internal stream, its forward runs on `stream`, and its
+ * output is copied back on a second internal stream, so copies in, compute and copies out of
+ * different slices overlap.  Layouts as for hils_forward.  The workspace (device memory, owned by
+ * the caller, 16-byte aligned) holds the two slots and the slice forward's workspace; its size comes
+ * from hils_forward_host_workspace_size.  Stream-ordered: the copies start after the work already
+ * queued on `stream`, and work queued on `stream` afterwards (a synchronisation, an event) sees O on
+ * the host.  Calls from several host threads are serialised while they enqueue.  Errors: those of
+ * hils_forward, HILS_ERR_INVALID_ARG for a NULL host pointer, HILS_ERR_WORKSPACE for a short
+ * workspace, HILS_ERR_CUDA if a copy or the internal streams fail (work already queued may then be
+ * partly done).  Single-token decode normally keeps its caches on the device and calls hils_forward.
+ */
+HILS_API hils_status hils_forward_host_workspace_size(const hils_problem *p, size_t *bytes);
+HILS_API hils_status hils_forward_host(const hils_problem *p, const void *Q, const void *K, const void *V,
+                              const void *L, void *O, void *workspace, size_t workspace_bytes,
+                              void *stream);
 
 /*
  * Selection with a local window and a per-chunk bias (Sec. 2 Preliminary and

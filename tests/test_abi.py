@@ -22,7 +22,7 @@ def test_header_symbols_exported():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) <= set(hils.EXPORTS) | set(names)
-    assert hils.hils_version() == 121
+    assert hils.hils_version() == 122
 
 
 def test_struct_layout_matches_header():
@@ -192,7 +192,7 @@ def test_header_is_plain_c_and_links(tmp_path):
     subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
                            "-L", libdir, "-lhils", "-Wl,-rpath," + libdir, "-o", str(exe)])
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
-    assert out[0] == "121"
+    assert out[0] == "122"
 
 
 def _bf16(**kw):
@@ -233,3 +233,50 @@ def test_describe_float32_and_errors():
     assert lib.hils_describe(ctypes.byref(prob()), buf, ctypes.c_size_t(8)) == hils.HILS_ERR_INVALID_ARG
     assert lib.hils_describe(ctypes.byref(prob()), None, ctypes.c_size_t(64)) == hils.HILS_ERR_INVALID_ARG
     assert lib.hils_describe(ctypes.byref(prob(N=0)), buf, ctypes.c_size_t(8)) == hils.HILS_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,slices", [
+    (dict(B=4, H=32, Hkv=8, N=8192, T=8192, k=16), 8),     # 32 (b, g) units, 4 per slice
+    (dict(B=1, H=16, Hkv=4, N=4096, T=4096, k=8), 4),      # one group per slice
+    (dict(B=3, H=8, Hkv=2, N=256, T=256, k=4), 6),
+    (dict(B=16, H=32, Hkv=8, N=1, T=4096, q_offset=4095, k=8), 8),   # whole batch elements per slice
+])
+def test_forward_host_workspace(kw, slices):
+    """Two device slots of one slice's Q, K, V, L, O plus the slice forward's workspace."""
+    p = _bf16(**kw)
+    need = hils.hils_forward_host_workspace_size(p)
+    b, hkv = kw["B"], kw["Hkv"]
+    per = b * hkv // slices
+    g = kw["H"] // hkv
+    nl = -(-kw["T"] // 64)
+    slot = sum(-(-x // 256) * 256 for x in (per * g * kw["N"] * 128 * 2, per * kw["T"] * 128 * 2,
+                                            per * kw["T"] * 128 * 2, per * nl * 128 * 2, per * g * kw["N"] * 128 * 2))
+    q = _bf16(**dict(kw, B=per // hkv if per >= hkv else 1, Hkv=min(per, hkv), H=min(per, hkv) * g))
+    fwd = -(-hils.hils_forward_workspace_size(q) // 256) * 256
+    assert need == 2 * slot + fwd
+
+
+def test_forward_host_errors():
+    """Host-side checks before any copy: NULL host pointers, a short workspace, a bad problem."""
+    lib = ctypes.CDLL(hils.LIB_PATH)
+    p = _bf16()
+    need = hils.hils_forward_host_workspace_size(p)
+    fake = ctypes.c_void_p(4096)   # never dereferenced: the call returns before any copy
+    args = [fake] * 5
+    assert lib.hils_forward_host(ctypes.byref(p), None, *args[1:], fake, ctypes.c_size_t(need), None) == \
+        hils.HILS_ERR_INVALID_ARG
+    assert lib.hils_forward_host(ctypes.byref(p), *args, fake, ctypes.c_size_t(need - 16), None) == \
+        hils.HILS_ERR_WORKSPACE
+    assert lib.hils_forward_host(ctypes.byref(prob(N=0)), *args, fake, ctypes.c_size_t(need), None) == \
+        hils.HILS_ERR_INVALID_ARG
+    assert lib.hils_forward_host_workspace_size(ctypes.byref(p), None) == hils.HILS_ERR_INVALID_ARG
+
+
+def test_every_export_has_argument_types():
+    """Each exported entry point taking arguments has ctypes argument types (an untyped pointer argument
+    would be passed as a 32-bit int)."""
+    src = open(os.path.join(ROOT, "include", "hils.h")).read()
+    for n in declared_symbols():
+        m = re.search(r"\b" + n + r"\s*\(([^)]*)\)", src)
+        if m and m.group(1).strip() not in ("", "void"):
+            assert getattr(hils._lib, n).argtypes is not None, n
