@@ -38,7 +38,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;          // warp 0 loads and issues, warp 1 holds TMEM, warps 2-9 rank
 constexpr int kRows = 128;               // queries per CTA (MMA M)
 constexpr int kD = 128;
 constexpr int kTile = 128;               // landmarks per tile (MMA N)
@@ -65,7 +65,7 @@ __host__ __device__ inline Layout make_layout(int k, int wc = 1)
     L.bar = L.l + kNSL * kTileBytes;
     L.misc = L.bar + 16 * 8;
     L.queue = L.misc + 16;
-    L.selc = L.queue + 8u * kQueue * kRows;
+    L.selc = L.queue + 2u * 8u * kQueue * kRows;   // one queue per (row, column half)
     L.total = L.selc + 4u * (uint32_t)(k + wc) * kRows;
     return L;
 }
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(S_FULL(s), 1);
-            mbar_init(S_FREE(s), 4);
+            mbar_init(S_FREE(s), 8);
         }
         mbar_init(MMA_DONE, 1);
         fence_mbar_init();
@@ -268,14 +268,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp >= 2) {
-        const int qq = warp & 3;
+        // two warps per quarter of the rows (TMEM lanes 32 qq ..): warps 2-5 rank the first two 32-column
+        // parts of every tile, warps 6-9 the last two; their lists merge after the scan
+        const int qq = warp & 3, ch = (warp - 2) >> 2;
         const int r = 32 * qq + lane;
         const bool valid = r < nq;
         const long long pos = (long long)p.q_offset + q0 + r;
         const int ci = (int)(pos / p.C);
         const int c_lim = ci - wc + 1;   // candidates c < c_lim
         const uint32_t trow = tmem + ((uint32_t)(32 * qq) << 16);
-        uint64_t *hk = queue + r;
+        uint64_t *hk = queue + (size_t)ch * kQueue * kRows + r;
         uint64_t top[RK];
 #pragma unroll
         for (int i = 0; i < RK; ++i) top[i] = 0ull;
@@ -289,11 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
 #pragma unroll 1
-            for (int part = 0; part < kTile / 32; ++part) {
+            for (int part = 2 * ch; part < 2 * ch + 2; ++part) {
                 uint32_t sv[32];
                 tmem_ld32(trow + (uint32_t)(t & 1) * kTile + 32u * part, sv);
                 tmem_wait_ld();
-                if (part == kTile / 32 - 1) {
+                if (part == 2 * ch + 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(S_FREE(t & 1));
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // the queue is full after kQueue candidates: insert them before going on.  The
                         // very first time the list is still empty: the queued keys are copied in and
                         // sorted by a network instead of inserted one by one.
-                        if (t == 0 && part == 0) {
+                        if (t == 0 && part == 2 * ch) {
 #pragma unroll
                             for (int i = 0; i < RK; ++i) top[i] = (i < kQueue && i < qn) ? hk[i * kRows] : 0ull;
                             list_sort_desc<RK>(top);
@@ -341,9 +343,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (!ok) *abort_flag = 1;
+        // the two column halves' lists of each row into one, kept by the first warp of the pair: the
+        // second one's list goes through the queue space, free once every epilogue warp has finished
+        // its scan (named barrier 2: the eight epilogue warps)
+        uint64_t *xl = queue + r;   // [RK][kRows]
+        asm volatile("bar.sync 2, 256;" ::: "memory");
+        if (ch == 1) {
+#pragma unroll
+            for (int i = 0; i < RK; ++i) xl[i * kRows] = top[i];
+        }
+        asm volatile("bar.sync 2, 256;" ::: "memory");
+        if (ch == 0) {
+            // both lists descending: the elementwise maximum against the other list reversed is bitonic
+            // and holds the RK largest; a merge network sorts it
+#pragma unroll
+            for (int i = 0; i < RK; ++i) {
+                const uint64_t x = xl[(RK - 1 - i) * kRows];
+                top[i] = top[i] > x ? top[i] : x;
+            }
+#pragma unroll
+            for (int stride = RK / 2; stride > 0; stride >>= 1)
+#pragma unroll
+                for (int i = 0; i < RK; ++i)
+                    if ((i & stride) == 0) {
+                        const uint64_t a = top[i], c2 = top[i + stride];
+                        top[i] = a > c2 ? a : c2;
+                        top[i + stride] = a > c2 ? c2 : a;
+                    }
+        }
         // the selection: chunk indices in rank order (k < RK: the list's first k keys), then the window's
         // past chunks ascending, own chunk last
-        if (valid) {
+        if (valid && ch == 0) {
             const size_t row_g = (((size_t)b * p.Hkv + g) * p.N) + q0 + r;
 #pragma unroll
             for (int j = 0; j < RK; ++j) {
