@@ -136,6 +136,13 @@ int forced_select_kernel()
     return 0;
 }
 
+// Test control: HILS_PREFILL_KERNEL=persistent runs the union attention as a persistent kernel.
+bool persistent_union()
+{
+    const char *v = getenv("HILS_PREFILL_KERNEL");
+    return v && strcmp(v, "persistent") == 0;
+}
+
 // Test control: HILS_DECODE_FUSED=0 keeps hils_forward's single-token decode on the two kernels
 // (selection, then attention) instead of the fused cooperative kernel.
 bool fused_decode_enabled()
@@ -258,6 +265,8 @@ cudaError_t launch_attend_prefill(const Dims &p, hils_dtype in, hils_dtype out, 
 {
     if (use_chunk_major(p, in))
         return launch_attend_prefill_cm(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s);
+    if (!force_cuda_cores() && persistent_union() && attend_tc_persistent_supported(p, in))
+        return launch_attend_prefill_tc_persistent(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s);
     if (!force_cuda_cores() && attend_tc_supported(p, in))
         return launch_attend_prefill_tc(p, out, Q, K, V, sel_idx, sel_score, O, ws, ctl, s);
     return launch_attend_prefill_simt(p, in, out, Q, K, V, sel_idx, sel_score, O, s);

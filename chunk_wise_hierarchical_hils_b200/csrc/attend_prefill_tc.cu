@@ -732,6 +732,11 @@ size_t attend_tc_ws_bytes(const Dims &p)
 
 // V converted to f16 into the workspace (the first v16_bytes), and one flag per (b, kv-head) slice
 // that holds a value f16 cannot represent (the next B * Hkv words); the flags are cleared first.
+const unsigned int *attend_tc_wide_flags(const Dims &p, const void *ws)
+{
+    return reinterpret_cast<const unsigned int *>(static_cast<const char *>(ws) + v16_bytes(p));
+}
+
 cudaError_t launch_v_to_f16(const Dims &p, const void *V, void *ws, cudaStream_t s)
 {
     const size_t n16 = (size_t)p.B * p.Hkv * p.T * kD / 8;

@@ -71,6 +71,12 @@ size_t attend_tc_ws_bytes(const Dims &p);   // V as f16 + one flag word per (b, 
 // V (bf16) converted to f16 at the start of ws, and per (b, kv-head) a flag set when a value's magnitude
 // is 65536 or more (the slice then takes a bf16 value product with V as given).
 cudaError_t launch_v_to_f16(const Dims &p, const void *V, void *ws, cudaStream_t s);
+const unsigned int *attend_tc_wide_flags(const Dims &p, const void *ws);   // launch_v_to_f16's flag words in ws
+// The same attention as a persistent kernel (one CTA per SM walking query tiles); same workspace.
+bool attend_tc_persistent_supported(const Dims &p, hils_dtype in);
+cudaError_t launch_attend_prefill_tc_persistent(const Dims &p, hils_dtype out, const void *Q, const void *K,
+                                                const void *V, const int32_t *sel_idx, const float *sel_score,
+                                                void *O, void *ws, const DeviceCtl &ctl, cudaStream_t s);
 // Chunk-major prefill attention (selection inverted per chunk, tiles of gathered query rows, partial
 // outputs added in L2): bf16, d = 128, C = 64.
 bool attend_cm_supported(const Dims &p, hils_dtype in);

@@ -80,6 +80,16 @@ def test_chunk_major_attention_too(w, monkeypatch):
     _check(st)
 
 
+@pytest.mark.parametrize("w", [CASES[1], CASES[3], CASES[5], CASES[6], CASES[7], CASES[8], CASES[10], CASES[11],
+                               CASES[12]], ids=lambda w: w.name)
+def test_persistent_union_attention(w, monkeypatch):
+    """The union attention as a persistent kernel (one CTA per SM walking query tiles, the next tile's
+    chunk union built while the current tile's last products run), forced on the tensor-core cases."""
+    monkeypatch.setenv("HILS_PREFILL_KERNEL", "persistent")
+    st, _ = parity.run_small(w)
+    _check(st)
+
+
 @pytest.mark.parametrize("attend", ["union", "chunk"])
 def test_both_prefill_attentions_with_bf16_output(attend, monkeypatch):
     monkeypatch.setenv("HILS_PREFILL_ATTEND", attend)
@@ -197,7 +207,7 @@ def test_exact_ties_lowest_index():
     _check(st)
 
 
-@pytest.mark.parametrize("attend", ["union", "chunk"])
+@pytest.mark.parametrize("attend", ["union", "chunk", "persistent"])
 def test_large_and_tiny_values(attend, monkeypatch):
     """V entries far outside N(0,1): +-1e5 (beyond f16's range), +-3e4 (inside it) and +-1e-6 (f16
     subnormals), planted in a few chunks of some (b, kv-head) slices, so that most rows of the blocks
@@ -211,7 +221,10 @@ def test_large_and_tiny_values(attend, monkeypatch):
     |v| <= 8 only keep the usual 1e-2; rows that attend to a planted large value get 2^-8 times it."""
     from synth import workloads as W
     from synth.philox import f64_to_f32, f32_to_bf16_bits, bf16_bits_to_f64
-    monkeypatch.setenv("HILS_PREFILL_ATTEND", attend)
+    if attend == "persistent":
+        monkeypatch.setenv("HILS_PREFILL_KERNEL", "persistent")
+    else:
+        monkeypatch.setenv("HILS_PREFILL_ATTEND", attend)
     w = wl("wide_values", B=2, H=8, Hkv=2, N=1024, T=1024, k=4, seed=140)
     inp = W.full_inputs(w)
     arr = {k: v[0].copy() for k, v in inp.items()}
