@@ -107,15 +107,24 @@ def decode_fused_applies(w, n_sm=148):
     return -(-n_past // 4096) <= S
 
 
-def kernels_per_step(w):
-    """Kernels of this library one step launches (the input generator and copies are not counted)."""
+def kernels_per_step(w, plan=None):
+    """Kernels of this library one step launches (the input generator, copies and memsets are not
+    counted), from the library's own description of the kernels it runs for the problem."""
+    if plan is None:
+        import chunk_wise_hierarchical_hils_b200 as hils
+        dt = {"f32": hils.HILS_F32, "bf16": hils.HILS_BF16}[w.dtype]
+        plan = hils.hils_describe(hils.problem(w.B, w.H, w.Hkv, w.N, w.T, w.d, w.C, w.k, w.q_offset, dt, dt))
     if w.N == 1:
-        if decode_fused_applies(w):
-            return 1      # the fused decode kernel (plus a memset of its tickets)
-        return 2          # decode landmark scan + top-k, decode attention (plus two ticket memsets)
-    # prefill: selection; [V to f16 (plus a memset of the slice flags) +] attention
-    tc = w.dtype == "bf16" and w.d == 128 and w.G in (1, 2, 4, 8, 16) and os.environ.get("HILS_PREFILL_KERNEL") != "simt"
-    return 3 if (tc and w.C == 64) else 2
+        return 1 if "forward=decode-fused" in plan else 2   # fused kernel; or scan + top-k, attention
+    n = 1                                                    # the selection
+    if "attend=chunk-major" in plan:
+        # V to f16; count, three scan launches, tile table, scatter; attention; finalize
+        n += 9
+    elif "attend=union-tc" in plan:
+        n += 2                                               # V to f16; attention
+    else:
+        n += 1                                               # CUDA-core attention
+    return n
 
 
 def kernel_traffic(kernel, workload):
@@ -604,7 +613,7 @@ def measure_forward(args, w, ws, rank, local, steps=None):
                    "inputs_copied": e2e_names,
                    "call": "hils_forward_host (pinned host buffers)" if w.N > 1 else
                            "query token H2D, hils_forward on the resident caches, output D2H"},
-           "gpu_launches": kernels_per_step(w) * steps, "clocks": clocks}
+           "gpu_launches": kernels_per_step(w, plan) * steps, "clocks": clocks}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, cores, desc, _ = cpu_baseline(w, args.cpu_blocks)
         rec["cpu_baseline"] = {"value": v, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc}
@@ -785,7 +794,7 @@ def run_window(args, w):
     pk, pk_kind = peaks()
     wk = w.with_(k=w.k + wc - 1)
     fl = attention_flops(wk)
-    peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    peak, peak_kind = tensor_peak(pk, pk_kind, ms * 1e-3 * args.steps)
     achieved = fl / (ms * 1e-3) / 1e12
     units = w.B * w.N if w.N > 1 else w.B
     line = {"metric": "HiLS fwd with a %d-chunk local window and chunk bias, tokens/s at 1 B200" % wc,
@@ -795,7 +804,7 @@ def run_window(args, w):
             "config": dict(config_of(w, ws), part="window", window_chunks=wc),
             "roofline": {"bound": "tensor", "kernel": "whole step (selection + attention)", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                         "peak_kind": pk_kind + " bf16 sustained", "algorithmic_flops_per_launch": fl},
+                         "peak_kind": peak_kind, "algorithmic_flops_per_launch": fl},
             "gpu_launches": kernels_per_step(w) * args.steps, "clocks": clocks,
             "timing": "CUDA-graph replays of one hils_forward_window call, CUDA events on the replay stream"}
     if rank == 0:
