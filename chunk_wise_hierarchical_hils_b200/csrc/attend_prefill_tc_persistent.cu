@@ -23,8 +23,8 @@
 //                        shared memory) on two chunks at once (N = 128, the
 //                        tensor core's efficient width) into one of two TMEM
 //                        S buffers;
-//   warp 3 (one thread)  tcgen05.mma issue of O += P V (f16, P from TMEM, V
-//                        from shared memory) on the same pairs (K = 128 keys);
+//   warp 3 (one thread)  tcgen05.mma issue of O += P V (f16 or bf16, P from
+//                        TMEM, V from shared memory) on the same pairs (K = 128 keys);
 //                        two issuers keep the tensor core busy while either
 //                        one waits;
 //   warps 4..15          three groups of four warps, one thread per row; group
@@ -32,12 +32,17 @@
 //                        the S buffer at once), takes the softmax over the
 //                        chunk's visible keys, scales it by the row's fusion
 //                        weight (0 if the row's query did not select the chunk)
-//                        and writes P (f16) to its half of a TMEM P buffer.  At
+//                        and writes P (16-bit) to its half of a TMEM P buffer.  At
 //                        the end the groups read O from TMEM and store it.
 // Because each chunk's softmax is normalised on its own and the fusion weights
 // are known before the loop, P already carries w_c / l_c and the accumulator
-// needs no rescaling between chunks.  V is read as f16 (converted once per call
-// by a streaming pass), so P can be kept in f16 with a 2^-11 rounding.
+// needs no rescaling between chunks.
+//
+// Value product precision, as in the per-tile kernel: a streaming pass converts
+// V to f16 once per call and flags every (b, kv-head) slice holding a value of
+// magnitude >= 65536; a tile of an unflagged slice reads the f16 copy and rounds
+// P to f16 (relative 2^-11), a tile of a flagged slice reads V as given and
+// rounds P to bf16, so V always enters the product exactly.
 //
 // Every barrier wait is bounded: on expiry the CTA records HILS_ERR_TIMEOUT,
 // stops issuing work, waits (with its own bound) for the copies and MMAs it has
