@@ -102,3 +102,29 @@ def test_reference_arm_other_ranks_exit_quietly():
                        timeout=600, cwd=ROOT, env=env)
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+
+
+@pytest.mark.parametrize("plan,n", [
+    ("forward=two-call select=tc-heads-resident attend=union-tc", 3),
+    ("forward=two-call select=tc-queries attend=chunk-major", 10),
+    ("forward=two-call select=cuda-cores attend=cuda-cores", 2),
+    ("forward=decode-fused select=decode-scan attend=decode-mma", 1),
+    ("forward=two-call select=decode-scan attend=decode-mma", 2),
+])
+def test_launches_per_step_follow_the_plan(plan, n):
+    """The JSON line's gpu_launches counts the library's kernels from the plan hils_describe reports."""
+    b = load_bench()
+    w = WORKLOADS["decode_128k"] if "decode" in plan else WORKLOADS["prefill_8k"]
+    assert b.kernels_per_step(w, plan) == n
+
+
+def test_traffic_entries_name_their_workload():
+    """Every traffic.json entry is keyed kernel@workload, names a bench workload and lists the sources
+    whose hashes gate it."""
+    data = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for k, rec in data.items():
+        if k.startswith("_"):
+            continue
+        kernel, wl = k.split("@")
+        assert rec["workload"] == wl and wl in WORKLOADS
+        assert rec["sources"] and rec["dram_bytes_per_launch"] > 0
